@@ -1,0 +1,268 @@
+"""Pins for the fp64 oracle against things other than itself: closed forms, brute force on
+tiny inputs, hand-derived golden routing cases and library routines (torch SDPA)."""
+import itertools
+import json
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle as O
+from free_adaptive_block_b200 import workloads as W
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden")
+
+
+# ------------------------------------------------------------------ geometry / pool
+def test_block_geometry_480p_real_size_mix():
+    # 30 x 52 latent frames cut into 8 x 16 blocks: per frame 4 x 4 blocks with
+    # real sizes 9 x 128, 3 x 96 (H edge, 6 rows), 3 x 32 (W edge, 4 cols), 1 x 24.
+    g = O.block_geometry(21, 30, 52, 1, 8, 16)
+    assert g.nB == 21 * 16
+    assert g.real_count.sum() == 21 * 30 * 52
+    per_frame = sorted(g.real_count[:16].tolist())
+    assert per_frame == sorted([128] * 9 + [96] * 3 + [32] * 3 + [24])
+    # a token belongs to the block of its (t // bt, y // bh, x // bw)
+    n = (5 * 30 + 29) * 52 + 50
+    assert g.block_of_token[n] == (5 * 4 + 3) * 4 + 3
+    assert n in set(g.tokens_of_block[(5 * 4 + 3) * 4 + 3].tolist())
+
+
+def test_block_geometry_720p_and_t_edge():
+    g = O.block_geometry(21, 45, 80, 1, 8, 16)
+    assert g.nB == 21 * 6 * 5
+    assert sorted(set(g.real_count.tolist())) == [80, 128]
+    g2 = O.block_geometry(5, 12, 20, 2, 4, 8)       # T, H, W all ragged
+    assert g2.nB == 3 * 3 * 3
+    assert g2.real_count.sum() == 5 * 12 * 20
+    assert g2.real_count.min() == 1 * 4 * 4          # the corner on the T and W edges
+
+
+def test_pool_closed_form_when_blocks_divide_the_latent():
+    rng = np.random.default_rng(0)
+    T, Hs, Ws, bt, bh, bw, d = 4, 8, 8, 2, 4, 4, 6
+    X = rng.standard_normal((2, 3, T * Hs * Ws, d))
+    g = O.block_geometry(T, Hs, Ws, bt, bh, bw)
+    got = O.pool(X, g)
+    r = X.reshape(2, 3, T // bt, bt, Hs // bh, bh, Ws // bw, bw, d).mean(axis=(3, 5, 7))
+    want = r.reshape(2, 3, -1, d)
+    np.testing.assert_allclose(got, want, rtol=0, atol=1e-13)
+
+
+def test_pool_ragged_against_explicit_loops():
+    rng = np.random.default_rng(1)
+    T, Hs, Ws, bt, bh, bw, d = 3, 5, 7, 2, 2, 3, 4
+    X = rng.standard_normal((1, 2, T * Hs * Ws, d))
+    g = O.block_geometry(T, Hs, Ws, bt, bh, bw)
+    got = O.pool(X, g)
+    nBy, nBx = -(-Hs // bh), -(-Ws // bw)
+    for h in range(2):
+        for tb in range(-(-T // bt)):
+            for yb in range(nBy):
+                for xb in range(nBx):
+                    acc, n = np.zeros(d), 0
+                    for t in range(tb * bt, min(T, tb * bt + bt)):
+                        for y in range(yb * bh, min(Hs, yb * bh + bh)):
+                            for x in range(xb * bw, min(Ws, xb * bw + bw)):
+                                acc += X[0, h, (t * Hs + y) * Ws + x]
+                                n += 1
+                    j = (tb * nBy + yb) * nBx + xb
+                    np.testing.assert_allclose(got[0, h, j], acc / n, atol=1e-14)
+
+
+# ------------------------------------------------------------------ routing
+def _route_row(scores, own, p, k):
+    """Route one hand-made row: Kp = identity and Qp rows = ln(scores) make the routing
+    logits equal ln(scores), so the routing scores are the given ones."""
+    s = np.asarray(scores, dtype=np.float64)
+    nB = s.size
+    logits = np.log(np.maximum(s, 1e-300))
+    Qp = np.tile(logits, (nB, 1))[None, None]
+    Kp = np.eye(nB)[None, None]
+    r = O.route(Qp, Kp, p, k, 1.0)
+    np.testing.assert_allclose(r.scores[0, 0, own], s / s.sum(), rtol=1e-12, atol=1e-300)
+    return r.keep[0, 0, own], int(r.counts[0, 0, own])
+
+
+def test_route_golden_hand_cases():
+    cases = json.load(open(os.path.join(GOLDEN, "route_cases.json")))["cases"]
+    for c in cases:
+        keep, count = _route_row(c["scores"], c["own"], c["p"], c["k"])
+        assert keep.astype(int).tolist() == c["keep"], c["name"]
+        assert count == c["count"], c["name"]
+
+
+def test_route_against_brute_force_on_tiny_config():
+    w = W.TINY
+    x = W.generate(w)
+    g = O.block_geometry(w.T, w.Hs, w.Ws, w.bt, w.bh, w.bw)
+    Qp, Kp = O.pool(x["q"], g), O.pool(x["k"], g)
+    scale = 1.0 / math.sqrt(w.d)
+    for p, k in itertools.product([0.0, 0.3, 0.6, 0.9, 0.97, 1.0], [0, 1, 2, 5, 8, 11]):
+        r = O.route(Qp, Kp, p, k, scale)
+        for h in range(w.H):
+            for qb in range(g.nB):
+                s_row = r.scores[0, h, qb]
+                want = O.brute_force_route_row(s_row, qb, p, k)
+                assert (r.keep[0, h, qb] == want).all(), (p, k, h, qb)
+                assert r.counts[0, h, qb] == want.sum()
+
+
+@pytest.mark.parametrize("wl", [W.SMALL_RAGGED, W.SMALL_RAGGED_T, W.TINY])
+def test_route_invariants_every_row(wl):
+    x = W.generate(wl)
+    g = O.block_geometry(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    Qp, Kp = O.pool(x["q"], g), O.pool(x["k"], g)
+    scale = 1.0 / math.sqrt(wl.d)
+    for p, k in [(wl.p, wl.k_floor), (0.5, 1), (0.95, 16), (0.0, 0), (1.0, 0)]:
+        r = O.route(Qp, Kp, p, k, scale)
+        for b in range(wl.B):
+            for h in range(wl.H):
+                for qb in range(g.nB):
+                    why = O.check_route_invariants(r.keep[b, h, qb], r.scores[b, h, qb], qb, p, k,
+                                                   tol=1e-12)
+                    assert why is None, (p, k, b, h, qb, why)
+                    assert r.keep[b, h, qb].sum() == r.counts[b, h, qb]
+
+
+def test_route_special_cases():
+    rng = np.random.default_rng(5)
+    Qp = rng.standard_normal((1, 2, 9, 8)) * 3
+    Kp = rng.standard_normal((1, 2, 9, 8))
+    assert O.route(Qp, Kp, 1.0, 0, 0.5).keep.all()
+    assert O.route(Qp, Kp, 0.3, 9, 0.5).keep.all()
+    assert O.route(Qp, Kp, 0.3, 50, 0.5).keep.all()
+    r = O.route(Qp, Kp, 0.0, 0, 0.5)
+    logits = np.einsum("bhid,bhjd->bhij", Qp, Kp)
+    for h in range(2):
+        for i in range(9):
+            want = {int(np.argmax(logits[0, h, i])), i}
+            assert set(np.nonzero(r.keep[0, h, i])[0].tolist()) == want
+
+
+def test_invariant_checker_rejects_planted_mistakes():
+    s = np.array([0.05, 0.4, 0.1, 0.25, 0.2])
+    good = np.array([1, 1, 0, 1, 1], bool)
+    assert O.check_route_invariants(good, s, 0, 0.7, 2) is None
+    assert O.check_route_invariants(np.array([1, 1, 1, 1, 0], bool), s, 0, 0.7, 2) is not None
+    assert O.check_route_invariants(np.array([0, 1, 0, 1, 1], bool), s, 0, 0.7, 2) is not None
+    assert O.check_route_invariants(np.array([1, 1, 1, 1, 1], bool), s, 0, 0.7, 2) is not None
+    assert O.check_route_invariants(np.array([1, 1, 0, 1, 0], bool), s, 0, 0.7, 2) is not None
+
+
+def test_pack_unpack_roundtrip_and_bit_order():
+    keep = np.zeros((1, 40), bool)
+    keep[0, [0, 33, 39]] = True
+    words = O.pack_mask(keep)
+    assert words.tolist() == [[1, (1 << 1) | (1 << 7)]]
+    rng = np.random.default_rng(2)
+    k2 = rng.random((3, 4, 70)) < 0.4
+    assert (O.unpack_mask(O.pack_mask(k2), 70) == k2).all()
+
+
+# ------------------------------------------------------------------ attention
+def _small_inputs(seed=3, B=1, H=2, T=2, Hs=6, Ws=10, d=16):
+    rng = np.random.default_rng(seed)
+    N = T * Hs * Ws
+    Q = rng.standard_normal((B, H, N, d)) * 1.5
+    K = rng.standard_normal((B, H, N, d))
+    V = rng.standard_normal((B, H, N, d))
+    return Q, K, V, O.block_geometry(T, Hs, Ws, 1, 4, 4)
+
+
+def test_masked_all_blocks_equals_dense():
+    Q, K, V, g = _small_inputs()
+    keep = np.ones((1, 2, g.nB, g.nB), bool)
+    tokens, out, lse = O.masked_attn(Q, K, V, keep, g, 0.25)
+    dout, dlse = O.dense_attn(Q, K, V, 0.25, tokens)
+    np.testing.assert_allclose(out, dout, atol=1e-12)
+    np.testing.assert_allclose(lse, dlse, atol=1e-12)
+
+
+def test_dense_matches_torch_sdpa_fp64():
+    Q, K, V, g = _small_inputs(seed=4)
+    out, lse = O.dense_attn(Q, K, V, 0.3)
+    tq, tk, tv = (torch.from_numpy(a) for a in (Q, K, V))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, scale=0.3)
+    np.testing.assert_allclose(out, ref.numpy(), atol=1e-12)
+    ref_lse = torch.logsumexp(tq @ tk.transpose(-1, -2) * 0.3, dim=-1)
+    np.testing.assert_allclose(lse, ref_lse.numpy(), atol=1e-12)
+
+
+def test_masked_matches_torch_sdpa_with_boolean_mask():
+    Q, K, V, g = _small_inputs(seed=6)
+    rng = np.random.default_rng(7)
+    keep = rng.random((1, 2, g.nB, g.nB)) < 0.4
+    keep[..., np.arange(g.nB), np.arange(g.nB)] = True
+    tokens, out, lse = O.masked_attn(Q, K, V, keep, g, 0.2)
+    bt = g.block_of_token
+    tok_mask = keep[:, :, bt][:, :, :, bt]                    # [B,H,N,N] token-level mask
+    tq, tk, tv = (torch.from_numpy(a) for a in (Q, K, V))
+    ref = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk, tv, attn_mask=torch.from_numpy(tok_mask), scale=0.2)
+    np.testing.assert_allclose(out, ref.numpy()[:, :, tokens], atol=1e-12)
+
+
+def test_lse_merge_identity_over_disjoint_key_sets():
+    Q, K, V, g = _small_inputs(seed=8)
+    rng = np.random.default_rng(9)
+    keep = rng.random((1, 2, g.nB, g.nB)) < 0.6
+    keep[..., np.arange(g.nB), np.arange(g.nB)] = True
+    split = rng.random(keep.shape) < 0.5
+    A = keep & split
+    Bm = keep & ~split
+    # make sure both halves are non-empty in every row
+    own = np.arange(g.nB)
+    A[..., own, own] = True
+    Bm[..., own, own] = False
+    Bm |= keep & ~A
+    Bm[..., own, (own + 1) % g.nB] |= ~Bm.any(-1)
+    full = A | Bm
+    _, out, lse = O.masked_attn(Q, K, V, full, g, 0.3)
+    _, oa, la = O.masked_attn(Q, K, V, A, g, 0.3)
+    _, ob, lb = O.masked_attn(Q, K, V, Bm, g, 0.3)
+    np.testing.assert_allclose(np.logaddexp(la, lb), lse, atol=1e-12)
+    wa, wb = np.exp(la - lse)[..., None], np.exp(lb - lse)[..., None]
+    np.testing.assert_allclose(wa * oa + wb * ob, out, atol=1e-12)
+
+
+def test_masked_attention_brute_force_loops():
+    Q, K, V, g = _small_inputs(seed=10, H=1, T=1, Hs=4, Ws=8, d=4)
+    keep = np.zeros((1, 1, g.nB, g.nB), bool)
+    keep[0, 0, 0, [0]] = True          # a single kept block: softmax over that block only
+    keep[0, 0, 1, [0, 1]] = True
+    tokens, out, lse = O.masked_attn(Q, K, V, keep, g, 0.7)
+    for row, i in enumerate(tokens.tolist()):
+        qb = g.block_of_token[i]
+        keys = [j for j in range(Q.shape[2]) if keep[0, 0, qb, g.block_of_token[j]]]
+        z = [math.exp(0.7 * sum(Q[0, 0, i, c] * K[0, 0, j, c] for c in range(4))) for j in keys]
+        tot = sum(z)
+        assert abs(lse[0, 0, row] - math.log(tot)) < 1e-12
+        for c in range(4):
+            o = sum(zj * V[0, 0, j, c] for zj, j in zip(z, keys)) / tot
+            assert abs(out[0, 0, row, c] - o) < 1e-12
+
+
+def test_layer_composes_the_three_steps():
+    w = W.TINY
+    x = W.generate(w)
+    g = O.block_geometry(w.T, w.Hs, w.Ws, w.bt, w.bh, w.bw)
+    res = O.layer(x["q"], x["k"], x["v"], g, 1.0, 0, 1 / 8.0)
+    dout, dlse = O.dense_attn(x["q"], x["k"], x["v"], 1 / 8.0, res["tokens"])
+    np.testing.assert_allclose(res["out"], dout, atol=1e-12)
+    np.testing.assert_allclose(res["lse"], dlse, atol=1e-12)
+
+
+def test_comparison_band_flags_rows_near_p():
+    # scores 0.5, 0.3, 0.2: with p = 0.8 the second prefix sum equals p, so fp32
+    # rounding may move the cut; the row must be reported ambiguous.
+    s = np.array([0.5, 0.3, 0.2])
+    Qp = np.tile(np.log(s), (3, 1))[None, None]
+    r = O.route(Qp, np.eye(3)[None, None], 0.8, 1, 1.0)
+    ex, amb = O.comparison_band(r, 0.8, 1)
+    assert amb[0, 0].all()
+    r2 = O.route(Qp, np.eye(3)[None, None], 0.6, 1, 1.0)
+    ex2, amb2 = O.comparison_band(r2, 0.6, 1)
+    assert not amb2.any()
