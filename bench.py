@@ -1,0 +1,413 @@
+#!/usr/bin/env python
+"""Benchmark of one adaptive block-sparse attention layer (pool -> route -> attention)
+on the Wan2.1-1.3B 480p self-attention shape (12 heads, 21x30x52 latent = 32760 tokens,
+d = 128, 3D blocks 1x8x16, p = 0.9, k_floor = 4), seeded synthetic inputs.
+
+One step = fvattn_block_pool + fvattn_route + fvattn_block_sparse_attn over the whole
+layer, inputs resident in HBM.  Each step is timed on the device with CUDA events on the
+launching stream; L2 is flushed (256 MiB write) between steps, outside the events.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep]
+
+With --gpus N > 1 (launched by torchrun) every rank runs an independent replica (the
+path has no exchange step); the time is the max over ranks and the value counts the
+work of all ranks.  --impl reference times the fp64 CPU oracle on a bounded sample of
+the same workload.  Prints one JSON line (rank 0).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import threading
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+from free_adaptive_block_b200 import metrics as MX  # noqa: E402
+from free_adaptive_block_b200 import workloads as W  # noqa: E402
+
+METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16 peak"
+UNIT = "TFLOP/s"
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            pk = json.load(f)
+        return dict(bf16=float(pk["bf16_tflops"]), bf16_sustained=float(pk["bf16_tflops_sustained"]),
+                    hbm=float(pk["hbm_gbs"]), source="measured")
+    except Exception:
+        return dict(bf16=1590.0, bf16_sustained=1400.0, hbm=6650.0, source="fallback")
+
+
+def config_of(wl, extra=None):
+    c = {"workload": wl.name, "B": wl.B, "H": wl.H, "N": wl.N, "latent": f"{wl.T}x{wl.Hs}x{wl.Ws}",
+         "d": wl.d, "block": f"{wl.bt}x{wl.bh}x{wl.bw}", "p": wl.p, "k_floor": wl.k_floor,
+         "l2": "flushed between steps (256 MiB write, outside the timed events)"}
+    if extra:
+        c.update(extra)
+    return c
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.lines = []
+        self.thread = None
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "200"],
+                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+        except Exception:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        if self.thread:
+            self.thread.join(timeout=2)
+        sm, smax, reasons = [], [], set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 8:
+                continue
+            try:
+                sm.append(float(parts[0]))
+                smax.append(float(parts[1]))
+            except ValueError:
+                continue
+            for nm, v in zip(names, parts[4:8]):
+                if v.lower().startswith("active"):
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(smax) if smax else None,
+                "reasons": sorted(reasons), "samples": len(sm)}
+
+
+# ----------------------------------------------------------------------------- GPU arm
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import free_adaptive_block_b200 as fv
+
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl = W.WAN21_480P
+    g = fv.Geometry(**wl.geom())
+    scale = float(np.float32(1.0 / math.sqrt(wl.d)))
+    peaks = load_peaks()
+
+    x = W.generate(wl)
+    host = {n: torch.from_numpy(W.bf16_bits(x[n])).view(torch.bfloat16) for n in ("q", "k", "v")}
+    q, k, v = (host[n].to(dev) for n in ("q", "k", "v"))
+    buf = fv.LayerBuffers.allocate(g, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fv.attention_layer(g, q, k, v, wl.p, wl.k_floor, scale, buf, stream)
+
+    # warm-up (also the mask used for the FLOP count)
+    for _ in range(max(args.warmup, 3)):
+        step()
+        flush.fill_(1.0)
+    torch.cuda.synchronize(dev)
+    if fv.fvattn_device_status(buf.workspace, stream) != 0:
+        raise RuntimeError("attention kernel reported a timeout")
+    keep = MX.unpack_words(buf.mask.cpu().numpy().view(np.uint32), g.nB)
+    real = MX.real_counts(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    eff = MX.effective_flops(keep, real, wl.d)
+    kept_frac = float(keep.mean())
+
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    sampler = ClockSampler(local_rank) if rank == 0 else None
+    if world > 1:
+        torch.distributed.barrier()
+    torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.start()
+        time.sleep(0.3)
+    for i in range(args.steps):
+        e = ev[i]
+        e[0].record(stream)
+        fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream)
+        e[1].record(stream)
+        fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts, stream)
+        e[2].record(stream)
+        fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse, buf.workspace,
+                                    buf.sm_busy_ns, stream)
+        e[3].record(stream)
+        flush.fill_(float(i))
+    torch.cuda.synchronize(dev)
+    if world > 1:
+        torch.distributed.barrier()
+    clocks = sampler.stop() if sampler else None
+    t_pool = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    t_route = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
+    t_attn = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
+    total_ms = sum(t_pool) + sum(t_route) + sum(t_attn)
+    if world > 1:
+        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        total_ms = float(t.item())
+    busy = buf.sm_busy_ns.cpu().numpy()
+    busy = busy[busy > 0]
+    if fv.fvattn_device_status(buf.workspace, stream) != 0:
+        raise RuntimeError("attention kernel reported a timeout")
+
+    # dense baseline (p = 1 through the same kernel), same protocol
+    dense_t = []
+    for i in range(max(args.warmup, 3) + min(args.steps, 10)):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace, None, stream)
+        b.record(stream)
+        flush.fill_(float(i))
+        torch.cuda.synchronize(dev)
+        if i >= max(args.warmup, 3):
+            dense_t.append(a.elapsed_time(b))
+    dense_ms = statistics.median(dense_t)
+
+    # end to end through the public API with host buffers (pinned), copies timed
+    pinned = {n: host[n].pin_memory() for n in ("q", "k", "v")}
+    out_h = torch.empty(buf.out.shape, dtype=torch.bfloat16).pin_memory()
+    lse_h = torch.empty(buf.lse.shape, dtype=torch.float32).pin_memory()
+    e2e_t = []
+    n_e2e = min(args.steps, 5)
+    for i in range(2 + n_e2e):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        qd, kd, vd = (pinned[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
+        fv.attention_layer(g, qd, kd, vd, wl.p, wl.k_floor, scale, buf, stream)
+        out_h.copy_(buf.out, non_blocking=True)
+        lse_h.copy_(buf.lse, non_blocking=True)
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        if i >= 2:
+            e2e_t.append(a.elapsed_time(b))
+    e2e_ms = statistics.mean(e2e_t)
+    h2d = sum(pinned[n].numel() * 2 for n in ("q", "k", "v"))
+    d2h = out_h.numel() * 2 + lse_h.numel() * 4
+
+    ms_step = total_ms / args.steps
+    attn_ms = statistics.mean(t_attn)
+    value = eff * world / (ms_step * 1e-3) / 1e12
+    attn_tflops = eff / (attn_ms * 1e-3) / 1e12
+    pr_bytes = MX.pool_route_bytes(wl.B, wl.H, wl.N, g.nB, wl.d, g.words)
+    pr_ms = statistics.mean(t_pool) + statistics.mean(t_route)
+    line = {
+        "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
+        "data": "synthetic", "config": config_of(wl),
+        "ms_per_layer": round(ms_step, 4),
+        "attn_ms": round(attn_ms, 4),
+        "attn_effective_tflops": round(attn_tflops, 2),
+        "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
+        "pool_ms": round(statistics.mean(t_pool), 4), "route_ms": round(statistics.mean(t_route), 4),
+        "pool_route_gbs": round(pr_bytes / (pr_ms * 1e-3) / 1e9, 1),
+        "pool_route_frac_of_hbm": round(pr_bytes / (pr_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
+        "dense_attn_ms": round(dense_ms, 4),
+        "dense_attn_tflops": round(MX.dense_flops(wl.B, wl.H, wl.N, wl.d) / (dense_ms * 1e-3) / 1e12, 2),
+        "speedup_vs_dense_attn": round(dense_ms / attn_ms, 3),
+        "kept_block_frac": round(kept_frac, 4),
+        "effective_flop_per_layer": eff,
+        "sm_busy_max_over_mean": round(float(busy.max() / busy.mean()), 4) if busy.size else None,
+        "roofline": {"bound": "tensor", "kernel": "fvattn_block_sparse_attn (prep + attn_kernel)",
+                     "achieved": round(attn_tflops, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
+                     "frac": round(attn_tflops / peaks["bf16"], 4), "traffic": None,
+                     "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
+        "e2e": {"value": round(eff * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clocks,
+    }
+    return line
+
+
+# ----------------------------------------------------------------------------- CPU oracle
+def oracle_sample(wl, x, n_qblocks: int, seed: int = 5):
+    """The oracle on a bounded sample: pool and route of the whole layer, masked
+    attention of n_qblocks query blocks per head.  Returns (seconds, effective flops)."""
+    sys.path.insert(0, ROOT)
+    import oracle as O
+    og = O.block_geometry(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    scale = 1.0 / math.sqrt(wl.d)
+    qbs = W.sample_qblocks(wl, n_qblocks, seed=seed)
+    t0 = time.perf_counter()
+    Qp, Kp = O.pool(x["q"], og), O.pool(x["k"], og)
+    r = O.route(Qp, Kp, wl.p, wl.k_floor, scale)
+    O.masked_attn(x["q"], x["k"], x["v"], r.keep, og, scale, qbs)
+    dt = time.perf_counter() - t0
+    real = og.real_count
+    sub = r.keep[:, :, qbs, :]
+    eff = float(4.0 * wl.d * ((sub.astype(np.int64) @ real) * real[qbs][None, None, :]).sum())
+    return dt, eff
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads") for i in threadpool_info() if i.get("num_threads")]
+        return int(max(n)) if n else os.cpu_count()
+    except Exception:
+        return os.cpu_count()
+
+
+def cpu_baseline(wl, x, budget_s: float = 15.0):
+    dt, eff = oracle_sample(wl, x, 2)
+    n = max(2, min(wl.nB, int(2 * budget_s / max(dt, 1e-3))))
+    dt, eff = oracle_sample(wl, x, n)
+    return {"value": round(eff / dt / 1e12, 6), "unit": UNIT, "cores": cpu_threads(), "kind": "oracle",
+            "seconds": round(dt, 2),
+            "sample": f"fp64 NumPy oracle: pool + route of the whole layer, masked attention of {n} "
+                      f"query blocks per head ({wl.H} heads); TFLOP/s = effective FLOPs of the sample / time"}
+
+
+def run_reference(args):
+    wl = W.WAN21_480P
+    x = W.generate(wl)
+    # size one step to ~2-4 s of CPU work
+    dt, _ = oracle_sample(wl, x, 1)
+    n = max(1, min(wl.nB, int(3.0 / max(dt, 1e-3))))
+    for _ in range(args.warmup):
+        oracle_sample(wl, x, n)
+    secs, flops = [], []
+    for i in range(args.steps):
+        dt, eff = oracle_sample(wl, x, n, seed=100 + i)
+        secs.append(dt)
+        flops.append(eff)
+    total = sum(secs)
+    value = sum(flops) / total / 1e12
+    sample = (f"fp64 NumPy oracle per step: pool + route of the whole layer and masked attention of "
+              f"{n} sampled query blocks per head ({wl.H} heads)")
+    return {"metric": METRIC, "value": round(value, 6), "unit": UNIT, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": round(1e3 * total / args.steps, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic", "config": config_of(wl), "impl": "reference",
+            "cpu_baseline": {"value": round(value, 6), "unit": UNIT, "cores": cpu_threads(),
+                             "kind": "oracle", "sample": sample},
+            "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def run_sweep(args, local_rank):
+    """Config-5 sweep: p x k_floor at the 480p shape; one JSON line per point (stdout)."""
+    import torch
+    import free_adaptive_block_b200 as fv
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    wl0 = W.WAN21_480P
+    g = fv.Geometry(**wl0.geom())
+    scale = float(np.float32(1.0 / math.sqrt(wl0.d)))
+    x = W.generate(wl0)
+    q, k, v = (torch.from_numpy(W.bf16_bits(x[n])).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+    buf = fv.LayerBuffers.allocate(g, dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    real = MX.real_counts(wl0.T, wl0.Hs, wl0.Ws, wl0.bt, wl0.bh, wl0.bw)
+    peaks = load_peaks()
+
+    def timed(fn, reps):
+        ts = []
+        for i in range(3 + reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record()
+            fn()
+            b.record()
+            flush.fill_(float(i))
+            torch.cuda.synchronize()
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    dense_ms = timed(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace), args.steps)
+    for wl in W.sweep():
+        fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
+        fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts)
+        torch.cuda.synchronize()
+        keep = MX.unpack_words(buf.mask.cpu().numpy().view(np.uint32), g.nB)
+        eff = MX.effective_flops(keep, real, wl.d)
+        ms = timed(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
+                                                        buf.workspace, buf.sm_busy_ns), args.steps)
+        busy = buf.sm_busy_ns.cpu().numpy()
+        busy = busy[busy > 0]
+        print(json.dumps({"sweep_point": wl.name, "p": wl.p, "k_floor": wl.k_floor,
+                          "kept_block_frac": round(float(keep.mean()), 4), "attn_ms": round(ms, 4),
+                          "effective_tflops": round(eff / (ms * 1e-3) / 1e12, 2),
+                          "frac_of_bf16_peak": round(eff / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
+                          "dense_attn_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / ms, 3),
+                          "sm_busy_max_over_mean": round(float(busy.max() / busy.mean()), 4)}), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--sweep", action="store_true", help="also time the 15 p/k points (config 5)")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+    rank = int(os.environ.get("RANK", 0))
+    world = int(os.environ.get("WORLD_SIZE", 1))
+    local_rank = int(os.environ.get("LOCAL_RANK", 0))
+
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+
+    if world > 1:
+        import datetime
+        import torch
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    try:
+        line = run_ours(args, rank, world, local_rank)
+        if rank == 0:
+            if world == 1 and not args.no_cpu_baseline:
+                line["cpu_baseline"] = cpu_baseline(W.WAN21_480P, W.generate(W.WAN21_480P))
+            print(json.dumps(line), flush=True)
+        if args.sweep and rank == 0:
+            run_sweep(args, local_rank)
+    finally:
+        if world > 1:
+            import torch
+            torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

@@ -1,0 +1,253 @@
+"""Python binding of libfvattn: adaptive block-sparse attention for video DiTs on B200.
+
+Argument marshalling only: every step of the path runs in the library's CUDA kernels
+(sm_100a).  PyTorch provides device memory and streams.  There is no CPU fallback:
+if ``libfvattn.so`` is missing or cannot be loaded, every call raises.
+
+Entry points mirror the C ABI in ``include/fvattn.h``:
+
+* ``fvattn_block_pool``   3D block mean-pooling of Q and K
+* ``fvattn_route``        per-head Top-p routing with a Top-k floor -> packed mask, counts
+* ``fvattn_block_sparse_attn``  attention over the kept key blocks -> out, lse
+* ``fvattn_dense_attn``   the same kernel with every key block kept
+
+and ``attention_layer`` strings the three steps together for one layer.
+"""
+from __future__ import annotations
+
+import ctypes
+import dataclasses
+import math
+import os
+from typing import Optional
+
+__all__ = [
+    "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
+    "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
+    "fvattn_dense_attn", "fvattn_device_status", "fvattn_status_string", "attention_layer",
+    "LayerBuffers",
+]
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+LIB_PATH = os.path.join(_HERE, "libfvattn.so")
+
+FVATTN_OK = 0
+STATUS_NAMES = {0: "FVATTN_OK", 1: "FVATTN_ERR_INVALID_ARG", 2: "FVATTN_ERR_UNSUPPORTED",
+                3: "FVATTN_ERR_WORKSPACE", 4: "FVATTN_ERR_CUDA", 5: "FVATTN_ERR_DEVICE_TIMEOUT"}
+
+
+class FvattnError(RuntimeError):
+    def __init__(self, fn: str, status: int):
+        self.status = status
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} "
+                         f"({fvattn_status_string(status)})")
+
+
+class _CGeom(ctypes.Structure):
+    _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "T", "Hs", "Ws", "d", "bt", "bh", "bw")]
+
+
+@dataclasses.dataclass(frozen=True)
+class Geometry:
+    B: int
+    H: int
+    T: int
+    Hs: int
+    Ws: int
+    d: int
+    bt: int
+    bh: int
+    bw: int
+
+    @property
+    def N(self) -> int:
+        return self.T * self.Hs * self.Ws
+
+    @property
+    def nB(self) -> int:
+        return (-(-self.T // self.bt)) * (-(-self.Hs // self.bh)) * (-(-self.Ws // self.bw))
+
+    @property
+    def words(self) -> int:
+        return -(-self.nB // 32)
+
+    def c(self) -> _CGeom:
+        return _CGeom(self.B, self.H, self.T, self.Hs, self.Ws, self.d, self.bt, self.bh, self.bw)
+
+
+_lib = None
+
+_SIGS = {
+    "fvattn_num_blocks": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_block_pool": (ctypes.c_int, [ctypes.c_void_p] * 6),
+    "fvattn_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                    ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                    ctypes.c_void_p]),
+    "fvattn_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_void_p]),
+    "fvattn_num_sms": (ctypes.c_int, []),
+    "fvattn_block_sparse_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                                ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                ctypes.c_size_t, ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_dense_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+}
+
+
+def lib() -> ctypes.CDLL:
+    """Load libfvattn.so (built in-tree by ``_build.py`` / ``__graft_entry__.build``)."""
+    global _lib
+    if _lib is None:
+        if not os.path.exists(LIB_PATH):
+            raise RuntimeError(f"{LIB_PATH} is missing: build it with "
+                               "`python -m free_adaptive_block_b200._build` (nvcc, sm_100a)")
+        handle = ctypes.CDLL(LIB_PATH)
+        for name, (res, args) in _SIGS.items():
+            f = getattr(handle, name)
+            f.restype = res
+            f.argtypes = args
+        _lib = handle
+    return _lib
+
+
+def fvattn_status_string(status: int) -> str:
+    return lib().fvattn_status_string(int(status)).decode()
+
+
+def _ok(fn: str, status: int) -> None:
+    if status != FVATTN_OK:
+        raise FvattnError(fn, status)
+
+
+def _stream(stream) -> Optional[int]:
+    import torch
+    if stream is None:
+        return torch.cuda.current_stream().cuda_stream
+    return getattr(stream, "cuda_stream", stream)
+
+
+def _ptr(t, dtype, shape, name):
+    if t is None:
+        return None
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if shape is not None and tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    return t.data_ptr()
+
+
+def fvattn_num_blocks(g: Geometry):
+    nB, words = ctypes.c_int(), ctypes.c_int()
+    cg = g.c()
+    _ok("fvattn_num_blocks", lib().fvattn_num_blocks(ctypes.byref(cg), ctypes.byref(nB), ctypes.byref(words)))
+    return nB.value, words.value
+
+
+def fvattn_block_pool(g: Geometry, q, k, q_pool, k_pool, stream=None) -> None:
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_block_pool", lib().fvattn_block_pool(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        _ptr(q_pool, torch.float32, pooled, "q_pool"), _ptr(k_pool, torch.float32, pooled, "k_pool"),
+        _stream(stream)))
+
+
+def fvattn_route(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: float, mask, counts,
+                 stream=None) -> None:
+    import torch
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_route", lib().fvattn_route(
+        ctypes.byref(cg), _ptr(q_pool, torch.float32, pooled, "q_pool"),
+        _ptr(k_pool, torch.float32, pooled, "k_pool"), float(p), int(k_floor), float(scale),
+        _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"), _stream(stream)))
+
+
+def fvattn_attn_workspace_size(g: Geometry) -> int:
+    cg = g.c()
+    return int(lib().fvattn_attn_workspace_size(ctypes.byref(cg)))
+
+
+def fvattn_num_sms() -> int:
+    return int(lib().fvattn_num_sms())
+
+
+def fvattn_block_sparse_attn(g: Geometry, q, k, v, mask, scale: float, out, lse, workspace,
+                             sm_busy_ns=None, stream=None) -> None:
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    cg = g.c()
+    _ok("fvattn_block_sparse_attn", lib().fvattn_block_sparse_attn(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        _ptr(v, torch.bfloat16, tok, "v"), _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        float(scale), _ptr(out, torch.bfloat16, tok, "out"), _ptr(lse, torch.float32, tok[:3], "lse"),
+        _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(),
+        _ptr(sm_busy_ns, torch.int64, None, "sm_busy_ns"), _stream(stream)))
+
+
+def fvattn_dense_attn(g: Geometry, q, k, v, scale: float, out, lse, workspace, sm_busy_ns=None,
+                      stream=None) -> None:
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    cg = g.c()
+    _ok("fvattn_dense_attn", lib().fvattn_dense_attn(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        _ptr(v, torch.bfloat16, tok, "v"), float(scale), _ptr(out, torch.bfloat16, tok, "out"),
+        _ptr(lse, torch.float32, tok[:3], "lse"), _ptr(workspace, torch.uint8, None, "workspace"),
+        workspace.numel(), _ptr(sm_busy_ns, torch.int64, None, "sm_busy_ns"), _stream(stream)))
+
+
+def fvattn_device_status(workspace, stream=None) -> int:
+    import torch
+    return int(lib().fvattn_device_status(_ptr(workspace, torch.uint8, None, "workspace"),
+                                          _stream(stream)))
+
+
+@dataclasses.dataclass
+class LayerBuffers:
+    """Device buffers of one layer (allocated with torch)."""
+    q_pool: "object"
+    k_pool: "object"
+    mask: "object"
+    counts: "object"
+    out: "object"
+    lse: "object"
+    workspace: "object"
+    sm_busy_ns: "object"
+
+    @classmethod
+    def allocate(cls, g: Geometry, device="cuda") -> "LayerBuffers":
+        import torch
+        ws = torch.empty(fvattn_attn_workspace_size(g), dtype=torch.uint8, device=device)
+        return cls(q_pool=torch.empty(g.B, g.H, g.nB, g.d, dtype=torch.float32, device=device),
+                   k_pool=torch.empty(g.B, g.H, g.nB, g.d, dtype=torch.float32, device=device),
+                   mask=torch.empty(g.B, g.H, g.nB, g.words, dtype=torch.int32, device=device),
+                   counts=torch.empty(g.B, g.H, g.nB, dtype=torch.int32, device=device),
+                   out=torch.empty(g.B, g.H, g.N, g.d, dtype=torch.bfloat16, device=device),
+                   lse=torch.empty(g.B, g.H, g.N, dtype=torch.float32, device=device),
+                   workspace=ws,
+                   sm_busy_ns=torch.zeros(max(1, fvattn_num_sms()), dtype=torch.int64, device=device))
+
+
+def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optional[float] = None,
+                    buffers: Optional[LayerBuffers] = None, stream=None) -> LayerBuffers:
+    """One adaptive block-sparse attention layer: pool -> route -> block-sparse attention.
+    Returns the buffers holding mask, counts, out and lse (asynchronous on `stream`)."""
+    if scale is None:
+        scale = 1.0 / math.sqrt(g.d)
+    b = buffers if buffers is not None else LayerBuffers.allocate(g, q.device)
+    fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
+    fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
+    fvattn_block_sparse_attn(g, q, k, v, b.mask, scale, b.out, b.lse, b.workspace, b.sm_busy_ns, stream)
+    return b

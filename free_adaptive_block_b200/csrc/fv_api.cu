@@ -1,0 +1,211 @@
+// C-ABI entry points of libfvattn (declared in include/fvattn.h): argument checks on
+// the host, TMA tensor-map encoding, kernel launches.  Nothing here allocates device
+// memory or synchronises, except fvattn_device_status.
+#include <cudaTypedefs.h>
+#include <math.h>
+
+#include <mutex>
+
+#include "fv_launch.h"
+#include "fvattn.h"
+
+namespace {
+
+using fv::Geo;
+
+constexpr int kMaxBlocks = 2048;   // route keeps a row of nB scores per warp in shared memory
+
+fvattn_status_t make_geo(const fvattn_geom_t* gi, Geo* g) {
+  if (gi == nullptr) return FVATTN_ERR_INVALID_ARG;
+  if (gi->B < 1 || gi->H < 1 || gi->T < 1 || gi->Hs < 1 || gi->Ws < 1 || gi->d < 1 ||
+      gi->bt < 1 || gi->bh < 1 || gi->bw < 1)
+    return FVATTN_ERR_INVALID_ARG;
+  if (gi->d != 64 && gi->d != 128) return FVATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(gi->bt) * gi->bh * gi->bw > 128) return FVATTN_ERR_UNSUPPORTED;
+  const long long N = static_cast<long long>(gi->T) * gi->Hs * gi->Ws;
+  if (N >= (1LL << 31)) return FVATTN_ERR_UNSUPPORTED;
+  Geo r;
+  r.B = gi->B; r.H = gi->H; r.T = gi->T; r.Hs = gi->Hs; r.Ws = gi->Ws; r.d = gi->d;
+  r.bt = gi->bt; r.bh = gi->bh; r.bw = gi->bw;
+  r.nBt = (gi->T + gi->bt - 1) / gi->bt;
+  r.nBy = (gi->Hs + gi->bh - 1) / gi->bh;
+  r.nBx = (gi->Ws + gi->bw - 1) / gi->bw;
+  const long long nB = static_cast<long long>(r.nBt) * r.nBy * r.nBx;
+  if (nB > kMaxBlocks) return FVATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(gi->B) * gi->H * nB >= (1LL << 24)) return FVATTN_ERR_UNSUPPORTED;
+  if (static_cast<long long>(gi->B) * gi->H * N * gi->d >= (1LL << 40)) return FVATTN_ERR_UNSUPPORTED;
+  r.nB = static_cast<int>(nB);
+  r.words = (r.nB + 31) / 32;
+  r.N = static_cast<int>(N);
+  *g = r;
+  return FVATTN_OK;
+}
+
+fvattn_status_t check_ptr(const void* p) {
+  if (p == nullptr) return FVATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p) & 15u) return FVATTN_ERR_UNSUPPORTED;
+  return FVATTN_OK;
+}
+
+#define FV_CHECK(expr)                       \
+  do {                                       \
+    const fvattn_status_t s_ = (expr);       \
+    if (s_ != FVATTN_OK) return s_;          \
+  } while (0)
+
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  });
+  return fn;
+}
+
+// 5D map over a bf16 [B*H][T][Hs][Ws][d] tensor; box = 64 channels x box_x columns x
+// bh rows x bt frames x 1 slice, 128-byte swizzle, zero fill out of range.
+bool encode_map(CUtensorMap* m, const void* ptr, const Geo& g, int box_x) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const cuuint64_t es = 2;
+  cuuint64_t dims[5] = {static_cast<cuuint64_t>(g.d), static_cast<cuuint64_t>(g.Ws),
+                        static_cast<cuuint64_t>(g.Hs), static_cast<cuuint64_t>(g.T),
+                        static_cast<cuuint64_t>(g.B) * g.H};
+  cuuint64_t strides[4] = {g.d * es, static_cast<cuuint64_t>(g.Ws) * g.d * es,
+                           static_cast<cuuint64_t>(g.Hs) * g.Ws * g.d * es,
+                           static_cast<cuuint64_t>(g.T) * g.Hs * g.Ws * g.d * es};
+  cuuint32_t box[5] = {64u, static_cast<cuuint32_t>(box_x), static_cast<cuuint32_t>(g.bh),
+                       static_cast<cuuint32_t>(g.bt), 1u};
+  cuuint32_t estr[5] = {1, 1, 1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 5, const_cast<void*>(ptr), dims, strides,
+                        box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+int current_num_sms() {
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) return 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return 0;
+  return n;
+}
+
+fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, const void* v,
+                         const uint32_t* mask, float scale, void* out, float* lse, void* ws,
+                         size_t ws_bytes, unsigned long long* busy, fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr(q));
+  FV_CHECK(check_ptr(k));
+  FV_CHECK(check_ptr(v));
+  FV_CHECK(check_ptr(out));
+  FV_CHECK(check_ptr(lse));
+  if (mask != nullptr) FV_CHECK(check_ptr(mask));
+  if (busy != nullptr && (reinterpret_cast<uintptr_t>(busy) & 7u)) return FVATTN_ERR_UNSUPPORTED;
+  if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  if (ws == nullptr || ws_bytes < fv::attn_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(ws) & 15u) return FVATTN_ERR_UNSUPPORTED;
+  const int nsm = current_num_sms();
+  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
+  fv::AttnMaps maps;
+  if (!encode_map(&maps.q, q, g, g.bw) || !encode_map(&maps.qe, q, g, rx_edge) ||
+      !encode_map(&maps.k, k, g, g.bw) || !encode_map(&maps.ke, k, g, rx_edge) ||
+      !encode_map(&maps.v, v, g, g.bw) || !encode_map(&maps.ve, v, g, rx_edge))
+    return FVATTN_ERR_CUDA;
+  const cudaError_t e = fv::launch_attn(g, maps, mask, scale, out, lse, ws, busy, nsm,
+                                        reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+fvattn_status_t fvattn_num_blocks(const fvattn_geom_t* gi, int* nB, int* words) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  if (nB) *nB = g.nB;
+  if (words) *words = g.words;
+  return FVATTN_OK;
+}
+
+fvattn_status_t fvattn_block_pool(const fvattn_geom_t* gi, const void* q, const void* k,
+                                  float* q_pool, float* k_pool, fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr(q));
+  FV_CHECK(check_ptr(k));
+  FV_CHECK(check_ptr(q_pool));
+  FV_CHECK(check_ptr(k_pool));
+  const cudaError_t e = fv::launch_pool(g, q, k, q_pool, k_pool, reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+fvattn_status_t fvattn_route(const fvattn_geom_t* gi, const float* q_pool, const float* k_pool,
+                             float p, int k_floor, float scale, uint32_t* mask, int32_t* counts,
+                             fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr(q_pool));
+  FV_CHECK(check_ptr(k_pool));
+  FV_CHECK(check_ptr(mask));
+  FV_CHECK(check_ptr(counts));
+  if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
+  if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  const cudaError_t e = fv::launch_route(g, q_pool, k_pool, p, k_floor, scale, mask, counts,
+                                         reinterpret_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+}
+
+size_t fvattn_attn_workspace_size(const fvattn_geom_t* gi) {
+  Geo g;
+  if (make_geo(gi, &g) != FVATTN_OK) return 0;
+  return fv::attn_ws_bytes(g);
+}
+
+int fvattn_num_sms(void) { return current_num_sms(); }
+
+fvattn_status_t fvattn_block_sparse_attn(const fvattn_geom_t* g, const void* q, const void* k,
+                                         const void* v, const uint32_t* mask, float scale,
+                                         void* out, float* lse, void* workspace, size_t ws_bytes,
+                                         unsigned long long* sm_busy_ns, fvattn_stream_t stream) {
+  if (mask == nullptr) return FVATTN_ERR_INVALID_ARG;
+  return run_attn(g, q, k, v, mask, scale, out, lse, workspace, ws_bytes, sm_busy_ns, stream);
+}
+
+fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void* q, const void* k,
+                                  const void* v, float scale, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes,
+                                  unsigned long long* sm_busy_ns, fvattn_stream_t stream) {
+  return run_attn(g, q, k, v, nullptr, scale, out, lse, workspace, ws_bytes, sm_busy_ns, stream);
+}
+
+fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream) {
+  if (workspace == nullptr) return FVATTN_ERR_INVALID_ARG;
+  uint32_t hdr[2] = {0, 0};
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaMemcpyAsync(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, st) != cudaSuccess)
+    return FVATTN_ERR_CUDA;
+  if (cudaStreamSynchronize(st) != cudaSuccess) return FVATTN_ERR_CUDA;
+  return (hdr[1] & fv::kErrTimeout) ? FVATTN_ERR_DEVICE_TIMEOUT : FVATTN_OK;
+}
+
+const char* fvattn_status_string(fvattn_status_t s) {
+  switch (s) {
+    case FVATTN_OK: return "ok";
+    case FVATTN_ERR_INVALID_ARG: return "invalid argument";
+    case FVATTN_ERR_UNSUPPORTED: return "unsupported shape, size or alignment";
+    case FVATTN_ERR_WORKSPACE: return "workspace missing or too small";
+    case FVATTN_ERR_CUDA: return "CUDA call failed";
+    case FVATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+  }
+  return "unknown status";
+}
+
+}  // extern "C"

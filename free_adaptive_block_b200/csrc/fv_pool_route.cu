@@ -1,0 +1,338 @@
+// 3D block mean-pooling and per-head Top-p / Top-k block routing.
+//
+// FVAttn explainer (arXiv 2607.16190), 核心方法 §1 稀疏路由前端: tokens are grouped
+// into video-aware 3D blocks and each head decides per block which key blocks a
+// query block keeps: the minimal set whose cumulative similarity mass reaches p
+// (Top-p), at least k of them (Top-k safety floor).  The routing score is the
+// softmax over key blocks of the pooled q . pooled k / sqrt(d); the query's own
+// block is always kept.
+#include <cuda_bf16.h>
+#include <float.h>
+
+#include "fv_common.cuh"
+#include "fv_launch.h"
+
+namespace fv {
+
+// ----------------------------------------------------------------------------
+// Pooling: one CTA per (b*h, block).  Thread t owns the 16-byte chunk t % (d/8) of
+// the tokens t / (d/8), t / (d/8) + 256 / (d/8), ...  of the block; partial sums
+// are folded with warp shuffles, then across warps through shared memory.
+// Loads are 16-byte vectors, and a warp reads whole 256-byte token rows.
+// ----------------------------------------------------------------------------
+constexpr int kPoolThreads = 256;
+
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, const uint4* __restrict__ q,
+                                                            const uint4* __restrict__ k,
+                                                            float* __restrict__ qp,
+                                                            float* __restrict__ kp) {
+  constexpr int CH = D / 8;               // 16-byte chunks per token
+  constexpr int G = kPoolThreads / CH;     // tokens processed side by side
+  constexpr int MAXR = 128 / G;            // a block holds at most 128 tokens
+  __shared__ float red[2][kPoolThreads / 32][D];
+
+  const int j = blockIdx.x;
+  const int bhi = blockIdx.y;
+  const BlockInfo bi = block_info(g, j);
+  const int nreal = bi.nvalid;
+  const int plane = bi.ry * bi.rx;
+  const int ch = threadIdx.x % CH;
+  const int grp = threadIdx.x / CH;
+  const size_t base = static_cast<size_t>(bhi) * g.N;
+  const int t0 = bi.tb * g.bt, y0 = bi.yb * g.bh, x0 = bi.xb * g.bw;
+
+  uint4 vq[MAXR], vk[MAXR];
+#pragma unroll
+  for (int i = 0; i < MAXR; ++i) {
+    const int r = grp + i * G;
+    if (r < nreal) {
+      const int tt = r / plane;
+      const int r2 = r - tt * plane;
+      const int yy = r2 / bi.rx;
+      const int xx = r2 - yy * bi.rx;
+      const size_t n = base + (static_cast<size_t>(t0 + tt) * g.Hs + (y0 + yy)) * g.Ws + (x0 + xx);
+      vq[i] = __ldg(q + n * CH + ch);
+      vk[i] = __ldg(k + n * CH + ch);
+    } else {
+      vq[i] = make_uint4(0, 0, 0, 0);
+      vk[i] = make_uint4(0, 0, 0, 0);
+    }
+  }
+  float aq[8], ak[8];
+#pragma unroll
+  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.f;
+#pragma unroll
+  for (int i = 0; i < MAXR; ++i) {
+    const uint32_t wq[4] = {vq[i].x, vq[i].y, vq[i].z, vq[i].w};
+    const uint32_t wk[4] = {vk[i].x, vk[i].y, vk[i].z, vk[i].w};
+#pragma unroll
+    for (int e = 0; e < 4; ++e) {
+      aq[2 * e] += __uint_as_float(wq[e] << 16);
+      aq[2 * e + 1] += __uint_as_float(wq[e] & 0xFFFF0000u);
+      ak[2 * e] += __uint_as_float(wk[e] << 16);
+      ak[2 * e + 1] += __uint_as_float(wk[e] & 0xFFFF0000u);
+    }
+  }
+  // lanes l, l + CH, ... of a warp hold the same chunk
+#pragma unroll
+  for (int off = CH; off < 32; off <<= 1) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      aq[e] += __shfl_xor_sync(0xffffffffu, aq[e], off);
+      ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], off);
+    }
+  }
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  if (lane < CH) {
+#pragma unroll
+    for (int e = 0; e < 8; ++e) {
+      red[0][warp][lane * 8 + e] = aq[e];
+      red[1][warp][lane * 8 + e] = ak[e];
+    }
+  }
+  __syncthreads();
+  const float inv = 1.f / static_cast<float>(nreal);
+  for (int t = threadIdx.x; t < 2 * D; t += kPoolThreads) {
+    const int which = t / D, dd = t - which * D;
+    float s = 0.f;
+#pragma unroll
+    for (int w = 0; w < kPoolThreads / 32; ++w) s += red[which][w][dd];
+    float* dst = which ? kp : qp;
+    dst[(static_cast<size_t>(bhi) * g.nB + j) * D + dd] = s * inv;
+  }
+}
+
+cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, float* kp,
+                        cudaStream_t st) {
+  dim3 grid(g.nB, g.B * g.H);
+  if (g.d == 128)
+    pool_kernel<128><<<grid, kPoolThreads, 0, st>>>(g, static_cast<const uint4*>(q),
+                                                     static_cast<const uint4*>(k), qp, kp);
+  else
+    pool_kernel<64><<<grid, kPoolThreads, 0, st>>>(g, static_cast<const uint4*>(q),
+                                                    static_cast<const uint4*>(k), qp, kp);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// Routing: one CTA per (b*h, 8 query blocks); warp w owns query block
+// blockIdx.x * 8 + w.  Logits come from key tiles of 32 blocks staged transposed in
+// shared memory (lane = key block).  Then, per warp: softmax over all key blocks,
+// and a bitwise search for the Top-p cut over an order-preserving integer key of
+// the logits, so no sort is needed:
+//   u* = the largest key with mass(key >= u*) >= p  -> the key of the m_p-th block,
+// equal keys are taken in ascending block index.  The Top-k floor lengthens the
+// prefix with a second search on counts.  Reductions are warp shuffles in a fixed
+// order, so the result is deterministic.
+// ----------------------------------------------------------------------------
+constexpr int kRouteRows = 8;
+constexpr int kRouteThreads = kRouteRows * 32;
+
+__device__ __forceinline__ uint32_t order_key(float x) {
+  const uint32_t u = __float_as_uint(x);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+__device__ __forceinline__ int warp_sum_i(int v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, off));
+  return v;
+}
+
+template <int D>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float* __restrict__ qp,
+                                                              const float* __restrict__ kp, float p,
+                                                              int k_floor, float scale,
+                                                              uint32_t* __restrict__ mask,
+                                                              int32_t* __restrict__ counts) {
+  extern __shared__ __align__(16) unsigned char route_smem[];
+  const int words = g.words;
+  const int nBpad = words * 32;
+  float* sQ = reinterpret_cast<float*>(route_smem);                  // [8][D]
+  float* sKT = sQ + kRouteRows * D;                                   // [D][33]
+  uint32_t* sKey = reinterpret_cast<uint32_t*>(sKT + D * 33);         // [8][nBpad]
+  float* sS = reinterpret_cast<float*>(sKey + kRouteRows * nBpad);    // [8][nBpad]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bhi = blockIdx.y;
+  const int nB = g.nB;
+  const int qb = blockIdx.x * kRouteRows + warp;
+  const float* kph = kp + static_cast<size_t>(bhi) * nB * D;
+
+  for (int e = threadIdx.x; e < kRouteRows * D; e += kRouteThreads) {
+    const int r = e / D, dd = e - r * D;
+    const int row = blockIdx.x * kRouteRows + r;
+    sQ[e] = row < nB ? qp[(static_cast<size_t>(bhi) * nB + row) * D + dd] : 0.f;
+  }
+  uint32_t* myKey = sKey + warp * nBpad;
+  float* myS = sS + warp * nBpad;
+  for (int kt = 0; kt < words; ++kt) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * D; e += kRouteThreads) {
+      const int key = e / D, dd = e - key * D;
+      const int j = kt * 32 + key;
+      sKT[dd * 33 + key] = j < nB ? kph[static_cast<size_t>(j) * D + dd] : 0.f;
+    }
+    __syncthreads();
+    float acc = 0.f;
+    const float* qrow = sQ + warp * D;
+#pragma unroll 16
+    for (int dd = 0; dd < D; ++dd) acc = fmaf(qrow[dd], sKT[dd * 33 + lane], acc);
+    const int j = kt * 32 + lane;
+    const float logit = acc * scale;
+    myKey[j] = j < nB ? order_key(logit) : 0u;
+    myS[j] = j < nB ? logit : -INFINITY;
+  }
+  __syncwarp();
+  if (qb >= nB) return;
+
+  // softmax over the key blocks (fp32)
+  float mx = -INFINITY;
+  for (int c = 0; c < words; ++c) mx = fmaxf(mx, myS[c * 32 + lane]);
+  mx = warp_max(mx);
+  float z = 0.f;
+  for (int c = 0; c < words; ++c) {
+    const int i = c * 32 + lane;
+    const float e = i < nB ? expf(myS[i] - mx) : 0.f;
+    myS[i] = e;
+    z += e;
+  }
+  z = warp_sum(z);
+  const float inv_z = 1.f / z;
+  float total = 0.f;
+  for (int c = 0; c < words; ++c) {
+    const int i = c * 32 + lane;
+    const float s = myS[i] * inv_z;
+    myS[i] = s;
+    total += s;
+  }
+  total = warp_sum(total);
+
+  auto mass_ge = [&](uint32_t u) {
+    float m = 0.f;
+    for (int c = 0; c < words; ++c) {
+      const int i = c * 32 + lane;
+      m += (i < nB && myKey[i] >= u) ? myS[i] : 0.f;
+    }
+    return warp_sum(m);
+  };
+  auto count_ge = [&](uint32_t u) {
+    int n = 0;
+    for (int c = 0; c < words; ++c) {
+      const int i = c * 32 + lane;
+      n += (i < nB && myKey[i] >= u) ? 1 : 0;
+    }
+    return warp_sum_i(n);
+  };
+  auto count_gt_eq = [&](uint32_t u, int& gt, int& eq, float& gt_mass, float& eq_score) {
+    int a = 0, b = 0;
+    float m = 0.f, es = 0.f;
+    for (int c = 0; c < words; ++c) {
+      const int i = c * 32 + lane;
+      if (i < nB) {
+        const uint32_t key = myKey[i];
+        if (key > u) { ++a; m += myS[i]; }
+        if (key == u) { ++b; es = myS[i]; }
+      }
+    }
+    gt = warp_sum_i(a);
+    eq = warp_sum_i(b);
+    gt_mass = warp_sum(m);
+    eq_score = warp_max(es);
+  };
+
+  const int floor_k = min(max(k_floor, 0), nB);
+  int m_p;
+  uint32_t u = 0;
+  int ties_needed = 0;
+  if (p >= 1.f || total < p) {
+    m_p = nB;
+  } else {
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = u | (1u << bit);
+      if (mass_ge(cand) >= p) u = cand;
+    }
+    int gt, eq;
+    float gt_mass, eq_s;
+    count_gt_eq(u, gt, eq, gt_mass, eq_s);
+    float acc = gt_mass;
+    int r = 0;
+    while (acc < p && r < eq) {
+      acc += eq_s;
+      ++r;
+    }
+    m_p = gt + r;
+    ties_needed = r;
+  }
+  const int M = max(max(m_p, floor_k), 1);
+  if (M >= nB) {
+    u = 0;
+    ties_needed = nB;     // every block
+  } else if (M > m_p) {
+    uint32_t v = 0;
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = v | (1u << bit);
+      if (count_ge(cand) >= M) v = cand;
+    }
+    int gt, eq;
+    float gm, es;
+    count_gt_eq(v, gt, eq, gm, es);
+    u = v;
+    ties_needed = M - gt;
+  }
+
+  uint32_t* mrow = mask + (static_cast<size_t>(bhi) * nB + qb) * words;
+  int tie_base = 0, cnt = 0;
+  for (int c = 0; c < words; ++c) {
+    const int i = c * 32 + lane;
+    const bool valid = i < nB;
+    const uint32_t key = valid ? myKey[i] : 0u;
+    const bool tie = valid && key == u;
+    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+    const int rank = tie_base + __popc(tb & ((1u << lane) - 1u));
+    tie_base += __popc(tb);
+    const bool kept = valid && (key > u || (tie && rank < ties_needed) || i == qb);
+    const uint32_t word = __ballot_sync(0xffffffffu, kept);
+    cnt += __popc(word);
+    if (lane == 0) mrow[c] = word;
+  }
+  if (lane == 0) counts[static_cast<size_t>(bhi) * nB + qb] = cnt;
+}
+
+size_t route_smem_bytes(const Geo& g) {
+  const size_t nBpad = static_cast<size_t>(g.words) * 32;
+  return (static_cast<size_t>(kRouteRows) * g.d + static_cast<size_t>(g.d) * 33) * 4 +
+         static_cast<size_t>(kRouteRows) * nBpad * 8;
+}
+
+cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                         float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
+  dim3 grid((g.nB + kRouteRows - 1) / kRouteRows, g.B * g.H);
+  const size_t smem = route_smem_bytes(g);
+  cudaError_t e;
+  if (g.d == 128) {
+    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    route_kernel<128><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
+  } else {
+    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             static_cast<int>(smem));
+    if (e != cudaSuccess) return e;
+    route_kernel<64><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
+  }
+  return cudaGetLastError();
+}
+
+}  // namespace fv

@@ -1,0 +1,154 @@
+/*
+ * fvattn — training-free adaptive block-sparse attention for video diffusion
+ * transformers, on NVIDIA B200 (sm_100a).
+ *
+ * The method: "FVAttn: Adaptive Sparse Attention with Runtime Load Balancing for
+ * Video Generation" (explainer of arXiv 2607.16190), section 核心方法 §1
+ * 稀疏路由前端 (sparse-routing frontend): spatio-temporal tokens are grouped into
+ * 3D blocks (video-aware block organisation); each head routes per query block
+ * with Top-p over block similarity mass plus a Top-k safety floor; attention then
+ * runs only over the selected key blocks (the kernel that replaces FlashAttention,
+ * 核心方法 §2, attn_kernel.run()).
+ *
+ * Conventions shared by every entry point
+ * ---------------------------------------
+ * - Tensors are row-major and contiguous.  Q, K, V and out are bf16
+ *   [B][H][N][d], N = T*Hs*Ws, token n of a (b,h) slice at latent position
+ *   (t, y, x) with n = (t*Hs + y)*Ws + x  ("T-major").
+ * - 3D block (tb, yb, xb) covers t in [tb*bt, tb*bt+bt), y in [yb*bh, ...),
+ *   x in [xb*bw, ...), clipped to the latent: edge blocks are partial.  Blocks are
+ *   numbered T-major: j = (tb*nBy + yb)*nBx + xb, nBt = ceil(T/bt), nBy =
+ *   ceil(Hs/bh), nBx = ceil(Ws/bw), nB = nBt*nBy*nBx.
+ * - Every pointer argument is a DEVICE pointer, 16-byte aligned, owned by the
+ *   caller.  The library allocates no device memory and keeps no state between
+ *   calls apart from cached driver entry points.
+ * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
+ *   stream) and never synchronise.  Argument errors are detected on the host
+ *   before anything is launched.  Launch failures return FVATTN_ERR_CUDA;
+ *   faults during execution surface at the caller's next synchronisation.
+ * - No C++ exception crosses this interface.
+ * - Supported: d in {64, 128}; 1 <= bt*bh*bw <= 128; nB <= 2048; B*H*nB < 2^24.
+ */
+#ifndef FVATTN_H_
+#define FVATTN_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#if defined(__GNUC__)
+#define FVATTN_API __attribute__((visibility("default")))
+#else
+#define FVATTN_API
+#endif
+
+struct CUstream_st;                          /* cudaStream_t is struct CUstream_st* */
+typedef struct CUstream_st* fvattn_stream_t;
+
+typedef enum {
+  FVATTN_OK = 0,
+  FVATTN_ERR_INVALID_ARG = 1,     /* null pointer, bad size, p/k/scale out of domain */
+  FVATTN_ERR_UNSUPPORTED = 2,     /* valid but unsupported: d, block size, alignment */
+  FVATTN_ERR_WORKSPACE = 3,       /* workspace missing or smaller than required */
+  FVATTN_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
+  FVATTN_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up a bounded wait (see fvattn_device_status) */
+} fvattn_status_t;
+
+typedef struct {
+  int B, H;          /* batch, heads                                  */
+  int T, Hs, Ws;     /* latent frames, height, width (tokens)          */
+  int d;             /* head dimension: 64 or 128                      */
+  int bt, bh, bw;    /* 3D block extent in frames, rows, columns       */
+} fvattn_geom_t;
+
+/* Number of 3D blocks nB and of 32-bit mask words per mask row, ceil(nB/32).
+ * Returns FVATTN_ERR_INVALID_ARG for a null or malformed geometry. */
+FVATTN_API fvattn_status_t fvattn_num_blocks(const fvattn_geom_t* g, int* nB, int* words);
+
+/* 3D block mean-pooling (video-aware block organisation, FVAttn explainer
+ * 核心方法 §1).  For every (b, h, block j):
+ *   q_pool[b][h][j][:] = mean of q[b][h][n][:] over the real tokens n of block j,
+ * and likewise k_pool from k.  Edge blocks average over their real tokens only.
+ *   q, k    : bf16 [B][H][N][d]              (read)
+ *   q_pool, k_pool : fp32 [B][H][nB][d]       (written)
+ * Accumulation in fp32. */
+FVATTN_API fvattn_status_t fvattn_block_pool(const fvattn_geom_t* g, const void* q, const void* k,
+                                  float* q_pool, float* k_pool, fvattn_stream_t stream);
+
+/* Per-head Top-p block routing with a Top-k floor (FVAttn explainer 核心方法 §1,
+ * "Top-p 路由" and "Top-k 安全底").  For every (b, h, query block i):
+ *   l_j = (q_pool[i] . k_pool[j]) * scale over all key blocks j,
+ *   s   = softmax_j(l)                              (the routing score),
+ *   order the key blocks by s descending, ties to the lower index,
+ *   m_p = the shortest prefix with cumulative mass >= p (nB when p >= 1 or when
+ *         the total mass falls short of p),
+ *   m   = max(m_p, min(k_floor, nB)),
+ *   kept = the first m blocks of that order, plus block i itself.
+ * Outputs:
+ *   mask   : uint32 [B][H][nB][words]; bit (j % 32) of word (j / 32) is set when
+ *            key block j is kept; bits at j >= nB are zero.
+ *   counts : int32  [B][H][nB]; number of kept blocks (popcount of the row).
+ * Arguments: 0 <= p (p >= 1 keeps every block), k_floor >= 0, scale > 0 and
+ * finite (normally 1/sqrt(d), the same scale the attention uses).
+ * Scores and masses are fp32; selection uses the logits' order. */
+FVATTN_API fvattn_status_t fvattn_route(const fvattn_geom_t* g, const float* q_pool, const float* k_pool,
+                             float p, int k_floor, float scale,
+                             uint32_t* mask, int32_t* counts, fvattn_stream_t stream);
+
+/* Bytes of device workspace fvattn_block_sparse_attn / fvattn_dense_attn need
+ * for geometry g (a tile queue and a status word).  0 for a malformed geometry. */
+FVATTN_API size_t fvattn_attn_workspace_size(const fvattn_geom_t* g);
+
+/* Number of entries fvattn_block_sparse_attn writes to sm_busy_ns: the number of
+ * streaming multiprocessors of the current device (0 on error). */
+FVATTN_API int fvattn_num_sms(void);
+
+/* Block-sparse attention over the kept key blocks (the attention kernel of the
+ * FVAttn explainer 核心方法 §2; online softmax over the kept blocks in ascending
+ * block order).  For every real query token n of query block i of (b, h):
+ *   lse[n] = ln sum_{m in kept(i)} exp((q_n . k_m) * scale),
+ *   out[n] = sum_{m in kept(i)} exp((q_n . k_m) * scale - lse[n]) v_m,
+ * where m runs over the real tokens of the key blocks whose mask bit is set.
+ *   q, k, v : bf16 [B][H][N][d]      (read)
+ *   mask    : uint32 [B][H][nB][words], as written by fvattn_route; every row
+ *             must have at least one bit set (fvattn_route always sets bit i).
+ *   out     : bf16 [B][H][N][d]      (written, every token)
+ *   lse     : fp32 [B][H][N]         (written, every token)
+ *   workspace, ws_bytes : >= fvattn_attn_workspace_size(g) bytes, 16-byte aligned,
+ *             contents need not be initialised; not to be shared by calls that
+ *             run concurrently.
+ *   sm_busy_ns : optional (NULL to skip) uint64 [fvattn_num_sms()]; receives, per SM,
+ *             the nanoseconds from the start of its CTA to the end of its last tile.
+ * Products are bf16 x bf16 with fp32 accumulation; the softmax is fp32 with P
+ * rounded to bf16 before the P.V product.  Work is scheduled by a persistent
+ * kernel over (b, h, query block) tiles taken from a queue ordered by decreasing
+ * cost (longest processing time first). */
+FVATTN_API fvattn_status_t fvattn_block_sparse_attn(const fvattn_geom_t* g, const void* q, const void* k,
+                                         const void* v, const uint32_t* mask, float scale,
+                                         void* out, float* lse,
+                                         void* workspace, size_t ws_bytes,
+                                         unsigned long long* sm_busy_ns, fvattn_stream_t stream);
+
+/* Dense attention: fvattn_block_sparse_attn with every key block kept (the p = 1
+ * case), without reading a mask.  Same arguments otherwise. */
+FVATTN_API fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void* q, const void* k,
+                                  const void* v, float scale, void* out, float* lse,
+                                  void* workspace, size_t ws_bytes,
+                                  unsigned long long* sm_busy_ns, fvattn_stream_t stream);
+
+/* Synchronises `stream` and reports whether the last attention call that used
+ * `workspace` gave up a bounded wait inside the kernel: FVATTN_OK or
+ * FVATTN_ERR_DEVICE_TIMEOUT (FVATTN_ERR_CUDA if the synchronisation failed). */
+FVATTN_API fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream);
+
+/* Static, human-readable name of a status code. */
+FVATTN_API const char* fvattn_status_string(fvattn_status_t s);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FVATTN_H_ */

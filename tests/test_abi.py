@@ -1,0 +1,87 @@
+"""The C ABI without a GPU: the library loads, exports every entry point the header
+declares, and rejects bad arguments on the host before touching CUDA."""
+import ctypes
+import os
+import re
+
+import pytest
+
+import free_adaptive_block_b200 as fv
+from free_adaptive_block_b200 import _build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    _build.build()
+    return fv.lib()
+
+
+def header_functions():
+    src = open(os.path.join(ROOT, "include", "fvattn.h")).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fvattn_[a-z_]+)\s*\(", src)))
+
+
+def test_exports_every_declared_symbol(L):
+    names = header_functions()
+    assert len(names) >= 9
+    for n in names:
+        assert hasattr(L, n), n
+
+
+G480 = fv.Geometry(B=1, H=12, T=21, Hs=30, Ws=52, d=128, bt=1, bh=8, bw=16)
+
+
+def test_geometry_queries(L):
+    assert fv.fvattn_num_blocks(G480) == (336, 11)
+    assert fv.fvattn_num_blocks(fv.Geometry(1, 2, 4, 8, 8, 64, 2, 4, 4)) == (8, 1)
+    ws = fv.fvattn_attn_workspace_size(G480)
+    assert ws >= 256 + 8 * 12 * 336 and ws % 256 == 0
+
+
+def call_route(L, g, qp=0x1000, kp=0x2000, p=0.9, k=4, scale=0.088, mask=0x3000, counts=0x4000):
+    cg = g.c()
+    return L.fvattn_route(ctypes.byref(cg), qp, kp, p, k, scale, mask, counts, None)
+
+
+def test_host_side_argument_checks(L):
+    E = {v: k for k, v in fv.STATUS_NAMES.items()}
+    assert call_route(L, G480, qp=None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert call_route(L, G480, p=float("nan")) == E["FVATTN_ERR_INVALID_ARG"]
+    assert call_route(L, G480, p=-0.1) == E["FVATTN_ERR_INVALID_ARG"]
+    assert call_route(L, G480, k=-1) == E["FVATTN_ERR_INVALID_ARG"]
+    assert call_route(L, G480, scale=0.0) == E["FVATTN_ERR_INVALID_ARG"]
+    assert call_route(L, G480, mask=0x3004) == E["FVATTN_ERR_UNSUPPORTED"]     # misaligned
+    bad_d = fv.Geometry(1, 12, 21, 30, 52, 96, 1, 8, 16)
+    assert call_route(L, bad_d) == E["FVATTN_ERR_UNSUPPORTED"]
+    big_block = fv.Geometry(1, 1, 4, 16, 16, 128, 2, 8, 16)        # 256 tokens per block
+    assert call_route(L, big_block) == E["FVATTN_ERR_UNSUPPORTED"]
+    zero = fv.Geometry(1, 0, 4, 16, 16, 128, 1, 8, 16)
+    assert call_route(L, zero) == E["FVATTN_ERR_INVALID_ARG"]
+    assert L.fvattn_route(None, 0x1000, 0x2000, 0.9, 4, 0.1, 0x3000, 0x4000, None) == E["FVATTN_ERR_INVALID_ARG"]
+    cg = G480.c()
+    # attention: missing mask, missing / short workspace
+    assert L.fvattn_block_sparse_attn(ctypes.byref(cg), 0x1000, 0x2000, 0x3000, None, 0.1, 0x4000,
+                                      0x5000, 0x6000, 1 << 20, None, None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert L.fvattn_dense_attn(ctypes.byref(cg), 0x1000, 0x2000, 0x3000, 0.1, 0x4000, 0x5000,
+                               None, 1 << 20, None, None) == E["FVATTN_ERR_WORKSPACE"]
+    assert L.fvattn_dense_attn(ctypes.byref(cg), 0x1000, 0x2000, 0x3000, 0.1, 0x4000, 0x5000,
+                               0x6000, 64, None, None) == E["FVATTN_ERR_WORKSPACE"]
+    assert L.fvattn_block_pool(ctypes.byref(cg), 0x1000, None, 0x3000, 0x4000, None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert L.fvattn_device_status(None, None) == E["FVATTN_ERR_INVALID_ARG"]
+
+
+def test_status_strings(L):
+    for code in range(6):
+        assert fv.fvattn_status_string(code)
+    assert fv.fvattn_status_string(99) == "unknown status"
+
+
+def test_binding_raises_without_cuda_tensors(L):
+    import torch
+    q = torch.zeros(1, 2, 256, 64, dtype=torch.bfloat16)
+    g = fv.Geometry(1, 2, 4, 8, 8, 64, 2, 4, 4)
+    with pytest.raises(ValueError):
+        fv.fvattn_block_pool(g, q, q, torch.zeros(1, 2, 8, 64), torch.zeros(1, 2, 8, 64), stream=0)
