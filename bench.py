@@ -185,6 +185,13 @@ def run_ours(args, rank, world, local_rank):
     if fv.fvattn_device_status(buf.workspace, stream) != 0:
         raise RuntimeError("attention kernel reported a timeout")
 
+    if args.layer_only:
+        ms_step = total_ms / args.steps
+        return {"metric": METRIC, "value": round(eff * world / (ms_step * 1e-3) / 1e12, 3), "unit": UNIT,
+                "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+                "ms_per_step": round(ms_step, 4), "attn_ms": round(statistics.mean(t_attn), 4),
+                "layer_only": True}
+
     # dense baseline (p = 1 through the same kernel), same protocol
     dense_t = []
     for i in range(max(args.warmup, 3) + min(args.steps, 10)):
@@ -379,6 +386,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", action="store_true", help="also time the 15 p/k points (config 5)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--layer-only", action="store_true",
+                    help="time the layer steps only (no dense, e2e or CPU legs); for profilers")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))
@@ -398,7 +407,7 @@ def main():
     try:
         line = run_ours(args, rank, world, local_rank)
         if rank == 0:
-            if world == 1 and not args.no_cpu_baseline:
+            if world == 1 and not (args.no_cpu_baseline or args.layer_only):
                 line["cpu_baseline"] = cpu_baseline(W.WAN21_480P, W.generate(W.WAN21_480P))
             print(json.dumps(line), flush=True)
         if args.sweep and rank == 0:
