@@ -33,14 +33,17 @@ LIB_PATH = os.path.join(_HERE, "libfvattn.so")
 
 FVATTN_OK = 0
 STATUS_NAMES = {0: "FVATTN_OK", 1: "FVATTN_ERR_INVALID_ARG", 2: "FVATTN_ERR_UNSUPPORTED",
-                3: "FVATTN_ERR_WORKSPACE", 4: "FVATTN_ERR_CUDA", 5: "FVATTN_ERR_DEVICE_TIMEOUT"}
+                3: "FVATTN_ERR_WORKSPACE", 4: "FVATTN_ERR_CUDA", 5: "FVATTN_ERR_DEVICE_TIMEOUT",
+                6: "FVATTN_ERR_DEVICE"}
 
 
 class FvattnError(RuntimeError):
     def __init__(self, fn: str, status: int):
         self.status = status
-        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} "
-                         f"({fvattn_status_string(status)})")
+        detail = fvattn_status_string(status)
+        if status == 4:
+            detail += ": " + lib().fvattn_last_cuda_error().decode()
+        super().__init__(f"{fn} failed: {STATUS_NAMES.get(status, status)} ({detail})")
 
 
 class _CGeom(ctypes.Structure):
@@ -95,6 +98,7 @@ _SIGS = {
                                          ctypes.c_void_p, ctypes.c_void_p]),
     "fvattn_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "fvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
+    "fvattn_last_cuda_error": (ctypes.c_char_p, []),
 }
 
 

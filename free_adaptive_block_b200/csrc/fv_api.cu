@@ -13,6 +13,14 @@ namespace {
 
 using fv::Geo;
 
+thread_local cudaError_t g_last_cuda_error = cudaSuccess;
+
+fvattn_status_t cuda_status(cudaError_t e) {
+  if (e == cudaSuccess) return FVATTN_OK;
+  g_last_cuda_error = e;
+  return FVATTN_ERR_CUDA;
+}
+
 constexpr int kMaxBlocks = 2048;   // route keeps a row of nB scores per warp in shared memory
 
 fvattn_status_t make_geo(const fvattn_geom_t* gi, Geo* g) {
@@ -24,6 +32,7 @@ fvattn_status_t make_geo(const fvattn_geom_t* gi, Geo* g) {
   if (static_cast<long long>(gi->bt) * gi->bh * gi->bw > 128) return FVATTN_ERR_UNSUPPORTED;
   const long long N = static_cast<long long>(gi->T) * gi->Hs * gi->Ws;
   if (N >= (1LL << 31)) return FVATTN_ERR_UNSUPPORTED;
+  if (gi->Ws > 65535 || gi->Hs > 65535 || gi->T > 32767) return FVATTN_ERR_UNSUPPORTED;
   Geo r;
   r.B = gi->B; r.H = gi->H; r.T = gi->T; r.Hs = gi->Hs; r.Ws = gi->Ws; r.d = gi->d;
   r.bt = gi->bt; r.bh = gi->bh; r.bw = gi->bw;
@@ -36,6 +45,8 @@ fvattn_status_t make_geo(const fvattn_geom_t* gi, Geo* g) {
   if (static_cast<long long>(gi->B) * gi->H * N * gi->d >= (1LL << 40)) return FVATTN_ERR_UNSUPPORTED;
   r.nB = static_cast<int>(nB);
   r.words = (r.nB + 31) / 32;
+  r.r_nBx = 1.0f / static_cast<float>(r.nBx);
+  r.r_plane = 1.0f / static_cast<float>(r.nBy * r.nBx);
   r.N = static_cast<int>(N);
   *g = r;
   return FVATTN_OK;
@@ -110,16 +121,15 @@ fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, 
   if (ws == nullptr || ws_bytes < fv::attn_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
   if (reinterpret_cast<uintptr_t>(ws) & 15u) return FVATTN_ERR_UNSUPPORTED;
   const int nsm = current_num_sms();
-  if (nsm <= 0) return FVATTN_ERR_CUDA;
+  if (nsm <= 0) return cuda_status(cudaGetLastError() == cudaSuccess ? cudaErrorNoDevice : cudaGetLastError());
   const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
   fv::AttnMaps maps;
   if (!encode_map(&maps.q, q, g, g.bw) || !encode_map(&maps.qe, q, g, rx_edge) ||
       !encode_map(&maps.k, k, g, g.bw) || !encode_map(&maps.ke, k, g, rx_edge) ||
       !encode_map(&maps.v, v, g, g.bw) || !encode_map(&maps.ve, v, g, rx_edge))
     return FVATTN_ERR_CUDA;
-  const cudaError_t e = fv::launch_attn(g, maps, mask, scale, out, lse, ws, busy, nsm,
-                                        reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(fv::launch_attn(g, maps, mask, scale, out, lse, ws, busy, nsm,
+                                     reinterpret_cast<cudaStream_t>(stream)));
 }
 
 }  // namespace
@@ -142,8 +152,7 @@ fvattn_status_t fvattn_block_pool(const fvattn_geom_t* gi, const void* q, const 
   FV_CHECK(check_ptr(k));
   FV_CHECK(check_ptr(q_pool));
   FV_CHECK(check_ptr(k_pool));
-  const cudaError_t e = fv::launch_pool(g, q, k, q_pool, k_pool, reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(fv::launch_pool(g, q, k, q_pool, k_pool, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fvattn_status_t fvattn_route(const fvattn_geom_t* gi, const float* q_pool, const float* k_pool,
@@ -158,9 +167,8 @@ fvattn_status_t fvattn_route(const fvattn_geom_t* gi, const float* q_pool, const
   if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
   if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
-  const cudaError_t e = fv::launch_route(g, q_pool, k_pool, p, k_floor, scale, mask, counts,
-                                         reinterpret_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? FVATTN_OK : FVATTN_ERR_CUDA;
+  return cuda_status(fv::launch_route(g, q_pool, k_pool, p, k_floor, scale, mask, counts,
+                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t fvattn_attn_workspace_size(const fvattn_geom_t* gi) {
@@ -190,10 +198,17 @@ fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stre
   if (workspace == nullptr) return FVATTN_ERR_INVALID_ARG;
   uint32_t hdr[2] = {0, 0};
   cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
-  if (cudaMemcpyAsync(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, st) != cudaSuccess)
-    return FVATTN_ERR_CUDA;
-  if (cudaStreamSynchronize(st) != cudaSuccess) return FVATTN_ERR_CUDA;
-  return (hdr[1] & fv::kErrTimeout) ? FVATTN_ERR_DEVICE_TIMEOUT : FVATTN_OK;
+  fvattn_status_t s = cuda_status(cudaMemcpyAsync(hdr, workspace, sizeof(hdr), cudaMemcpyDeviceToHost, st));
+  if (s != FVATTN_OK) return s;
+  s = cuda_status(cudaStreamSynchronize(st));
+  if (s != FVATTN_OK) return s;
+  if (hdr[1] & fv::kErrTimeout) return FVATTN_ERR_DEVICE_TIMEOUT;
+  if (hdr[1] & fv::kErrLayout) return FVATTN_ERR_DEVICE;
+  return FVATTN_OK;
+}
+
+const char* fvattn_last_cuda_error(void) {
+  return g_last_cuda_error == cudaSuccess ? "no error" : cudaGetErrorString(g_last_cuda_error);
 }
 
 const char* fvattn_status_string(fvattn_status_t s) {
@@ -204,6 +219,7 @@ const char* fvattn_status_string(fvattn_status_t s) {
     case FVATTN_ERR_WORKSPACE: return "workspace missing or too small";
     case FVATTN_ERR_CUDA: return "CUDA call failed";
     case FVATTN_ERR_DEVICE_TIMEOUT: return "a kernel gave up a bounded wait";
+    case FVATTN_ERR_DEVICE: return "a kernel found its shared-memory layout misaligned and did no work";
   }
   return "unknown status";
 }

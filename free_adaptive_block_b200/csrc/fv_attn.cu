@@ -28,16 +28,70 @@
 
 namespace fv {
 
-constexpr int kAttnThreads = 192;
+constexpr int kSoftWarps = 8;          // softmax warps: two per TMEM lane quarter
+// Three warpgroups: warps 0-3 (producer, MMA issuer, two idle warps) and two softmax
+// warpgroups (warps 4-7 and 8-11).  Launched at 168 registers a thread (the register
+// file is split per SM partition, and each partition holds one warp of each group);
+// setmaxnreg then moves registers from the first group to the softmax groups:
+// 128 * 80 + 256 * 208 = 63488 <= 384 * 168 = 64512.
+constexpr int kAttnThreads = 384;
+constexpr int kRegsCtl = 80;
+constexpr int kRegsSoft = 208;
+static_assert(128 * kRegsCtl + 256 * kRegsSoft <= kAttnThreads * 168, "register split exceeds the launch budget");
 constexpr int kNK = 3;                 // K ring depth
 constexpr int kNV = 3;                 // V ring depth
 constexpr int kTR = 2;                 // tile-id ring depth
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle column)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;          // S buffers: columns [0,128) and [128,256)
-constexpr uint32_t kColO = 256;        // O accumulator: [256, 256 + d)
-constexpr uint32_t kColP = 384;        // P buffers (bf16 pairs): [384,448) and [448,512)
+constexpr uint32_t kColS = 0;          // S of chain c: columns [128c, 128c+128); P (bf16 pairs) over its first 64
+constexpr uint32_t kColO = 256;        // O of chain c: columns [256 + d*c, 256 + d*c + d)
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
+#ifndef FV_POLY_EVERY
+#define FV_POLY_EVERY 0
+#endif
+// When nonzero, one exponential pair in kPolyEvery (interior blocks) goes to the FMA
+// pipe (ex2_poly2) instead of the MUFU unit.  Off by default: measured slower so far.
+constexpr int kPolyEvery = FV_POLY_EVERY;
+
+// True in exactly one lane of the (converged) warp.
+__device__ __forceinline__ bool elect_one() {
+  uint32_t pred;
+  asm volatile(
+      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
+      : "=r"(pred));
+  return pred != 0;
+}
+
+__device__ __forceinline__ float max3f(float a, float b, float c) {
+  float r;
+  asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
+  return r;
+}
+
+// 2^x for a pair of x <= 8 on the FMA pipe (Blackwell f32x2 arithmetic), for the P
+// values of the online softmax.  Cody-Waite style range reduction x = j + f with
+// j = round(x), f in [-1/2, 1/2] (adding 1.5 * 2^23 leaves j in the low mantissa
+// bits), a degree-3 polynomial for 2^f whose coefficients are this file's own minimax
+// (Remez exchange) fit of the relative error on [-1/2, 1/2] (max relative error
+// 7.5e-5, far below the 2^-9 of the bf16 P it feeds), and 2^j added to the exponent
+// field with one integer multiply-add.  x is clamped at -125 so the exponent field
+// cannot underflow; 2^-125 is 2e-38, nothing next to the row's terms.
+__device__ __forceinline__ void ex2_poly2(float xa, float xb, float& ya, float& yb) {
+  const uint64_t x = f32x2(fmaxf(xa, -125.0f), fmaxf(xb, -125.0f));
+  const uint64_t magic = f32x2(12582912.0f, 12582912.0f);
+  const uint64_t t = fadd2(x, magic);
+  const uint64_t jf = fsub2(t, magic);
+  const uint64_t f = fsub2(x, jf);
+  uint64_t p = ffma2(f32x2(0.0551716685295105f, 0.0551716685295105f), f,
+                     f32x2(0.2426111251115799f, 0.2426111251115799f));
+  p = ffma2(p, f, f32x2(0.6932609677314758f, 0.6932609677314758f));
+  p = ffma2(p, f, f32x2(0.9999280571937561f, 0.9999280571937561f));
+  float pa, pb, ta, tb;
+  unpack_f32x2(p, pa, pb);
+  unpack_f32x2(t, ta, tb);
+  ya = __uint_as_float(__float_as_uint(ta) * 8388608u + __float_as_uint(pa));
+  yb = __uint_as_float(__float_as_uint(tb) * 8388608u + __float_as_uint(pb));
+}
 
 struct AttnParams {
   Geo g;
@@ -55,20 +109,32 @@ struct __align__(8) AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kNK], k_empty[kNK];
   uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[2], s_empty[2];
+  uint64_t s_full[2];     // per softmax chain
   uint64_t p_full[2];
-  uint64_t pv_done, o_empty;
+  uint64_t pv_done[2], o_empty;
+  uint64_t xbar[4];       // end-of-tile (max, sum) exchange, per TMEM lane quarter: written
+  uint64_t xread[4];      //   ... and read by both warps of the quarter pair
   uint64_t t_full[kTR], t_empty[kTR];
   uint64_t fin;
   int tile[kTR];
+  uint32_t mrow[kTR][64]; // the tile's mask row (nB <= 2048), read by every role
   uint32_t tmem_base;
   int abort;
+  float xm[2][128];       // [chain][row], guarded by xbar / xread
+  float xl[2][128];
 };
 
 template <int D>
 __host__ __device__ constexpr int tile_bytes() { return (D / 64) * kChunkBytes; }
+// Dynamic shared memory: Q | K ring | V ring (each 1024-byte aligned for the 128-byte
+// swizzle) followed by the barrier block.  The dynamic window starts right after the
+// 1 KB the hardware reserves per CTA, which is 1024-byte aligned; the kernel checks
+// it and reports an error instead of running misaligned.
 template <int D>
-__host__ __device__ constexpr int attn_smem_bytes() { return tile_bytes<D>() * (1 + kNK + kNV) + 1024; }
+__host__ __device__ constexpr int attn_smem_bytes() {
+  return tile_bytes<D>() * (1 + kNK + kNV) + static_cast<int>(sizeof(AttnBars));
+}
+static_assert(attn_smem_bytes<128>() <= 232448, "attention kernel exceeds 227 KB of shared memory");
 
 // Iterates the set bits of a mask row in ascending order (or every block when dense).
 struct KvIter {
@@ -86,7 +152,7 @@ struct KvIter {
     while (bits == 0) {
       ++w;
       if (w >= words) return -1;
-      bits = __ldg(row + w);
+      bits = row[w];
     }
     const int b = __ffs(bits) - 1;
     bits &= bits - 1;
@@ -107,8 +173,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const AttnParams prm) {
   constexpr int NCH = D / 64;              // 64-column chunks per row
   constexpr int TILE = tile_bytes<D>();
-  extern __shared__ unsigned char attn_dsm[];
-  __shared__ AttnBars bars;
+  extern __shared__ __align__(1024) unsigned char attn_dsm[];
+  AttnBars& bars = *reinterpret_cast<AttnBars*>(attn_dsm + TILE * (1 + kNK + kNV));
 
   const uint64_t t_start = globaltimer();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
@@ -117,9 +183,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   volatile int* abort = &bars.abort;
 
   // 1024-byte aligned operand area: Q | K ring | V ring
-  const uint32_t dsm0 = smem_u32(attn_dsm);
-  const uint32_t base = (dsm0 + 1023u) & ~1023u;
-  unsigned char* gbase = attn_dsm + (base - dsm0);
+  const uint32_t base = smem_u32(attn_dsm);
+  if (base & 1023u) {                      // uniform over the CTA: nothing launched yet
+    if (threadIdx.x == 0) atomicOr(err, kErrLayout);
+    return;
+  }
+  unsigned char* gbase = attn_dsm;
   const uint32_t sQ = base;
   auto sK = [&](int s) { return base + static_cast<uint32_t>(TILE * (1 + s)); };
   auto sV = [&](int s) { return base + static_cast<uint32_t>(TILE * (1 + kNK + s)); };
@@ -131,12 +200,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kNV; ++i) { mbar_init(&bars.v_full[i], 1); mbar_init(&bars.v_empty[i], 1); }
     for (int i = 0; i < 2; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_empty[i], 4);
-      mbar_init(&bars.p_full[i], 4);
+      mbar_init(&bars.p_full[i], kSoftWarps / 2);
     }
-    mbar_init(&bars.pv_done, 1);
-    mbar_init(&bars.o_empty, 4);
-    for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 5); }
+    for (int i = 0; i < 4; ++i) { mbar_init(&bars.xbar[i], 2); mbar_init(&bars.xread[i], 2); }
+    mbar_init(&bars.pv_done[0], 1);
+    mbar_init(&bars.pv_done[1], 1);
+    mbar_init(&bars.o_empty, kSoftWarps);
+    for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 1 + kSoftWarps); }
     mbar_init(&bars.fin, 1);
     bars.abort = 0;
     fence_barrier_init();
@@ -165,131 +235,196 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
   uint32_t kc = 0, vc = 0, qc = 0;   // producer-side counters (also used in the drain)
 
-  if (warp == 0) {
+  if (warp < 4) {
+   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(kRegsCtl));
+   // The producer and MMA warps run their loops with all 32 lanes converged, so that
+   // tile ids, coordinates and descriptors are warp-uniform; one elected lane issues
+   // each TMA copy, MMA and commit.
+   auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
+     return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err));
+   };
+   if (warp == 0) {
     // ------------------------------------------------------------ TMA producer
-    if (lane == 0) {
-      uint32_t tcount = 0;
-      bool ok = true;
-      while (ok) {
-        const int pos = static_cast<int>(atomicAdd(prm.hdr, 1u));
-        const int tile = pos < prm.ntiles ? __ldg(prm.order + pos) : -1;
-        const int slot = tcount % kTR;
-        if (!mbar_wait(&bars.t_empty[slot], ((tcount / kTR) & 1) ^ 1, abort, err)) break;
+    uint32_t tcount = 0;
+    bool ok = true;
+    while (ok) {
+      int pos = 0;
+      if (lane == 0) pos = static_cast<int>(atomicAdd(prm.hdr, 1u));
+      pos = __shfl_sync(0xffffffffu, pos, 0);
+      const int tile = pos < prm.ntiles ? __ldg(prm.order + pos) : -1;
+      const int slot = tcount % kTR;
+      if (!wwait(&bars.t_empty[slot], ((tcount / kTR) & 1) ^ 1)) break;
+      if (tile >= 0 && prm.mask != nullptr) {
+        const uint32_t* src = prm.mask + static_cast<size_t>(tile) * g.words;
+        for (int w = lane; w < g.words; w += 32) bars.mrow[slot][w] = __ldg(src + w);
+      }
+      __syncwarp();
+      if (lane == 0) {
         bars.tile[slot] = tile;
         mbar_arrive(&bars.t_full[slot]);
-        ++tcount;
-        if (tile < 0) break;
-        int bhi, qb;
-        decode_tile(g, tile, bhi, qb);
-        const BlockInfo qi = block_info(g, qb);
-        if (!mbar_wait(&bars.q_empty, (qc & 1) ^ 1, abort, err)) break;
+      }
+      __syncwarp();
+      ++tcount;
+      if (tile < 0) break;
+      int bhi, qb;
+      decode_tile(g, tile, bhi, qb);
+      const BlockInfo qi = block_info(g, qb);
+      if (!wwait(&bars.q_empty, (qc & 1) ^ 1)) break;
+      if (elect_one()) {
         mbar_arrive_expect_tx(&bars.q_full, static_cast<uint32_t>(qi.rows * 128 * NCH));
         for (int c = 0; c < NCH; ++c)
           tma_load_5d(sQ + c * kChunkBytes, qi.xedge ? &tmQe : &tmQ, &bars.q_full, c * 64,
                       qi.xb * g.bw, qi.yb * g.bh, qi.tb * g.bt, bhi);
-        ++qc;
-        KvIter it;
-        it.init(prm.mask ? prm.mask + static_cast<size_t>(tile) * g.words : nullptr, g.nB, g.words);
-        for (int kb = it.advance(); kb >= 0; kb = it.advance()) {
-          const BlockInfo ki = block_info(g, kb);
-          const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
-          const int ks = kc % kNK;
-          if (!mbar_wait(&bars.k_empty[ks], ((kc / kNK) & 1) ^ 1, abort, err)) { ok = false; break; }
+      }
+      __syncwarp();
+      ++qc;
+      KvIter it;
+      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
+      const int full_rows = g.bt * g.bh * g.bw;
+      for (int kb = it.advance(); kb >= 0; kb = it.advance()) {
+        const BlkEnt ki = blk_of(g, kb);
+        const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
+        const bool xedge = ki.rows != full_rows;
+        const int ks = kc % kNK;
+        if (!wwait(&bars.k_empty[ks], ((kc / kNK) & 1) ^ 1)) { ok = false; break; }
+        if (elect_one()) {
           mbar_arrive_expect_tx(&bars.k_full[ks], bytes);
           for (int c = 0; c < NCH; ++c)
-            tma_load_5d(sK(ks) + c * kChunkBytes, ki.xedge ? &tmKe : &tmK, &bars.k_full[ks],
-                        c * 64, ki.xb * g.bw, ki.yb * g.bh, ki.tb * g.bt, bhi);
-          ++kc;
-          const int vs = vc % kNV;
-          if (!mbar_wait(&bars.v_empty[vs], ((vc / kNV) & 1) ^ 1, abort, err)) { ok = false; break; }
+            tma_load_5d(sK(ks) + c * kChunkBytes, xedge ? &tmKe : &tmK, &bars.k_full[ks],
+                        c * 64, ki.x0, ki.y0, ki.t0, bhi);
+        }
+        __syncwarp();
+        ++kc;
+        const int vs = vc % kNV;
+        if (!wwait(&bars.v_empty[vs], ((vc / kNV) & 1) ^ 1)) { ok = false; break; }
+        if (elect_one()) {
           mbar_arrive_expect_tx(&bars.v_full[vs], bytes);
           for (int c = 0; c < NCH; ++c)
-            tma_load_5d(sV(vs) + c * kChunkBytes, ki.xedge ? &tmVe : &tmV, &bars.v_full[vs],
-                        c * 64, ki.xb * g.bw, ki.yb * g.bh, ki.tb * g.bt, bhi);
-          ++vc;
+            tma_load_5d(sV(vs) + c * kChunkBytes, xedge ? &tmVe : &tmV, &bars.v_full[vs],
+                        c * 64, ki.x0, ki.y0, ki.t0, bhi);
         }
+        __syncwarp();
+        ++vc;
       }
     }
-  } else if (warp == 1) {
+   } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      uint32_t tcount = 0, mkc = 0, mvc = 0, mqc = 0, sc = 0, pc = 0, tiles = 0;
-      const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
-      bool ok = true;
-      while (ok) {
-        const int slot = tcount % kTR;
-        if (!mbar_wait(&bars.t_full[slot], (tcount / kTR) & 1, abort, err)) break;
-        const int tile = bars.tile[slot];
-        mbar_arrive(&bars.t_empty[slot]);
-        ++tcount;
-        if (tile < 0) break;
-        if (!mbar_wait(&bars.q_full, mqc & 1, abort, err)) break;
-        ++mqc;
-        KvIter it;
-        it.init(prm.mask ? prm.mask + static_cast<size_t>(tile) * g.words : nullptr, g.nB, g.words);
-        bool have_prev = false, first_pv = true;
-        int prev_npad = 0;
-        auto issue_pv = [&](int npad) -> bool {
-          const int b = pc & 1;
-          if (!mbar_wait(&bars.p_full[b], (pc >> 1) & 1, abort, err)) return false;
-          const int vs = mvc % kNV;
-          if (!mbar_wait(&bars.v_full[vs], (mvc / kNV) & 1, abort, err)) return false;
-          if (first_pv && !mbar_wait(&bars.o_empty, (tiles & 1) ^ 1, abort, err)) return false;
-          tc_fence_after();
-          for (int kk = 0; kk < npad / 16; ++kk) {
-            const uint64_t bdesc = sdesc_sw128(sV(vs) + kk * 2048, kChunkBytes, 1024);
-            mma_ts(tmem + kColO, tmem + kColP + b * 64 + kk * 8, bdesc, idesc_pv,
-                   (first_pv && kk == 0) ? 0u : 1u);
-          }
-          mma_commit(&bars.v_empty[vs]);
-          mma_commit(&bars.pv_done);
-          ++mvc;
-          ++pc;
-          first_pv = false;
-          return true;
-        };
-        for (int kb = it.advance(); kb >= 0; kb = it.advance()) {
-          const int npad = block_info(g, kb).npad;
-          const int ks = mkc % kNK;
-          if (!mbar_wait(&bars.k_full[ks], (mkc / kNK) & 1, abort, err)) { ok = false; break; }
-          const int b = sc & 1;
-          if (!mbar_wait(&bars.s_empty[b], ((sc >> 1) & 1) ^ 1, abort, err)) { ok = false; break; }
-          tc_fence_after();
-          const uint32_t idesc_s = idesc_bf16_f32(128, npad, 0, 0);
+    // Two softmax chains per tile: chain 0 takes the tile's even KV blocks, chain 1
+    // the odd ones.  Chain c has its own S buffer (P is written back over it) and its
+    // own O accumulator.  Issue order: S_0, S_1, then PV_j, S_j+2 for j = 0, 1, ...
+    // so the chains run half a period apart and one chain's softmax overlaps the other
+    // chain's P.V and S.  S_j+2 overwrites the buffer P_j lives in, so it waits for PV_j.
+    uint32_t tcount = 0, mkc = 0, mvc = 0, mqc = 0, tiles = 0;
+    uint32_t pvn[2] = {0u, 0u};          // P.V products issued per chain (all tiles)
+    const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+    const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
+    const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
+    const uint64_t dV0 = sdesc_sw128(sV(0), kChunkBytes, 1024);
+    bool ok = true;
+    while (ok) {
+      const int slot = tcount % kTR;
+      if (!wwait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
+      const int tile = bars.tile[slot];
+      ++tcount;
+      if (tile < 0) break;
+      if (!wwait(&bars.q_full, mqc & 1)) break;
+      ++mqc;
+      KvIter it;
+      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
+      int npad_r[4] = {0, 0, 0, 0};
+      int ns = 0;
+      bool ended = false;
+      // S_ns: returns false on a failed wait
+      auto try_s = [&]() -> bool {
+        if (ended) return true;
+        const int kb = it.advance();
+        if (kb < 0) { ended = true; return true; }
+        const int j = ns;
+        const int c = j & 1;
+        const int npad = blk_of(g, kb).npad;
+        npad_r[j & 3] = npad;
+        const int ks = mkc % kNK;
+        if (!wwait(&bars.k_full[ks], (mkc / kNK) & 1)) return false;
+        if (pvn[c] > 0 && !wwait(&bars.pv_done[c], (pvn[c] - 1) & 1)) return false;
+        tc_fence_after();
+        const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
+        const uint32_t tS = tmem + kColS + c * 128;
+        const uint32_t idesc_s = idesc_bf16_f32(128, npad, 0, 0);
+        if (elect_one()) {
 #pragma unroll
           for (int kk = 0; kk < D / 16; ++kk) {
-            const uint32_t off = (kk >> 2) * kChunkBytes + (kk & 3) * 32;
-            mma_ss(tmem + kColS + b * 128, sdesc_sw128(sQ + off, 16, 1024),
-                   sdesc_sw128(sK(ks) + off, 16, 1024), idesc_s, kk > 0 ? 1u : 0u);
+            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
+            mma_ss(tS, dQ + off, dK + off, idesc_s, kk > 0 ? 1u : 0u);
           }
-          mma_commit(&bars.s_full[b]);
+          mma_commit(&bars.s_full[c]);
           mma_commit(&bars.k_empty[ks]);
-          ++mkc;
-          ++sc;
-          if (have_prev && !issue_pv(prev_npad)) { ok = false; break; }
-          have_prev = true;
-          prev_npad = npad;
         }
-        if (!ok) break;
-        mma_commit(&bars.q_empty);
-        if (have_prev && !issue_pv(prev_npad)) break;
-        ++tiles;
+        __syncwarp();
+        ++mkc;
+        ++ns;
+        return true;
+      };
+      auto issue_pv = [&](int j) -> bool {
+        const int c = j & 1;
+        const int npad = npad_r[j & 3];
+        if (!wwait(&bars.p_full[c], pvn[c] & 1)) return false;
+        const int vs = mvc % kNV;
+        if (!wwait(&bars.v_full[vs], (mvc / kNV) & 1)) return false;
+        if (j == 0 && !wwait(&bars.o_empty, (tiles & 1) ^ 1)) return false;
+        tc_fence_after();
+        const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
+        const uint32_t tP = tmem + kColS + c * 128;
+        const uint32_t tO = tmem + kColO + c * D;
+        const int nk = npad >> 4;
+        if (elect_one()) {
+#pragma unroll
+          for (int kk = 0; kk < 8; ++kk) {
+            if (kk < nk)
+              mma_ts(tO, tP + kk * 8, dV + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
+                     (j < 2 && kk == 0) ? 0u : 1u);
+          }
+          mma_commit(&bars.v_empty[vs]);
+          mma_commit(&bars.pv_done[c]);
+        }
+        __syncwarp();
+        ++mvc;
+        ++pvn[c];
+        return true;
+      };
+      // PV_j then S_j+2 (same chain): while one chain's softmax runs, the tensor core
+      // works on the other chain's P.V and next S.
+      if (!try_s() || !try_s()) break;
+      for (int j = 0; j < ns && ok; ++j) {
+        if (!issue_pv(j) || !try_s()) { ok = false; break; }
       }
+      if (!ok) break;
+      if (elect_one()) mma_commit(&bars.q_empty);
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.t_empty[slot]);   // done with the tile's mask row
+      ++tiles;
     }
+   }
   } else {
+    asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoft));
     // ------------------------------------------------------------ softmax + epilogue
+    // Warpgroup c = (w-4)/4 runs chain c: the tile's KV blocks j with j % 2 == c.  One
+    // thread per query row (TMEM lane 32*(w%4) + lane), all 128 key columns of a block
+    // in registers.  At the end of a tile the two chains' (max, sum) are exchanged per
+    // row through shared memory and a bounded mbarrier, and chain c writes output
+    // columns [c*d/2, (c+1)*d/2) of  (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
+    const int chain = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    uint32_t tcount = 0, sc = 0, pvc = 0;
+    const uint32_t tS = tmem + lane_off + kColS + chain * 128;
+    const uint32_t tO0 = tmem + lane_off + kColO;
+    uint32_t tcount = 0, sn = 0, xn = 0;
     const float sl2 = prm.scale_log2;
+    const uint64_t sl2x2 = f32x2(sl2, sl2);
     while (true) {
       const int slot = tcount % kTR;
-      bool okw = mbar_wait(&bars.t_full[slot], (tcount / kTR) & 1, abort, err);
-      if (!__all_sync(0xffffffffu, okw)) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.t_full[slot], (tcount / kTR) & 1, abort, err))) break;
       const int tile = bars.tile[slot];
-      __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.t_empty[slot]);
       ++tcount;
       if (tile < 0) break;
       int bhi, qb;
@@ -297,120 +432,174 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const BlockInfo qi = block_info(g, qb);
       const int token = box_row_token(g, qi, row);
 
-      float m_ref = -INFINITY, l = 0.f;
-      int j = 0;
+      float m = -INFINITY, l = 0.f;
+      int nblk = 0, j = 0;
       bool ok = true;
       KvIter it;
-      it.init(prm.mask ? prm.mask + static_cast<size_t>(tile) * g.words : nullptr, g.nB, g.words);
-      for (int kb = it.advance(); kb >= 0; kb = it.advance()) {
-        const BlockInfo ki = block_info(g, kb);
-        // validity of the 128 key columns of this block (same for every row)
+      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
+      for (int kb = it.advance(); kb >= 0; kb = it.advance(), ++j) {
+        if ((j & 1) != chain) continue;
+        const BlkEnt ki = blk_of(g, kb);
+        const bool full = ki.prefix && ki.nvalid >= 128;
         uint32_t vm[4];
         if (ki.prefix) {
 #pragma unroll
-          for (int q = 0; q < 4; ++q) {
-            const int n = ki.nvalid - 32 * q;
-            vm[q] = n >= 32 ? 0xffffffffu : (n <= 0 ? 0u : ((1u << n) - 1u));
+          for (int w4 = 0; w4 < 4; ++w4) {
+            const int nn = ki.nvalid - 32 * w4;
+            vm[w4] = nn >= 32 ? 0xffffffffu : (nn <= 0 ? 0u : ((1u << nn) - 1u));
           }
         } else {
 #pragma unroll
-          for (int q = 0; q < 4; ++q)
-            vm[q] = __ballot_sync(0xffffffffu, box_row_token(g, ki, 32 * q + lane) >= 0);
+          for (int w4 = 0; w4 < 4; ++w4)
+            vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, block_info(g, kb), 32 * w4 + lane) >= 0);
         }
-        const int b = sc & 1;
-        okw = mbar_wait(&bars.s_full[b], (sc >> 1) & 1, abort, err);
-        if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
+        if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[chain], sn & 1, abort, err))) { ok = false; break; }
         tc_fence_after();
+        // The whole row of S in one TMEM round trip (loads are grouped, then one wait:
+        // a TMEM store issued after a load waits for it, so loads and stores are not
+        // interleaved).
         float s[128];
-        // all 128 columns (columns past the block's rows are masked below); loads
-        // under a data-dependent condition would push the row out to local memory
 #pragma unroll
-        for (int c = 0; c < 4; ++c)
-          tmem_ld32(tmem + lane_off + kColS + b * 128 + 32 * c, reinterpret_cast<uint32_t*>(s + 32 * c));
+        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, reinterpret_cast<uint32_t*>(s + 32 * c));
         tmem_wait_ld();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_empty[b]);
-        ++sc;
-
-        float mx = -INFINITY;
+        const int nact = (ki.npad + 31) >> 5;    // 32-column chunks below npad (uniform)
+        if (!full) {
 #pragma unroll
-        for (int c = 0; c < 128; ++c) {
-          const bool v = (vm[c >> 5] >> (c & 31)) & 1u;
-          s[c] = v ? s[c] * sl2 : -INFINITY;
-          mx = fmaxf(mx, s[c]);
+          for (int c = 0; c < 128; ++c) s[c] = ((vm[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
         }
-        float m_use = m_ref, alpha = 1.f;
+        float mq[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) {
+          float mm = max3f(s[32 * r], s[32 * r + 1], s[32 * r + 2]);
+#pragma unroll
+          for (int c = 3; c < 31; c += 2) mm = max3f(mm, s[32 * r + c], s[32 * r + c + 1]);
+          mq[r] = fmaxf(mm, s[32 * r + 31]);
+        }
+        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
+        float alpha = 1.f;
         bool rebase = false;
-        if (j == 0) {
-          m_use = mx;
-        } else if (mx > m_ref + kRebase) {
-          m_use = mx;
-          alpha = ex2(m_ref - mx);
+        if (nblk == 0) {
+          m = mx;
+        } else if (mx > m + kRebase) {
+          alpha = ex2(m - mx);
+          m = mx;
           rebase = true;
         }
-        uint32_t pk[64];
-        float rs = 0.f;
+        // The chain's previous P.V finished before this S was computed (the MMA
+        // warp waits for it), so O can be re-based here directly.
+        if (__any_sync(0xffffffffu, rebase)) {
+          const uint32_t tO = tO0 + chain * D;
+#pragma unroll 1
+          for (int c = 0; c < D / 32; ++c) {
+            uint32_t o[32];
+            tmem_ld32(tO + 32 * c, o);
+            tmem_wait_ld();
 #pragma unroll
-        for (int c = 0; c < 64; ++c) {
-          const float p0 = ex2(s[2 * c] - m_use);
-          const float p1 = ex2(s[2 * c + 1] - m_use);
-          rs += p0 + p1;
-          pk[c] = pack_bf16x2(p0, p1);
-        }
-        l = l * alpha + rs;
-        m_ref = m_use;
-        if (j > 0) {
-          okw = mbar_wait(&bars.pv_done, pvc & 1, abort, err);
-          if (!__all_sync(0xffffffffu, okw)) { ok = false; break; }
-          ++pvc;
-          tc_fence_after();
-          if (__any_sync(0xffffffffu, rebase)) {
-#pragma unroll
-            for (int c = 0; c < D / 32; ++c) {
-              uint32_t o[32];
-              tmem_ld32(tmem + lane_off + kColO + 32 * c, o);
-              tmem_wait_ld();
-#pragma unroll
-              for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-              tmem_st32(tmem + lane_off + kColO + 32 * c, o);
-            }
+            for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
+            tmem_st32(tO + 32 * c, o);
           }
         }
+        // P = 2^(s * scale * log2 e - m), packed to bf16 pairs; stored after all of it
+        // is computed (P column k/2 holds keys k, k+1, over S columns already read).
+        const uint64_t nmx2 = f32x2(-m, -m);
+        uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        uint32_t pk[64];
 #pragma unroll
-        for (int c = 0; c < 2; ++c) tmem_st32(tmem + lane_off + kColP + b * 64 + 32 * c, pk + 32 * c);
+        for (int c32 = 0; c32 < 4; ++c32) {
+          if (c32 < nact) {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) {
+              const int c = 32 * c32 + 2 * e;
+              float x0, x1;
+              unpack_f32x2(ffma2(f32x2(s[c], s[c + 1]), sl2x2, nmx2), x0, x1);
+              float p0, p1;
+              if (full && kPolyEvery > 0 && (e % kPolyEvery) == kPolyEvery - 1) {
+                ex2_poly2(x0, x1, p0, p1);
+              } else {
+                p0 = ex2(x0);
+                p1 = ex2(x1);
+              }
+              acc[e & 3] = fadd2(acc[e & 3], f32x2(p0, p1));
+              pk[16 * c32 + e] = pack_bf16x2(p0, p1);
+            }
+          } else {
+#pragma unroll
+            for (int e = 0; e < 16; ++e) pk[16 * c32 + e] = 0u;
+          }
+        }
+        tmem_st32(tS, pk);
+        tmem_st32(tS + 32, pk + 32);
+        float sa, sb, sc2, sd;
+        unpack_f32x2(fadd2(acc[0], acc[1]), sa, sb);
+        unpack_f32x2(fadd2(acc[2], acc[3]), sc2, sd);
+        l = l * alpha + ((sa + sb) + (sc2 + sd));
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[b]);
-        ++j;
+        if (lane == 0) mbar_arrive(&bars.p_full[chain]);
+        ++sn;
+        ++nblk;
       }
       if (!ok) break;
-      // epilogue: O / l -> out (bf16), lse
-      okw = mbar_wait(&bars.pv_done, pvc & 1, abort, err);
-      if (!__all_sync(0xffffffffu, okw)) break;
-      ++pvc;
+      // ---- epilogue: wait for this chain's last P.V, exchange (m, l) with the partner
+      const int nkv = j;
+      if (nblk > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[chain], (sn - 1) & 1, abort, err))) break;
+      if (xn > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars.xread[quarter], (xn - 1) & 1, abort, err))) break;
+      bars.xm[chain][row] = m;
+      bars.xl[chain][row] = l;
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.xbar[quarter]);
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.xbar[quarter], xn & 1, abort, err))) break;
+      const float m_o = bars.xm[chain ^ 1][row];
+      const float l_o = bars.xl[chain ^ 1][row];
+      __syncwarp();
+      if (lane == 0) mbar_arrive(&bars.xread[quarter]);
+      ++xn;
+      const bool have0 = nkv >= 1, have1 = nkv >= 2;
+      const float m0 = chain == 0 ? m : m_o, m1 = chain == 0 ? m_o : m;
+      const float l0 = chain == 0 ? l : l_o, l1 = chain == 0 ? l_o : l;
+      const float mt = have1 ? fmaxf(m0, m1) : m0;
+      const float a0 = have0 ? ex2(m0 - mt) : 0.f;
+      const float a1 = have1 ? ex2(m1 - mt) : 0.f;
+      const float lt = l0 * a0 + l1 * a1;
+      const float inv = 1.f / lt;
+      const float w0 = a0 * inv, w1 = a1 * inv;
       tc_fence_after();
-      uint32_t o[D];
+      uint4* dst = reinterpret_cast<uint4*>(prm.out + (static_cast<size_t>(bhi) * g.N + (token >= 0 ? token : 0)) * D +
+                                            (D / 2) * chain);
 #pragma unroll
-      for (int c = 0; c < D / 32; ++c) tmem_ld32(tmem + lane_off + kColO + 32 * c, o + 32 * c);
-      tmem_wait_ld();
+      for (int c = 0; c < D / 64; ++c) {
+        uint32_t o0[32], o1[32];
+        tmem_ld32(tO0 + (D / 2) * chain + 32 * c, o0);
+        tmem_ld32(tO0 + D + (D / 2) * chain + 32 * c, o1);
+        tmem_wait_ld();
+        if (token >= 0) {
+#pragma unroll
+          for (int q8 = 0; q8 < 4; ++q8) {
+            float v[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float x1 = have1 ? __uint_as_float(o1[8 * q8 + e]) * w1 : 0.f;
+              v[e] = fmaf(__uint_as_float(o0[8 * q8 + e]), w0, x1);
+            }
+            uint4 wv;
+            wv.x = pack_bf16x2(v[0], v[1]);
+            wv.y = pack_bf16x2(v[2], v[3]);
+            wv.z = pack_bf16x2(v[4], v[5]);
+            wv.w = pack_bf16x2(v[6], v[7]);
+            dst[4 * c + q8] = wv;
+          }
+        }
+      }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(&bars.o_empty);
+      if (lane == 0) {
+        mbar_arrive(&bars.o_empty);
+        mbar_arrive(&bars.t_empty[slot]);   // done with the tile's mask row
+      }
       if (token >= 0) {
-        const float inv = 1.f / l;
-        uint4* dst = reinterpret_cast<uint4*>(prm.out + (static_cast<size_t>(bhi) * g.N + token) * D);
-#pragma unroll
-        for (int c = 0; c < D / 8; ++c) {
-          uint4 w;
-          w.x = pack_bf16x2(__uint_as_float(o[8 * c + 0]) * inv, __uint_as_float(o[8 * c + 1]) * inv);
-          w.y = pack_bf16x2(__uint_as_float(o[8 * c + 2]) * inv, __uint_as_float(o[8 * c + 3]) * inv);
-          w.z = pack_bf16x2(__uint_as_float(o[8 * c + 4]) * inv, __uint_as_float(o[8 * c + 5]) * inv);
-          w.w = pack_bf16x2(__uint_as_float(o[8 * c + 6]) * inv, __uint_as_float(o[8 * c + 7]) * inv);
-          dst[c] = w;
-        }
-        prm.lse[static_cast<size_t>(bhi) * g.N + token] = (m_ref + __log2f(l)) * 0.69314718055994531f;
+        if (chain == 0)
+          prm.lse[static_cast<size_t>(bhi) * g.N + token] = (mt + __log2f(lt)) * 0.69314718055994531f;
       }
     }
   }
@@ -448,22 +637,29 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 
 // ----------------------------------------------------------------------------
 // Schedule prep: one CTA.  Resets the queue counter, the error word and the SM busy
-// record; scores every tile by its issued work, sum over kept blocks of (rows padded
-// to 16 + a per-block overhead), and writes the tile order by decreasing cost
-// (2048 cost buckets, counting sort).  Order inside a bucket is arbitrary; it only
-// affects timing, never results.
+// record, then writes the tile order:
+//   * a tile's cost is its issued work, sum over kept blocks of (rows padded to 16 +
+//     a per-block overhead);
+//   * (b, h) slices are ranked by total cost, heaviest first, and a slice's tiles are
+//     contiguous in the order, heaviest first (counting sort on cost buckets).
+// Grouping by slice keeps the K/V tiles that concurrently running tiles read within a
+// slice or two, which fits in L2; ordering slices and tiles by decreasing cost keeps
+// the longest-processing-time-first tail (the last tiles are the lightest slice's
+// lightest).  Order inside a bucket is arbitrary: it changes timing, never results.
 // ----------------------------------------------------------------------------
 constexpr int kPrepThreads = 1024;
-constexpr int kBuckets = 2048;
+constexpr int kHistCells = 8192;       // slices x cost buckets
+constexpr int kMaxSlices = 1024;
 constexpr int kBlockOverhead = 64;
 
 __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_t* __restrict__ mask,
                                                             uint32_t* hdr, int* order, int* keys,
-                                                            int ntiles, unsigned long long* busy,
-                                                            int nsm) {
-  __shared__ int hist[kBuckets];
+                                                            int ntiles,
+                                                            unsigned long long* busy, int nsm) {
+  __shared__ int hist[kHistCells];
+  __shared__ unsigned long long total[kMaxSlices];
+  __shared__ int rank[kMaxSlices];
   __shared__ uint32_t edge[64];
-  __shared__ int wsum[32];
   const int t = threadIdx.x;
   if (t == 0) { hdr[0] = 0; hdr[1] = 0; }
   if (busy)
@@ -473,6 +669,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
     return;
   }
   const int words = g.words;
+  const int slices = g.B * g.H;
+  // slices beyond the shared tables fall back to one group (plain LPT order)
+  const bool grouped = slices <= kMaxSlices;
+  const int ngroups = grouped ? slices : 1;
+  int nbk = kHistCells / ngroups;
+  nbk = nbk >= 256 ? 256 : (nbk >= 128 ? 128 : (nbk >= 64 ? 64 : (nbk >= 32 ? 32 : (nbk >= 16 ? 16 : 8))));
   for (int w = t; w < words; w += kPrepThreads) {
     uint32_t bits = 0;
     for (int i = 0; i < 32; ++i) {
@@ -481,7 +683,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
     }
     edge[w] = bits;
   }
-  for (int i = t; i < kBuckets; i += kPrepThreads) hist[i] = 0;
+  for (int i = t; i < kHistCells; i += kPrepThreads) hist[i] = 0;
+  for (int i = t; i < ngroups; i += kPrepThreads) total[i] = 0ull;
   __syncthreads();
   const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
   const long long full = ((g.bt * g.bh * g.bw + 15) & ~15) + kBlockOverhead;
@@ -494,37 +697,53 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
       const uint32_t m = __ldg(row + w);
       cost += full * __popc(m) - (full - part) * __popc(m & edge[w]);
     }
-    int key = static_cast<int>(((maxcost - cost) * (kBuckets - 1)) / maxcost);
-    key = min(max(key, 0), kBuckets - 1);
+    int key = static_cast<int>(((maxcost - cost) * nbk) / (maxcost + 1));
+    key = min(max(key, 0), nbk - 1);
     keys[i] = key;
-    atomicAdd(&hist[key], 1);
+    atomicAdd(&total[grouped ? i / g.nB : 0], static_cast<unsigned long long>(cost));
   }
   __syncthreads();
-  // exclusive scan of the histogram: warp 0, 64 buckets per lane
+  for (int h = t; h < ngroups; h += kPrepThreads) {
+    int r = 0;
+    const unsigned long long th = total[h];
+    for (int o = 0; o < ngroups; ++o) {
+      const unsigned long long to = total[o];
+      r += (to > th) || (to == th && o < h);
+    }
+    rank[h] = r;
+  }
+  __syncthreads();
+  for (int i = t; i < ntiles; i += kPrepThreads)
+    atomicAdd(&hist[rank[grouped ? i / g.nB : 0] * nbk + keys[i]], 1);
+  __syncthreads();
+  // exclusive scan of the histogram in (slice rank, bucket) order: warp 0, 256 cells per lane
+  const int cells = ngroups * nbk;
+  const int per = (cells + 31) / 32;
   if (t < 32) {
     int run = 0;
-    for (int i = 0; i < kBuckets / 32; ++i) run += hist[t * (kBuckets / 32) + i];
+    for (int i = 0; i < per; ++i) {
+      const int idx = t * per + i;
+      if (idx < cells) run += hist[idx];
+    }
     int incl = run;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
       const int v = __shfl_up_sync(0xffffffffu, incl, off);
       if (t >= off) incl += v;
     }
-    wsum[t] = incl - run;
-  }
-  __syncthreads();
-  if (t < 32) {
-    int acc = wsum[t];
-    for (int i = 0; i < kBuckets / 32; ++i) {
-      const int idx = t * (kBuckets / 32) + i;
-      const int c = hist[idx];
-      hist[idx] = acc;
-      acc += c;
+    int acc = incl - run;
+    for (int i = 0; i < per; ++i) {
+      const int idx = t * per + i;
+      if (idx < cells) {
+        const int c = hist[idx];
+        hist[idx] = acc;
+        acc += c;
+      }
     }
   }
   __syncthreads();
   for (int i = t; i < ntiles; i += kPrepThreads) {
-    const int pos = atomicAdd(&hist[keys[i]], 1);
+    const int pos = atomicAdd(&hist[rank[grouped ? i / g.nB : 0] * nbk + keys[i]], 1);
     order[pos] = i;
   }
 }

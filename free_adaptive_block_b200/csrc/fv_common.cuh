@@ -19,7 +19,22 @@ struct Geo {
   int bt, bh, bw;
   int nBt, nBy, nBx, nB, words;
   int N;
+  float r_nBx, r_plane;   // 1/nBx and 1/(nBy*nBx), for division by multiplication
 };
+
+// a / d for 0 <= a < 2^24, 0 < d < 2^16, given rd ~ 1/d: the float estimate is off by
+// at most one, and one correction step makes it exact.
+__host__ __device__ inline int div_r(int a, int d, float rd) {
+#ifdef __CUDA_ARCH__
+  int q = __float2int_rz(__int2float_rn(a) * rd);
+#else
+  int q = static_cast<int>(static_cast<float>(a) * rd);
+#endif
+  const int r = a - q * d;
+  if (r < 0) --q;
+  else if (r >= d) ++q;
+  return q;
+}
 
 struct BlockInfo {
   int tb, yb, xb;    // block coordinates
@@ -34,9 +49,9 @@ struct BlockInfo {
 __host__ __device__ inline BlockInfo block_info(const Geo& g, int j) {
   BlockInfo b;
   const int per_t = g.nBy * g.nBx;
-  b.tb = j / per_t;
+  b.tb = div_r(j, per_t, g.r_plane);
   const int rem = j - b.tb * per_t;
-  b.yb = rem / g.nBx;
+  b.yb = div_r(rem, g.nBx, g.r_nBx);
   b.xb = rem - b.yb * g.nBx;
   b.rt = min(g.bt, g.T - b.tb * g.bt);
   b.ry = min(g.bh, g.Hs - b.yb * g.bh);
@@ -47,6 +62,24 @@ __host__ __device__ inline BlockInfo block_info(const Geo& g, int j) {
   b.nvalid = b.rt * b.ry * b.rx;   // the real token count (a prefix of the box when `prefix`)
   b.xedge = b.rx < g.bw;
   return b;
+}
+
+// What the attention roles need of key block j (TMA coordinates, rows, real tokens).
+struct BlkEnt {
+  int x0, y0, t0, rows, npad, nvalid;
+  bool prefix;
+};
+__host__ __device__ inline BlkEnt blk_of(const Geo& g, int j) {
+  const BlockInfo b = block_info(g, j);
+  BlkEnt e;
+  e.x0 = b.xb * g.bw;
+  e.y0 = b.yb * g.bh;
+  e.t0 = b.tb * g.bt;
+  e.rows = b.rows;
+  e.npad = b.npad;
+  e.nvalid = b.nvalid;
+  e.prefix = b.prefix;
+  return e;
 }
 
 // Row r of a loaded box (rows ordered (tt, yy, xx), x compact) -> token index, or -1
@@ -116,7 +149,7 @@ __device__ __forceinline__ uint32_t smid() {
 }
 
 // Status word bits written to the workspace when a kernel gives up a wait.
-enum : uint32_t { kErrTimeout = 1u };
+enum : uint32_t { kErrTimeout = 1u, kErrLayout = 2u };
 
 // A bounded wait on an mbarrier phase.  Returns false (after raising *abort and the
 // global error word) when the phase has not completed within `limit_ns`, or when
@@ -250,11 +283,85 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t* r) {
       FV_W8(0), FV_W8(8), FV_W8(16), FV_W8(24)
       : "memory");
 }
+
+// 16x256b shape: a warp reads 16 lanes x (8 columns per repetition); thread t holds,
+// for repetition i, (lane t/4, columns 8i + 2(t%4) + {0,1}) in r[4i], r[4i+1] and
+// (lane t/4 + 8, the same columns) in r[4i+2], r[4i+3].
+__device__ __forceinline__ void tmem_ld_16x256b_x8(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31}, [%32];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x256b_x8(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x8.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+__device__ __forceinline__ void tmem_ld_16x256b_x16(uint32_t taddr, uint32_t* r) {
+  asm volatile("tcgen05.ld.sync.aligned.16x256b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63}, [%64];"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]), "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]), "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]), "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31]), "=r"(r[32]), "=r"(r[33]), "=r"(r[34]), "=r"(r[35]), "=r"(r[36]), "=r"(r[37]), "=r"(r[38]), "=r"(r[39]), "=r"(r[40]), "=r"(r[41]), "=r"(r[42]), "=r"(r[43]), "=r"(r[44]), "=r"(r[45]), "=r"(r[46]), "=r"(r[47]), "=r"(r[48]), "=r"(r[49]), "=r"(r[50]), "=r"(r[51]), "=r"(r[52]), "=r"(r[53]), "=r"(r[54]), "=r"(r[55]), "=r"(r[56]), "=r"(r[57]), "=r"(r[58]), "=r"(r[59]), "=r"(r[60]), "=r"(r[61]), "=r"(r[62]), "=r"(r[63])
+               : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st_16x256b_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x256b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32,%33,%34,%35,%36,%37,%38,%39,%40,%41,%42,%43,%44,%45,%46,%47,%48,%49,%50,%51,%52,%53,%54,%55,%56,%57,%58,%59,%60,%61,%62,%63,%64};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31]), "r"(r[32]), "r"(r[33]), "r"(r[34]), "r"(r[35]), "r"(r[36]), "r"(r[37]), "r"(r[38]), "r"(r[39]), "r"(r[40]), "r"(r[41]), "r"(r[42]), "r"(r[43]), "r"(r[44]), "r"(r[45]), "r"(r[46]), "r"(r[47]), "r"(r[48]), "r"(r[49]), "r"(r[50]), "r"(r[51]), "r"(r[52]), "r"(r[53]), "r"(r[54]), "r"(r[55]), "r"(r[56]), "r"(r[57]), "r"(r[58]), "r"(r[59]), "r"(r[60]), "r"(r[61]), "r"(r[62]), "r"(r[63])
+               : "memory");
+}
+template <int N>
+__device__ __forceinline__ void tmem_ld_16x256b(uint32_t taddr, uint32_t* r) {
+  if constexpr (N == 16) tmem_ld_16x256b_x16(taddr, r); else tmem_ld_16x256b_x8(taddr, r);
+}
+template <int N>
+__device__ __forceinline__ void tmem_st_16x256b(uint32_t taddr, const uint32_t* r) {
+  if constexpr (N == 16) tmem_st_16x256b_x16(taddr, r); else tmem_st_16x256b_x8(taddr, r);
+}
+// 16x128b shape: for repetition j, thread t writes (lane t/4, column 4j + t%4) from
+// r[2j] and (lane t/4 + 8, the same column) from r[2j+1].
+__device__ __forceinline__ void tmem_st_16x128b_x16(uint32_t taddr, const uint32_t* r) {
+  asm volatile("tcgen05.st.sync.aligned.16x128b.x16.b32 [%0], {%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16,%17,%18,%19,%20,%21,%22,%23,%24,%25,%26,%27,%28,%29,%30,%31,%32};"
+               :: "r"(taddr), "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+               : "memory");
+}
+
+__device__ __forceinline__ void tmem_st16(uint32_t taddr, const uint32_t* r) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x16.b32 [%0], "
+      "{%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15,%16};" ::"r"(taddr),
+      FV_W8(0), FV_W8(8)
+      : "memory");
+}
+
 __device__ __forceinline__ void tmem_wait_ld() {
   asm volatile("tcgen05.wait::ld.sync.aligned;" ::: "memory");
 }
 __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
+}
+
+// Packed pairs of fp32 (Blackwell f32x2 arithmetic: two lanes per instruction).
+__device__ __forceinline__ uint64_t f32x2(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void unpack_f32x2(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
+__device__ __forceinline__ uint64_t fsub2(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("sub.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
 }
 
 __device__ __forceinline__ float ex2(float x) {

@@ -116,18 +116,18 @@ cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, f
 }
 
 // ----------------------------------------------------------------------------
-// Routing: one CTA per (b*h, 8 query blocks); warp w owns query block
-// blockIdx.x * 8 + w.  Logits come from key tiles of 32 blocks staged transposed in
-// shared memory (lane = key block).  Then, per warp: softmax over all key blocks,
-// and a bitwise search for the Top-p cut over an order-preserving integer key of
-// the logits, so no sort is needed:
-//   u* = the largest key with mass(key >= u*) >= p  -> the key of the m_p-th block,
+// Routing: one CTA per (b*h, 16 query blocks); warp w owns query blocks 2w and 2w+1
+// of the CTA.  Logits come from key tiles of 32 blocks staged in shared memory (lane =
+// key block, 16-byte loads along d).  Then, per query block, with the row's logits and
+// scores held in registers: softmax over all key blocks, and a bitwise search for the
+// Top-p cut over an order-preserving integer key of the logits, so no sort is needed:
+//   u* = the largest key with mass(key >= u*) >= p  -> the key of the m_p-th block;
 // equal keys are taken in ascending block index.  The Top-k floor lengthens the
 // prefix with a second search on counts.  Reductions are warp shuffles in a fixed
 // order, so the result is deterministic.
 // ----------------------------------------------------------------------------
-constexpr int kRouteRows = 8;
-constexpr int kRouteThreads = kRouteRows * 32;
+constexpr int kRouteRows = 16;
+constexpr int kRouteThreads = 256;
 
 __device__ __forceinline__ uint32_t order_key(float x) {
   const uint32_t u = __float_as_uint(x);
@@ -150,107 +150,39 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
-template <int D>
-__global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float* __restrict__ qp,
-                                                              const float* __restrict__ kp, float p,
-                                                              int k_floor, float scale,
-                                                              uint32_t* __restrict__ mask,
-                                                              int32_t* __restrict__ counts) {
-  extern __shared__ __align__(16) unsigned char route_smem[];
-  const int words = g.words;
-  const int nBpad = words * 32;
-  float* sQ = reinterpret_cast<float*>(route_smem);                  // [8][D]
-  float* sKT = sQ + kRouteRows * D;                                   // [D][33]
-  uint32_t* sKey = reinterpret_cast<uint32_t*>(sKT + D * 33);         // [8][nBpad]
-  float* sS = reinterpret_cast<float*>(sKey + kRouteRows * nBpad);    // [8][nBpad]
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const int bhi = blockIdx.y;
-  const int nB = g.nB;
-  const int qb = blockIdx.x * kRouteRows + warp;
-  const float* kph = kp + static_cast<size_t>(bhi) * nB * D;
-
-  for (int e = threadIdx.x; e < kRouteRows * D; e += kRouteThreads) {
-    const int r = e / D, dd = e - r * D;
-    const int row = blockIdx.x * kRouteRows + r;
-    sQ[e] = row < nB ? qp[(static_cast<size_t>(bhi) * nB + row) * D + dd] : 0.f;
-  }
-  uint32_t* myKey = sKey + warp * nBpad;
-  float* myS = sS + warp * nBpad;
-  for (int kt = 0; kt < words; ++kt) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < 32 * D; e += kRouteThreads) {
-      const int key = e / D, dd = e - key * D;
-      const int j = kt * 32 + key;
-      sKT[dd * 33 + key] = j < nB ? kph[static_cast<size_t>(j) * D + dd] : 0.f;
-    }
-    __syncthreads();
-    float acc = 0.f;
-    const float* qrow = sQ + warp * D;
-#pragma unroll 16
-    for (int dd = 0; dd < D; ++dd) acc = fmaf(qrow[dd], sKT[dd * 33 + lane], acc);
-    const int j = kt * 32 + lane;
-    const float logit = acc * scale;
-    myKey[j] = j < nB ? order_key(logit) : 0u;
-    myS[j] = j < nB ? logit : -INFINITY;
-  }
-  __syncwarp();
-  if (qb >= nB) return;
-
-  // softmax over the key blocks (fp32)
+// Selection for one query block; the row's logits are in sL[i], i = c*32 + lane.
+template <int MAXW>
+__device__ __forceinline__ void select_row(const float* sL, int nB, int words, int qb, float p,
+                                           int k_floor, uint32_t* mrow, int32_t* cnt_out, int lane) {
+  uint32_t key[MAXW];
+  float sc[MAXW];
   float mx = -INFINITY;
-  for (int c = 0; c < words; ++c) mx = fmaxf(mx, myS[c * 32 + lane]);
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    const int i = c * 32 + lane;
+    const bool v = c < words && i < nB;
+    const float lg = v ? sL[c * 32 + lane] : -INFINITY;
+    key[c] = v ? order_key(lg) : 0u;
+    sc[c] = lg;
+    mx = fmaxf(mx, lg);
+  }
   mx = warp_max(mx);
   float z = 0.f;
-  for (int c = 0; c < words; ++c) {
-    const int i = c * 32 + lane;
-    const float e = i < nB ? expf(myS[i] - mx) : 0.f;
-    myS[i] = e;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    const float e = key[c] ? expf(sc[c] - mx) : 0.f;
+    sc[c] = e;
     z += e;
   }
   z = warp_sum(z);
   const float inv_z = 1.f / z;
   float total = 0.f;
-  for (int c = 0; c < words; ++c) {
-    const int i = c * 32 + lane;
-    const float s = myS[i] * inv_z;
-    myS[i] = s;
-    total += s;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    sc[c] *= inv_z;
+    total += sc[c];
   }
   total = warp_sum(total);
-
-  auto mass_ge = [&](uint32_t u) {
-    float m = 0.f;
-    for (int c = 0; c < words; ++c) {
-      const int i = c * 32 + lane;
-      m += (i < nB && myKey[i] >= u) ? myS[i] : 0.f;
-    }
-    return warp_sum(m);
-  };
-  auto count_ge = [&](uint32_t u) {
-    int n = 0;
-    for (int c = 0; c < words; ++c) {
-      const int i = c * 32 + lane;
-      n += (i < nB && myKey[i] >= u) ? 1 : 0;
-    }
-    return warp_sum_i(n);
-  };
-  auto count_gt_eq = [&](uint32_t u, int& gt, int& eq, float& gt_mass, float& eq_score) {
-    int a = 0, b = 0;
-    float m = 0.f, es = 0.f;
-    for (int c = 0; c < words; ++c) {
-      const int i = c * 32 + lane;
-      if (i < nB) {
-        const uint32_t key = myKey[i];
-        if (key > u) { ++a; m += myS[i]; }
-        if (key == u) { ++b; es = myS[i]; }
-      }
-    }
-    gt = warp_sum_i(a);
-    eq = warp_sum_i(b);
-    gt_mass = warp_sum(m);
-    eq_score = warp_max(es);
-  };
 
   const int floor_k = min(max(k_floor, 0), nB);
   int m_p;
@@ -261,15 +193,26 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
   } else {
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = u | (1u << bit);
-      if (mass_ge(cand) >= p) u = cand;
+      float m = 0.f;
+#pragma unroll
+      for (int c = 0; c < MAXW; ++c) m += key[c] >= cand ? sc[c] : 0.f;
+      if (warp_sum(m) >= p) u = cand;
     }
-    int gt, eq;
-    float gt_mass, eq_s;
-    count_gt_eq(u, gt, eq, gt_mass, eq_s);
-    float acc = gt_mass;
+    int gt = 0, eq = 0;
+    float gm = 0.f, es = 0.f;
+#pragma unroll
+    for (int c = 0; c < MAXW; ++c) {
+      if (key[c] > u) { ++gt; gm += sc[c]; }
+      if (key[c] == u && key[c] != 0u) { ++eq; es = sc[c]; }
+    }
+    gt = warp_sum_i(gt);
+    eq = warp_sum_i(eq);
+    gm = warp_sum(gm);
+    es = warp_max(es);
+    float acc = gm;
     int r = 0;
     while (acc < p && r < eq) {
-      acc += eq_s;
+      acc += es;
       ++r;
     }
     m_p = gt + r;
@@ -278,61 +221,135 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
   const int M = max(max(m_p, floor_k), 1);
   if (M >= nB) {
     u = 0;
-    ties_needed = nB;     // every block
+    ties_needed = nB;     // every block (keys of real blocks are nonzero)
   } else if (M > m_p) {
     uint32_t v = 0;
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = v | (1u << bit);
-      if (count_ge(cand) >= M) v = cand;
+      int n = 0;
+#pragma unroll
+      for (int c = 0; c < MAXW; ++c) n += key[c] >= cand ? 1 : 0;
+      if (warp_sum_i(n) >= M) v = cand;
     }
-    int gt, eq;
-    float gm, es;
-    count_gt_eq(v, gt, eq, gm, es);
+    int gt = 0;
+#pragma unroll
+    for (int c = 0; c < MAXW; ++c) gt += key[c] > v ? 1 : 0;
     u = v;
-    ties_needed = M - gt;
+    ties_needed = M - warp_sum_i(gt);
   }
 
-  uint32_t* mrow = mask + (static_cast<size_t>(bhi) * nB + qb) * words;
   int tie_base = 0, cnt = 0;
-  for (int c = 0; c < words; ++c) {
-    const int i = c * 32 + lane;
-    const bool valid = i < nB;
-    const uint32_t key = valid ? myKey[i] : 0u;
-    const bool tie = valid && key == u;
-    const uint32_t tb = __ballot_sync(0xffffffffu, tie);
-    const int rank = tie_base + __popc(tb & ((1u << lane) - 1u));
-    tie_base += __popc(tb);
-    const bool kept = valid && (key > u || (tie && rank < ties_needed) || i == qb);
-    const uint32_t word = __ballot_sync(0xffffffffu, kept);
-    cnt += __popc(word);
-    if (lane == 0) mrow[c] = word;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    if (c < words) {
+      const int i = c * 32 + lane;
+      const bool valid = key[c] != 0u;
+      const bool tie = valid && key[c] == u;
+      const uint32_t tb = __ballot_sync(0xffffffffu, tie);
+      const int rank = tie_base + __popc(tb & ((1u << lane) - 1u));
+      tie_base += __popc(tb);
+      const bool kept = valid && (key[c] > u || (tie && rank < ties_needed) || i == qb);
+      const uint32_t word = __ballot_sync(0xffffffffu, kept);
+      cnt += __popc(word);
+      if (lane == 0) mrow[c] = word;
+    }
   }
-  if (lane == 0) counts[static_cast<size_t>(bhi) * nB + qb] = cnt;
+  if (lane == 0) *cnt_out = cnt;
+}
+
+template <int D, int MAXW>
+__global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float* __restrict__ qp,
+                                                              const float* __restrict__ kp, float p,
+                                                              int k_floor, float scale,
+                                                              uint32_t* __restrict__ mask,
+                                                              int32_t* __restrict__ counts) {
+  extern __shared__ __align__(16) unsigned char route_smem[];
+  constexpr int KS = D + 4;                                      // padded key row (floats)
+  const int words = g.words;
+  const int nBpad = words * 32;
+  float* sQ = reinterpret_cast<float*>(route_smem);              // [16][D]
+  float* sK = sQ + kRouteRows * D;                               // [32][D + 4]
+  float* sL = sK + 32 * KS;                                      // [16][nBpad]
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int bhi = blockIdx.y;
+  const int nB = g.nB;
+  const int row0 = blockIdx.x * kRouteRows;
+  const float* kph = kp + static_cast<size_t>(bhi) * nB * D;
+
+  for (int e = threadIdx.x; e < kRouteRows * D / 4; e += kRouteThreads) {
+    const int r = e / (D / 4), d4 = e - r * (D / 4);
+    const int row = row0 + r;
+    reinterpret_cast<float4*>(sQ)[e] =
+        row < nB ? reinterpret_cast<const float4*>(qp + (static_cast<size_t>(bhi) * nB + row) * D)[d4]
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  }
+  const float4* q0 = reinterpret_cast<const float4*>(sQ + (2 * warp) * D);
+  const float4* q1 = reinterpret_cast<const float4*>(sQ + (2 * warp + 1) * D);
+  for (int kt = 0; kt < words; ++kt) {
+    __syncthreads();
+    for (int e = threadIdx.x; e < 32 * D / 4; e += kRouteThreads) {
+      const int key = e / (D / 4), d4 = e - key * (D / 4);
+      const int j = kt * 32 + key;
+      reinterpret_cast<float4*>(sK + key * KS)[d4] =
+          j < nB ? reinterpret_cast<const float4*>(kph + static_cast<size_t>(j) * D)[d4]
+                 : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+    __syncthreads();
+    const float4* kr = reinterpret_cast<const float4*>(sK + lane * KS);
+    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
+#pragma unroll 8
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      const float4 k4 = kr[d4], x = q0[d4], y = q1[d4];
+      a0 = fmaf(x.x, k4.x, a0); a1 = fmaf(x.y, k4.y, a1);
+      a0 = fmaf(x.z, k4.z, a0); a1 = fmaf(x.w, k4.w, a1);
+      b0 = fmaf(y.x, k4.x, b0); b1 = fmaf(y.y, k4.y, b1);
+      b0 = fmaf(y.z, k4.z, b0); b1 = fmaf(y.w, k4.w, b1);
+    }
+    sL[(2 * warp) * nBpad + kt * 32 + lane] = (a0 + a1) * scale;
+    sL[(2 * warp + 1) * nBpad + kt * 32 + lane] = (b0 + b1) * scale;
+  }
+  __syncwarp();
+  for (int r = 0; r < 2; ++r) {
+    const int lr = 2 * warp + r;
+    const int qb = row0 + lr;
+    if (qb >= nB) break;
+    select_row<MAXW>(sL + lr * nBpad, nB, words, qb, p, k_floor,
+                     mask + (static_cast<size_t>(bhi) * nB + qb) * words,
+                     counts + static_cast<size_t>(bhi) * nB + qb, lane);
+  }
 }
 
 size_t route_smem_bytes(const Geo& g) {
   const size_t nBpad = static_cast<size_t>(g.words) * 32;
-  return (static_cast<size_t>(kRouteRows) * g.d + static_cast<size_t>(g.d) * 33) * 4 +
-         static_cast<size_t>(kRouteRows) * nBpad * 8;
+  return (static_cast<size_t>(kRouteRows) * g.d + 32 * static_cast<size_t>(g.d + 4) +
+          static_cast<size_t>(kRouteRows) * nBpad) * 4;
+}
+
+template <int D, int MAXW>
+static cudaError_t launch_route_t(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                                  float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
+  dim3 grid((g.nB + kRouteRows - 1) / kRouteRows, g.B * g.H);
+  const size_t smem = route_smem_bytes(g);
+  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, MAXW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                       static_cast<int>(smem));
+  if (e != cudaSuccess) return e;
+  route_kernel<D, MAXW><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_route_d(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                                  float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
+  if (g.words <= 16) return launch_route_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 32) return launch_route_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  return launch_route_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, st);
 }
 
 cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
                          float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
-  dim3 grid((g.nB + kRouteRows - 1) / kRouteRows, g.B * g.H);
-  const size_t smem = route_smem_bytes(g);
-  cudaError_t e;
-  if (g.d == 128) {
-    e = cudaFuncSetAttribute(route_kernel<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    route_kernel<128><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
-  } else {
-    e = cudaFuncSetAttribute(route_kernel<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             static_cast<int>(smem));
-    if (e != cudaSuccess) return e;
-    route_kernel<64><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
-  }
-  return cudaGetLastError();
+  return g.d == 128 ? launch_route_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, st)
+                    : launch_route_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, st);
 }
 
 }  // namespace fv

@@ -54,7 +54,8 @@ typedef enum {
   FVATTN_ERR_UNSUPPORTED = 2,     /* valid but unsupported: d, block size, alignment */
   FVATTN_ERR_WORKSPACE = 3,       /* workspace missing or smaller than required */
   FVATTN_ERR_CUDA = 4,            /* a CUDA runtime/driver call failed */
-  FVATTN_ERR_DEVICE_TIMEOUT = 5   /* a kernel gave up a bounded wait (see fvattn_device_status) */
+  FVATTN_ERR_DEVICE_TIMEOUT = 5,  /* a kernel gave up a bounded wait (see fvattn_device_status) */
+  FVATTN_ERR_DEVICE = 6           /* a kernel detected an internal layout error and did no work */
 } fvattn_status_t;
 
 typedef struct {
@@ -140,9 +141,14 @@ FVATTN_API fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void*
                                   unsigned long long* sm_busy_ns, fvattn_stream_t stream);
 
 /* Synchronises `stream` and reports whether the last attention call that used
- * `workspace` gave up a bounded wait inside the kernel: FVATTN_OK or
- * FVATTN_ERR_DEVICE_TIMEOUT (FVATTN_ERR_CUDA if the synchronisation failed). */
+ * `workspace` ran cleanly: FVATTN_OK, FVATTN_ERR_DEVICE_TIMEOUT (a kernel gave up a
+ * bounded wait), FVATTN_ERR_DEVICE (a kernel found its shared memory misaligned and
+ * did no work), or FVATTN_ERR_CUDA if the synchronisation failed. */
 FVATTN_API fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream);
+
+/* Text of the CUDA error behind the calling thread's most recent FVATTN_ERR_CUDA
+ * ("no error" if there was none).  Static storage. */
+FVATTN_API const char* fvattn_last_cuda_error(void);
 
 /* Static, human-readable name of a status code. */
 FVATTN_API const char* fvattn_status_string(fvattn_status_t s);

@@ -74,7 +74,7 @@ def test_host_side_argument_checks(L):
 
 
 def test_status_strings(L):
-    for code in range(6):
+    for code in range(7):
         assert fv.fvattn_status_string(code)
     assert fv.fvattn_status_string(99) == "unknown status"
 
