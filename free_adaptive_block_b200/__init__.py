@@ -24,7 +24,7 @@ from typing import Optional
 __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
-    "fvattn_dense_attn", "fvattn_device_status", "fvattn_status_string", "attention_layer",
+    "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
     "LayerBuffers",
 ]
 
@@ -96,6 +96,10 @@ _SIGS = {
                                          ctypes.c_void_p, ctypes.c_float, ctypes.c_void_p,
                                          ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
                                          ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_block_sparse_attn_noalloc": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                                        ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                        ctypes.c_void_p]),
     "fvattn_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
     "fvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fvattn_last_cuda_error": (ctypes.c_char_p, []),
@@ -210,6 +214,20 @@ def fvattn_dense_attn(g: Geometry, q, k, v, scale: float, out, lse, workspace, s
         _ptr(v, torch.bfloat16, tok, "v"), float(scale), _ptr(out, torch.bfloat16, tok, "out"),
         _ptr(lse, torch.float32, tok[:3], "lse"), _ptr(workspace, torch.uint8, None, "workspace"),
         workspace.numel(), _ptr(sm_busy_ns, torch.int64, None, "sm_busy_ns"), _stream(stream)))
+
+
+def fvattn_block_sparse_attn_noalloc(g: Geometry, q, k, v, mask, scale: float, out, lse,
+                                     sm_busy_ns=None, stream=None) -> None:
+    """fvattn_block_sparse_attn without a workspace argument: for callers that cannot
+    allocate device memory; the library uses its own static scratch area instead."""
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    cg = g.c()
+    _ok("fvattn_block_sparse_attn_noalloc", lib().fvattn_block_sparse_attn_noalloc(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        _ptr(v, torch.bfloat16, tok, "v"), _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        float(scale), _ptr(out, torch.bfloat16, tok, "out"), _ptr(lse, torch.float32, tok[:3], "lse"),
+        _ptr(sm_busy_ns, torch.int64, None, "sm_busy_ns"), _stream(stream)))
 
 
 def fvattn_device_status(workspace, stream=None) -> int:

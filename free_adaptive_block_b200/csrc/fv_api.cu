@@ -132,6 +132,34 @@ fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, 
                                      reinterpret_cast<cudaStream_t>(stream)));
 }
 
+// Scratch for fvattn_block_sparse_attn_noalloc: the tile queue, the error word and the
+// LPT order live in this file-scope device array instead of a caller-provided workspace.
+// Every device that loads the library holds it until the process exits.
+constexpr size_t kNoAllocScratchBytes = size_t(1) << 20;   // 1 MiB: up to 131040 tiles
+static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratchBytes];
+
+constexpr int kMaxDevices = 64;
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices] = {};
+
+// Device address of g_noalloc_scratch on the current device, resolved once per device
+// (host code only holds a host-side stand-in for the symbol).
+fvattn_status_t noalloc_scratch(void** out) {
+  int dev = 0;
+  fvattn_status_t st = cuda_status(cudaGetDevice(&dev));
+  if (st != FVATTN_OK) return st;
+  if (dev < 0 || dev >= kMaxDevices) return FVATTN_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_noalloc_mu);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    st = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
+    if (st != FVATTN_OK) return st;
+    g_noalloc_addr[dev] = p;
+  }
+  *out = g_noalloc_addr[dev];
+  return FVATTN_OK;
+}
+
 }  // namespace
 
 extern "C" {
@@ -192,6 +220,19 @@ fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void* q, const v
                                   void* workspace, size_t ws_bytes,
                                   unsigned long long* sm_busy_ns, fvattn_stream_t stream) {
   return run_attn(g, q, k, v, nullptr, scale, out, lse, workspace, ws_bytes, sm_busy_ns, stream);
+}
+
+fvattn_status_t fvattn_block_sparse_attn_noalloc(const fvattn_geom_t* gi, const void* q, const void* k,
+                                                 const void* v, const uint32_t* mask, float scale,
+                                                 void* out, float* lse, unsigned long long* sm_busy_ns,
+                                                 fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  if (mask == nullptr) return FVATTN_ERR_INVALID_ARG;
+  if (fv::attn_ws_bytes(g) > kNoAllocScratchBytes) return FVATTN_ERR_WORKSPACE;
+  void* scratch = nullptr;
+  FV_CHECK(noalloc_scratch(&scratch));
+  return run_attn(gi, q, k, v, mask, scale, out, lse, scratch, kNoAllocScratchBytes, sm_busy_ns, stream);
 }
 
 fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream) {

@@ -133,6 +133,32 @@ FVATTN_API fvattn_status_t fvattn_block_sparse_attn(const fvattn_geom_t* g, cons
                                          void* workspace, size_t ws_bytes,
                                          unsigned long long* sm_busy_ns, fvattn_stream_t stream);
 
+/* fvattn_block_sparse_attn for callers that cannot allocate device memory: the same
+ * computation and arguments, minus the workspace, which comes from a scratch area the
+ * library itself reserves as a static device array of 1 MiB (held on every device
+ * that loads the library until the process exits).  It serves code that may not call
+ * cudaMalloc or reach a device allocator at the point of the call: runtimes that plan
+ * all device memory up front and forbid allocation on the serving path, plugins whose
+ * host framework owns every device buffer, callers without a handle to an allocator.
+ * The paper has no counterpart; this is an integration convenience of this library.
+ * - Allocates nothing: no cudaMalloc, cudaFree or allocating library call.
+ * - Geometries whose tile queue needs more than the scratch area (B*H*nB above
+ *   131040 tiles) are rejected with FVATTN_ERR_WORKSPACE.
+ * - The first call on a device resolves the scratch area's device address
+ *   (cudaGetSymbolAddress) with that device current; make that first call before any
+ *   stream capture.
+ * - Every call shares the one scratch area, which keeps the last call's contents (the
+ *   kernels reset what must start at zero).  Calls that overlap on the GPU (different
+ *   streams, or different host threads on one device) race on it: serialise them.
+ * - A device-side timeout of this entry point is not reported through
+ *   fvattn_device_status (there is no workspace to pass it). */
+FVATTN_API fvattn_status_t fvattn_block_sparse_attn_noalloc(const fvattn_geom_t* g, const void* q,
+                                                            const void* k, const void* v,
+                                                            const uint32_t* mask, float scale,
+                                                            void* out, float* lse,
+                                                            unsigned long long* sm_busy_ns,
+                                                            fvattn_stream_t stream);
+
 /* Dense attention: fvattn_block_sparse_attn with every key block kept (the p = 1
  * case), without reading a mask.  Same arguments otherwise. */
 FVATTN_API fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void* q, const void* k,
