@@ -35,6 +35,20 @@ from free_adaptive_block_b200 import metrics as MX  # noqa: E402
 from free_adaptive_block_b200 import workloads as W  # noqa: E402
 
 METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16 peak"
+
+# DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
+# `ncu --set full` capture; valid only for the kernel source it was taken from.
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "a686b3a7a8a5028d", "bytes": 390201344}
+
+
+def attn_traffic():
+    import hashlib
+    src = os.path.join(ROOT, "free_adaptive_block_b200", "csrc", "fv_attn.cu")
+    try:
+        h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
+    except OSError:
+        return None
+    return ATTN_NCU_TRAFFIC["bytes"] if h == ATTN_NCU_TRAFFIC["fv_attn.cu sha256[:16]"] else None
 UNIT = "TFLOP/s"
 
 
@@ -254,7 +268,7 @@ def run_ours(args, rank, world, local_rank):
         "sm_busy_max_over_mean": round(float(busy.max() / busy.mean()), 4) if busy.size else None,
         "roofline": {"bound": "tensor", "kernel": "fvattn_block_sparse_attn (prep + attn_kernel)",
                      "achieved": round(attn_tflops, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
-                     "frac": round(attn_tflops / peaks["bf16"], 4), "traffic": None,
+                     "frac": round(attn_tflops / peaks["bf16"], 4), "traffic": attn_traffic(),
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
         "e2e": {"value": round(eff * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
