@@ -11,12 +11,18 @@
 //   * warp 0 loads Q / K / V boxes with TMA (5D tensor maps over
 //     [B*H][T][Hs][Ws][d], 128-byte swizzle, out-of-range rows zero-filled; blocks on
 //     the W edge use a narrower box so their real rows stay compact), warp 1 issues
-//     tcgen05.mma (S = Q K^T into tensor memory, then O += P V with P read from
-//     tensor memory), warps 2..5 run the softmax, one TMEM lane (= query row) per
-//     thread, and write out / lse;
-//   * the running maximum is re-based lazily: O and l are rescaled only when the
-//     block maximum exceeds the reference by more than 2^8, which keeps the result
-//     exact (O / l and lse use the same reference) and P <= 256.
+//     tcgen05.mma (S_j = Q K_j^T into a three-deep ring of S buffers in tensor memory,
+//     then O += P_j V_j with P_j read from tensor memory over S_j);
+//   * two softmax warpgroups take the kept blocks alternately (even j, odd j), one
+//     TMEM lane (= query row) per thread.  They share one O accumulator, so every P_j
+//     is taken against one running reference per row: the group that owns block j
+//     receives the reference after block j-1 from the other group through shared
+//     memory, updates it with its own block maximum and hands it on before computing
+//     its exponentials, so the two groups' exponentials overlap each other and the
+//     tensor core;
+//   * the reference is re-based lazily: O and l are rescaled only when the block
+//     maximum exceeds the reference by more than 2^8, which keeps the result exact
+//     (O / l and lse use the same reference) and P <= 256.
 //
 // Every wait is bounded (fv::mbar_wait): a stuck pipeline sets an error bit in the
 // workspace, all roles leave their loops, outstanding copies and MMAs are drained,
@@ -28,23 +34,24 @@
 
 namespace fv {
 
-constexpr int kSoftWarps = 8;          // softmax warps: two per TMEM lane quarter
+constexpr int kSoftWarps = 8;          // softmax warps: one per TMEM lane quarter in each group
 // Three warpgroups: warps 0-3 (producer, MMA issuer, two idle warps) and two softmax
 // warpgroups (warps 4-7 and 8-11).  Launched at 168 registers a thread (the register
 // file is split per SM partition, and each partition holds one warp of each group);
 // setmaxnreg then moves registers from the first group to the softmax groups:
-// 128 * 80 + 256 * 208 = 63488 <= 384 * 168 = 64512.
+// 128 * 56 + 256 * 224 = 64512 = 384 * 168.
 constexpr int kAttnThreads = 384;
-constexpr int kRegsCtl = 80;
-constexpr int kRegsSoft = 208;
+constexpr int kRegsCtl = 56;
+constexpr int kRegsSoft = 224;
 static_assert(128 * kRegsCtl + 256 * kRegsSoft <= kAttnThreads * 168, "register split exceeds the launch budget");
 constexpr int kNK = 3;                 // K ring depth
 constexpr int kNV = 3;                 // V ring depth
 constexpr int kTR = 2;                 // tile-id ring depth
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle column)
 constexpr uint32_t kTmemCols = 512;
-constexpr uint32_t kColS = 0;          // S of chain c: columns [128c, 128c+128); P (bf16 pairs) over its first 64
-constexpr uint32_t kColO = 256;        // O of chain c: columns [256 + d*c, 256 + d*c + d)
+constexpr int kNS = 3;                 // S ring depth (tensor memory)
+constexpr uint32_t kColS = 0;          // S slot r: columns [128r, 128r+128); P (bf16 pairs) over its first 64
+constexpr uint32_t kColO = 128 * kNS;  // O: columns [384, 384 + d)
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
 #ifndef FV_POLY_EVERY
 #define FV_POLY_EVERY 0
@@ -109,10 +116,11 @@ struct __align__(8) AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kNK], k_empty[kNK];
   uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[2];     // per softmax chain
-  uint64_t p_full[2];
-  uint64_t pv_done[2], o_empty;
-  uint64_t xbar[4];       // end-of-tile (max, sum) exchange, per TMEM lane quarter: written
+  uint64_t s_full[kNS];   // per S slot
+  uint64_t p_full[kNS];
+  uint64_t pv_done[kNS], o_empty;
+  uint64_t hb[2][4];      // reference hand-off, [writing group][TMEM lane quarter]
+  uint64_t xbar[4];       // end-of-tile row-sum exchange, per TMEM lane quarter: written
   uint64_t xread[4];      //   ... and read by both warps of the quarter pair
   uint64_t t_full[kTR], t_empty[kTR];
   uint64_t fin;
@@ -120,8 +128,8 @@ struct __align__(8) AttnBars {
   uint32_t mrow[kTR][64]; // the tile's mask row (nB <= 2048), read by every role
   uint32_t tmem_base;
   int abort;
-  float xm[2][128];       // [chain][row], guarded by xbar / xread
-  float xl[2][128];
+  float hv[2][128];       // [group][row] reference after the group's latest block, guarded by hb
+  float xl[2][128];       // [group][row] row sums at the end of a tile, guarded by xbar / xread
 };
 
 template <int D>
@@ -198,13 +206,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     mbar_init(&bars.q_empty, 1);
     for (int i = 0; i < kNK; ++i) { mbar_init(&bars.k_full[i], 1); mbar_init(&bars.k_empty[i], 1); }
     for (int i = 0; i < kNV; ++i) { mbar_init(&bars.v_full[i], 1); mbar_init(&bars.v_empty[i], 1); }
-    for (int i = 0; i < 2; ++i) {
+    for (int i = 0; i < kNS; ++i) {
       mbar_init(&bars.s_full[i], 1);
       mbar_init(&bars.p_full[i], kSoftWarps / 2);
+      mbar_init(&bars.pv_done[i], 1);
     }
-    for (int i = 0; i < 4; ++i) { mbar_init(&bars.xbar[i], 2); mbar_init(&bars.xread[i], 2); }
-    mbar_init(&bars.pv_done[0], 1);
-    mbar_init(&bars.pv_done[1], 1);
+    for (int i = 0; i < 4; ++i) {
+      mbar_init(&bars.xbar[i], 2);
+      mbar_init(&bars.xread[i], 2);
+      mbar_init(&bars.hb[0][i], 1);
+      mbar_init(&bars.hb[1][i], 1);
+    }
     mbar_init(&bars.o_empty, kSoftWarps);
     for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 1 + kSoftWarps); }
     mbar_init(&bars.fin, 1);
@@ -309,13 +321,13 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
    } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issuer
-    // Two softmax chains per tile: chain 0 takes the tile's even KV blocks, chain 1
-    // the odd ones.  Chain c has its own S buffer (P is written back over it) and its
-    // own O accumulator.  Issue order: S_0, S_1, then PV_j, S_j+2 for j = 0, 1, ...
-    // so the chains run half a period apart and one chain's softmax overlaps the other
-    // chain's P.V and S.  S_j+2 overwrites the buffer P_j lives in, so it waits for PV_j.
-    uint32_t tcount = 0, mkc = 0, mvc = 0, mqc = 0, tiles = 0;
-    uint32_t pvn[2] = {0u, 0u};          // P.V products issued per chain (all tiles)
+    // Block j of the call's running block count c lives in S slot c mod kNS; S_c
+    // overwrites P_c-kNS, so it waits for that P.V.  O is one accumulator: the P.V
+    // products go in block order.  The S stream and the P.V stream are each issued in
+    // block order and interleave as their inputs become ready (non-blocking probes),
+    // which keeps every ring barrier at most one phase ahead of its probe.
+    uint32_t tcount = 0, mqc = 0, tiles = 0;
+    uint32_t gc = 0;                      // blocks issued so far (all tiles): ring position
     const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
     const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
@@ -331,73 +343,93 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       ++mqc;
       KvIter it;
       it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
-      int npad_r[4] = {0, 0, 0, 0};
-      int ns = 0;
+      uint32_t npk = 0;                 // npad/16 of blocks j..j+7, 4 bits each (ring)
+      int nknown = 0;
       bool ended = false;
-      // S_ns: returns false on a failed wait
-      auto try_s = [&]() -> bool {
-        if (ended) return true;
-        const int kb = it.advance();
-        if (kb < 0) { ended = true; return true; }
-        const int j = ns;
-        const int c = j & 1;
-        const int npad = blk_of(g, kb).npad;
-        npad_r[j & 3] = npad;
-        const int ks = mkc % kNK;
-        if (!wwait(&bars.k_full[ks], (mkc / kNK) & 1)) return false;
-        if (pvn[c] > 0 && !wwait(&bars.pv_done[c], (pvn[c] - 1) & 1)) return false;
-        tc_fence_after();
-        const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
-        const uint32_t tS = tmem + kColS + c * 128;
-        const uint32_t idesc_s = idesc_bf16_f32(128, npad, 0, 0);
-        if (elect_one()) {
-#pragma unroll
-          for (int kk = 0; kk < D / 16; ++kk) {
-            const uint64_t off = static_cast<uint64_t>(((kk >> 2) * kChunkBytes + (kk & 3) * 32) >> 4);
-            mma_ss(tS, dQ + off, dK + off, idesc_s, kk > 0 ? 1u : 0u);
-          }
-          mma_commit(&bars.s_full[c]);
-          mma_commit(&bars.k_empty[ks]);
+      int sn = 0, vn = 0;               // next S / next P.V block index of the tile
+      uint64_t t_prog = globaltimer();
+      uint32_t idle = 0;
+      while (true) {
+        while (!ended && nknown <= sn) {
+          const int kb = it.advance();
+          if (kb < 0) { ended = true; break; }
+          const uint32_t sh = 4u * (nknown & 7);
+          npk = (npk & ~(0xFu << sh)) | (static_cast<uint32_t>(blk_of(g, kb).npad >> 4) << sh);
+          ++nknown;
         }
-        __syncwarp();
-        ++mkc;
-        ++ns;
-        return true;
-      };
-      auto issue_pv = [&](int j) -> bool {
-        const int c = j & 1;
-        const int npad = npad_r[j & 3];
-        if (!wwait(&bars.p_full[c], pvn[c] & 1)) return false;
-        const int vs = mvc % kNV;
-        if (!wwait(&bars.v_full[vs], (mvc / kNV) & 1)) return false;
-        if (j == 0 && !wwait(&bars.o_empty, (tiles & 1) ^ 1)) return false;
-        tc_fence_after();
-        const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
-        const uint32_t tP = tmem + kColS + c * 128;
-        const uint32_t tO = tmem + kColO + c * D;
-        const int nk = npad >> 4;
-        if (elect_one()) {
+        bool progressed = false;
+        // ---- S_sn
+        if (sn < nknown && vn > sn - kNS) {
+          const uint32_t c = gc + sn;
+          const int ss = c % kNS;
+          const int ks = c % kNK;
+          bool rdy = mbar_test(&bars.k_full[ks], (c / kNK) & 1);
+          if (rdy && c >= kNS) rdy = mbar_test(&bars.pv_done[ss], ((c - kNS) / kNS) & 1);
+          if (__all_sync(0xffffffffu, rdy)) {
+            tc_fence_after();
+            const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
+            const uint32_t tS = tmem + kColS + ss * 128;
+            const uint32_t np = ((npk >> (4u * (sn & 7))) & 0xFu) << 4;
+            const uint32_t idesc_s = idesc_bf16_f32(128, np, 0, 0);
+            if (elect_one()) {
 #pragma unroll
-          for (int kk = 0; kk < 8; ++kk) {
-            if (kk < nk)
-              mma_ts(tO, tP + kk * 8, dV + static_cast<uint64_t>((kk * 2048) >> 4), idesc_pv,
-                     (j < 2 && kk == 0) ? 0u : 1u);
+              for (int q = 0; q < D / 16; ++q) {
+                const uint64_t off =
+                    static_cast<uint64_t>(((q >> 2) * kChunkBytes + (q & 3) * 32) >> 4);
+                mma_ss(tS, dQ + off, dK + off, idesc_s, q > 0 ? 1u : 0u);
+              }
+              mma_commit(&bars.s_full[ss]);
+              mma_commit(&bars.k_empty[ks]);
+            }
+            __syncwarp();
+            ++sn;
+            progressed = true;
           }
-          mma_commit(&bars.v_empty[vs]);
-          mma_commit(&bars.pv_done[c]);
         }
-        __syncwarp();
-        ++mvc;
-        ++pvn[c];
-        return true;
-      };
-      // PV_j then S_j+2 (same chain): while one chain's softmax runs, the tensor core
-      // works on the other chain's P.V and next S.
-      if (!try_s() || !try_s()) break;
-      for (int j = 0; j < ns && ok; ++j) {
-        if (!issue_pv(j) || !try_s()) { ok = false; break; }
+        // ---- O += P_vn V_vn
+        if (vn < sn) {
+          const uint32_t c = gc + vn;
+          const int ss = c % kNS;
+          const int vs = c % kNV;
+          bool rdy = mbar_test(&bars.p_full[ss], (c / kNS) & 1);
+          if (rdy) rdy = mbar_test(&bars.v_full[vs], (c / kNV) & 1);
+          if (rdy && vn == 0) rdy = mbar_test(&bars.o_empty, (tiles & 1) ^ 1);
+          if (__all_sync(0xffffffffu, rdy)) {
+            tc_fence_after();
+            const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
+            const uint32_t tP = tmem + kColS + ss * 128;
+            const int nk = (npk >> (4u * (vn & 7))) & 0xFu;
+            if (elect_one()) {
+#pragma unroll
+              for (int q = 0; q < 8; ++q) {
+                if (q < nk)
+                  mma_ts(tmem + kColO, tP + q * 8, dV + static_cast<uint64_t>((q * 2048) >> 4),
+                         idesc_pv, (vn == 0 && q == 0) ? 0u : 1u);
+              }
+              mma_commit(&bars.v_empty[vs]);
+              mma_commit(&bars.pv_done[ss]);
+            }
+            __syncwarp();
+            ++vn;
+            progressed = true;
+          }
+        }
+        if (ended && vn >= nknown) break;
+        if (progressed) {
+          idle = 0;
+          t_prog = globaltimer();
+        } else if ((++idle & 63u) == 0) {
+          if (*abort) { ok = false; break; }
+          if (globaltimer() - t_prog > 2000000000ull) {
+            *abort = 1;
+            if (lane == 0) atomicOr(err, kErrTimeout);
+            ok = false;
+            break;
+          }
+        }
       }
       if (!ok) break;
+      gc += nknown;
       if (elect_one()) mma_commit(&bars.q_empty);
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.t_empty[slot]);   // done with the tile's mask row
@@ -407,23 +439,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   } else {
     asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(kRegsSoft));
     // ------------------------------------------------------------ softmax + epilogue
-    // Warpgroup c = (w-4)/4 runs chain c: the tile's KV blocks j with j % 2 == c.  One
-    // thread per query row (TMEM lane 32*(w%4) + lane), all 128 key columns of a block
-    // in registers.  At the end of a tile the two chains' (max, sum) are exchanged per
-    // row through shared memory and a bounded mbarrier, and chain c writes output
-    // columns [c*d/2, (c+1)*d/2) of  (O_0 2^(m_0-m) + O_1 2^(m_1-m)) / (l_0 2^(m_0-m) + l_1 2^(m_1-m)).
-    const int chain = (warp - 4) >> 2;
+    // Group grp = (w-4)/4 takes the tile's kept blocks j with j % 2 == grp.  One thread
+    // per query row (TMEM lane 32*(w%4) + lane), the 128 key columns of a block in
+    // registers.  Per row the running reference m_j (log2 units) is one value for the
+    // whole tile: the group of block j takes m_j-1 from the other group (hv / hb, per
+    // lane quarter), sets m_j and hands it on before its exponentials.  Each group
+    // keeps its own row sum l against the reference of its latest block; at the end of
+    // the tile the group that did not run the last block takes the final reference
+    // from the other group's last hand-off, both rescale their l to it, exchange l
+    // (xl / xbar / xread) and each writes half of the output columns.
+    const int grp = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
-    const uint32_t tS = tmem + lane_off + kColS + chain * 128;
-    const uint32_t tO0 = tmem + lane_off + kColO;
-    uint32_t tcount = 0, sn = 0, xn = 0;
+    const uint32_t tS0 = tmem + lane_off + kColS;
+    const uint32_t tO = tmem + lane_off + kColO;
+    uint32_t tcount = 0, xn = 0, hr = 0;
+    uint32_t gc = 0;                    // blocks of all earlier tiles: S ring position
     const float sl2 = prm.scale_log2;
     const uint64_t sl2x2 = f32x2(sl2, sl2);
+    auto sync_wait = [&](uint64_t* bar, uint32_t parity) -> bool {
+      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err));
+    };
     while (true) {
       const int slot = tcount % kTR;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.t_full[slot], (tcount / kTR) & 1, abort, err))) break;
+      if (!sync_wait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
       const int tile = bars.tile[slot];
       ++tcount;
       if (tile < 0) break;
@@ -432,13 +472,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const BlockInfo qi = block_info(g, qb);
       const int token = box_row_token(g, qi, row);
 
-      float m = -INFINITY, l = 0.f;
-      int nblk = 0, j = 0;
+      float m = -INFINITY, l = 0.f;     // this group's latest reference and its row sum
+      int j = 0;
       bool ok = true;
       KvIter it;
       it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
       for (int kb = it.advance(); kb >= 0; kb = it.advance(), ++j) {
-        if ((j & 1) != chain) continue;
+        if ((j & 1) != grp) continue;
+        const uint32_t c = gc + j;
+        const int ss = c % kNS;
+        const uint32_t tS = tS0 + ss * 128;
         const BlkEnt ki = blk_of(g, kb);
         const bool full = ki.prefix && ki.nvalid >= 128;
         uint32_t vm[4];
@@ -453,141 +496,147 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           for (int w4 = 0; w4 < 4; ++w4)
             vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, block_info(g, kb), 32 * w4 + lane) >= 0);
         }
-        if (!__all_sync(0xffffffffu, mbar_wait(&bars.s_full[chain], sn & 1, abort, err))) { ok = false; break; }
+        if (!sync_wait(&bars.s_full[ss], (c / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
         // The whole row of S in one TMEM round trip (loads are grouped, then one wait:
         // a TMEM store issued after a load waits for it, so loads and stores are not
         // interleaved).
         float s[128];
 #pragma unroll
-        for (int c = 0; c < 4; ++c) tmem_ld32(tS + 32 * c, reinterpret_cast<uint32_t*>(s + 32 * c));
+        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, reinterpret_cast<uint32_t*>(s + 32 * q));
         tmem_wait_ld();
         const int nact = (ki.npad + 31) >> 5;    // 32-column chunks below npad (uniform)
         if (!full) {
 #pragma unroll
-          for (int c = 0; c < 128; ++c) s[c] = ((vm[c >> 5] >> (c & 31)) & 1u) ? s[c] : -INFINITY;
+          for (int q = 0; q < 128; ++q) s[q] = ((vm[q >> 5] >> (q & 31)) & 1u) ? s[q] : -INFINITY;
         }
         float mq[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
           float mm = max3f(s[32 * r], s[32 * r + 1], s[32 * r + 2]);
 #pragma unroll
-          for (int c = 3; c < 31; c += 2) mm = max3f(mm, s[32 * r + c], s[32 * r + c + 1]);
+          for (int q = 3; q < 31; q += 2) mm = max3f(mm, s[32 * r + q], s[32 * r + q + 1]);
           mq[r] = fmaxf(mm, s[32 * r + 31]);
         }
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
-        float alpha = 1.f;
+        // reference after block j-1, from the other group
+        float mref = mx;
         bool rebase = false;
-        if (nblk == 0) {
-          m = mx;
-        } else if (mx > m + kRebase) {
-          alpha = ex2(m - mx);
-          m = mx;
-          rebase = true;
+        float alpha = 1.f;
+        if (j > 0) {
+          if (!sync_wait(&bars.hb[grp ^ 1][quarter], hr & 1)) { ok = false; break; }
+          ++hr;
+          const float mp = bars.hv[grp ^ 1][row];
+          mref = mp;
+          if (mx > mp + kRebase) {
+            mref = mx;
+            alpha = ex2(mp - mx);
+            rebase = true;
+          }
         }
-        // The chain's previous P.V finished before this S was computed (the MMA
-        // warp waits for it), so O can be re-based here directly.
+        bars.hv[grp][row] = mref;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.hb[grp][quarter]);
+        // O holds P_0 V_0 + ... + P_j-1 V_j-1 against the old reference once P.V j-1
+        // has finished; re-base it before P_j goes in.
         if (__any_sync(0xffffffffu, rebase)) {
-          const uint32_t tO = tO0 + chain * D;
+          const uint32_t cp = c - 1;
+          if (!sync_wait(&bars.pv_done[cp % kNS], (cp / kNS) & 1)) { ok = false; break; }
+          tc_fence_after();
 #pragma unroll 1
-          for (int c = 0; c < D / 32; ++c) {
+          for (int q = 0; q < D / 32; ++q) {
             uint32_t o[32];
-            tmem_ld32(tO + 32 * c, o);
+            tmem_ld32(tO + 32 * q, o);
             tmem_wait_ld();
 #pragma unroll
             for (int e = 0; e < 32; ++e) o[e] = __float_as_uint(__uint_as_float(o[e]) * alpha);
-            tmem_st32(tO + 32 * c, o);
+            tmem_st32(tO + 32 * q, o);
           }
         }
-        // P = 2^(s * scale * log2 e - m), packed to bf16 pairs; stored after all of it
-        // is computed (P column k/2 holds keys k, k+1, over S columns already read).
+        // this group's row sum follows the reference (unchanged unless a group re-based)
+        if (mref != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mref);
+        m = mref;
+        // P = 2^(s * scale * log2 e - m), packed to bf16 pairs and stored 16 keys at a
+        // time over S columns already read (P column k/2 holds keys k, k+1).  Chunks at
+        // or past npad are neither computed nor stored: the P.V reads keys < npad only.
         const uint64_t nmx2 = f32x2(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
-        uint32_t pk[64];
 #pragma unroll
         for (int c32 = 0; c32 < 4; ++c32) {
           if (c32 < nact) {
 #pragma unroll
-            for (int e = 0; e < 16; ++e) {
-              const int c = 32 * c32 + 2 * e;
-              float x0, x1;
-              unpack_f32x2(ffma2(f32x2(s[c], s[c + 1]), sl2x2, nmx2), x0, x1);
-              float p0, p1;
-              if (full && kPolyEvery > 0 && (e % kPolyEvery) == kPolyEvery - 1) {
-                ex2_poly2(x0, x1, p0, p1);
-              } else {
-                p0 = ex2(x0);
-                p1 = ex2(x1);
-              }
-              acc[e & 3] = fadd2(acc[e & 3], f32x2(p0, p1));
-              pk[16 * c32 + e] = pack_bf16x2(p0, p1);
-            }
-          } else {
+            for (int h = 0; h < 2; ++h) {
+              uint32_t pk[8];
 #pragma unroll
-            for (int e = 0; e < 16; ++e) pk[16 * c32 + e] = 0u;
+              for (int e = 0; e < 8; ++e) {
+                const int q = 32 * c32 + 16 * h + 2 * e;
+                float x0, x1;
+                unpack_f32x2(ffma2(f32x2(s[q], s[q + 1]), sl2x2, nmx2), x0, x1);
+                float p0, p1;
+                if (full && kPolyEvery > 0 && (e % kPolyEvery) == kPolyEvery - 1) {
+                  ex2_poly2(x0, x1, p0, p1);
+                } else {
+                  p0 = ex2(x0);
+                  p1 = ex2(x1);
+                }
+                acc[e & 3] = fadd2(acc[e & 3], f32x2(p0, p1));
+                pk[e] = pack_bf16x2(p0, p1);
+              }
+              tmem_st8(tS + 16 * c32 + 8 * h, pk);
+            }
           }
         }
-        tmem_st32(tS, pk);
-        tmem_st32(tS + 32, pk + 32);
         float sa, sb, sc2, sd;
         unpack_f32x2(fadd2(acc[0], acc[1]), sa, sb);
         unpack_f32x2(fadd2(acc[2], acc[3]), sc2, sd);
-        l = l * alpha + ((sa + sb) + (sc2 + sd));
+        l += (sa + sb) + (sc2 + sd);
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[chain]);
-        ++sn;
-        ++nblk;
+        if (lane == 0) mbar_arrive(&bars.p_full[ss]);
       }
       if (!ok) break;
-      // ---- epilogue: wait for this chain's last P.V, exchange (m, l) with the partner
+      // ---- epilogue
       const int nkv = j;
-      if (nblk > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars.pv_done[chain], (sn - 1) & 1, abort, err))) break;
-      if (xn > 0 && !__all_sync(0xffffffffu, mbar_wait(&bars.xread[quarter], (xn - 1) & 1, abort, err))) break;
-      bars.xm[chain][row] = m;
-      bars.xl[chain][row] = l;
+      gc += nkv;
+      float mf = m;                      // final reference of the tile
+      if (nkv > 0 && ((nkv - 1) & 1) != grp) {
+        if (!sync_wait(&bars.hb[grp ^ 1][quarter], hr & 1)) break;
+        ++hr;
+        mf = bars.hv[grp ^ 1][row];
+      }
+      if (mf != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mf);
+      if (nkv > 0) {
+        const uint32_t cl = gc - 1;      // the tile's last P.V
+        if (!sync_wait(&bars.pv_done[cl % kNS], (cl / kNS) & 1)) break;
+      }
+      if (xn > 0 && !sync_wait(&bars.xread[quarter], (xn - 1) & 1)) break;
+      bars.xl[grp][row] = l;
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.xbar[quarter]);
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.xbar[quarter], xn & 1, abort, err))) break;
-      const float m_o = bars.xm[chain ^ 1][row];
-      const float l_o = bars.xl[chain ^ 1][row];
+      if (!sync_wait(&bars.xbar[quarter], xn & 1)) break;
+      const float lt = l + bars.xl[grp ^ 1][row];
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.xread[quarter]);
       ++xn;
-      const bool have0 = nkv >= 1, have1 = nkv >= 2;
-      const float m0 = chain == 0 ? m : m_o, m1 = chain == 0 ? m_o : m;
-      const float l0 = chain == 0 ? l : l_o, l1 = chain == 0 ? l_o : l;
-      const float mt = have1 ? fmaxf(m0, m1) : m0;
-      const float a0 = have0 ? ex2(m0 - mt) : 0.f;
-      const float a1 = have1 ? ex2(m1 - mt) : 0.f;
-      const float lt = l0 * a0 + l1 * a1;
       const float inv = 1.f / lt;
-      const float w0 = a0 * inv, w1 = a1 * inv;
       tc_fence_after();
       uint4* dst = reinterpret_cast<uint4*>(prm.out + (static_cast<size_t>(bhi) * g.N + (token >= 0 ? token : 0)) * D +
-                                            (D / 2) * chain);
+                                            (D / 2) * grp);
 #pragma unroll
-      for (int c = 0; c < D / 64; ++c) {
-        uint32_t o0[32], o1[32];
-        tmem_ld32(tO0 + (D / 2) * chain + 32 * c, o0);
-        tmem_ld32(tO0 + D + (D / 2) * chain + 32 * c, o1);
+      for (int q = 0; q < D / 64; ++q) {
+        uint32_t o[32];
+        tmem_ld32(tO + (D / 2) * grp + 32 * q, o);
         tmem_wait_ld();
         if (token >= 0) {
 #pragma unroll
           for (int q8 = 0; q8 < 4; ++q8) {
-            float v[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float x1 = have1 ? __uint_as_float(o1[8 * q8 + e]) * w1 : 0.f;
-              v[e] = fmaf(__uint_as_float(o0[8 * q8 + e]), w0, x1);
-            }
             uint4 wv;
-            wv.x = pack_bf16x2(v[0], v[1]);
-            wv.y = pack_bf16x2(v[2], v[3]);
-            wv.z = pack_bf16x2(v[4], v[5]);
-            wv.w = pack_bf16x2(v[6], v[7]);
-            dst[4 * c + q8] = wv;
+            wv.x = pack_bf16x2(__uint_as_float(o[8 * q8 + 0]) * inv, __uint_as_float(o[8 * q8 + 1]) * inv);
+            wv.y = pack_bf16x2(__uint_as_float(o[8 * q8 + 2]) * inv, __uint_as_float(o[8 * q8 + 3]) * inv);
+            wv.z = pack_bf16x2(__uint_as_float(o[8 * q8 + 4]) * inv, __uint_as_float(o[8 * q8 + 5]) * inv);
+            wv.w = pack_bf16x2(__uint_as_float(o[8 * q8 + 6]) * inv, __uint_as_float(o[8 * q8 + 7]) * inv);
+            dst[4 * q + q8] = wv;
           }
         }
       }
@@ -597,10 +646,8 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         mbar_arrive(&bars.o_empty);
         mbar_arrive(&bars.t_empty[slot]);   // done with the tile's mask row
       }
-      if (token >= 0) {
-        if (chain == 0)
-          prm.lse[static_cast<size_t>(bhi) * g.N + token] = (mt + __log2f(lt)) * 0.69314718055994531f;
-      }
+      if (token >= 0 && grp == 0)
+        prm.lse[static_cast<size_t>(bhi) * g.N + token] = (mf + __log2f(lt)) * 0.69314718055994531f;
     }
   }
 
