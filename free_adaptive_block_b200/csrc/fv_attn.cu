@@ -35,7 +35,7 @@
 namespace fv {
 
 constexpr int kSoftWarps = 8;          // softmax warps: one per TMEM lane quarter in each group
-// Three warpgroups: warps 0-3 (producer, MMA issuer, two idle warps) and two softmax
+// Three warpgroups: warps 0-3 (producer, S issuer, P.V issuer, one idle warp) and two softmax
 // warpgroups (warps 4-7 and 8-11).  Launched at 168 registers a thread (the register
 // file is split per SM partition, and each partition holds one warp of each group);
 // setmaxnreg then moves registers from the first group to the softmax groups:
@@ -45,13 +45,21 @@ constexpr int kRegsCtl = 56;
 constexpr int kRegsSoft = 224;
 static_assert(128 * kRegsCtl + 256 * kRegsSoft <= kAttnThreads * 168, "register split exceeds the launch budget");
 constexpr int kNK = 3;                 // K ring depth
-constexpr int kNV = 3;                 // V ring depth
+constexpr int kNV = 2;                 // V ring depth (P.V runs a softmax behind S: V has slack)
+constexpr int kMaxBlocks = 2048;       // blocks per (b, h) slice, the mask row limit
 constexpr int kTR = 2;                 // tile-id ring depth
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle column)
 constexpr uint32_t kTmemCols = 512;
-constexpr int kNS = 3;                 // S ring depth (tensor memory)
-constexpr uint32_t kColS = 0;          // S slot r: columns [128r, 128r+128); P (bf16 pairs) over its first 64
-constexpr uint32_t kColO = 128 * kNS;  // O: columns [384, 384 + d)
+// Tensor memory (512 columns x 128 lanes, lane = query row): two S slots of 128 fp32
+// columns, O (d columns) and two P slots of 64 columns (bf16 pairs).  An S slot is
+// free as soon as its softmax group has loaded it into registers, and P_c only waits
+// for the P.V two blocks back, so no tensor-core product waits on the one before it.
+constexpr int kNS = 2;                 // S ring depth
+constexpr int kNP = 2;                 // P ring depth
+constexpr uint32_t kColS = 0;          // S slot r: columns [128r, 128r+128)
+constexpr uint32_t kColO = 128 * kNS;  // O: columns [256, 256 + d)
+template <int D> __host__ __device__ constexpr uint32_t col_p() { return kColO + D; }   // P slot r: +64r
+static_assert(col_p<128>() + 64 * kNP <= 512, "tensor memory layout exceeds 512 columns");
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
 #ifndef FV_POLY_EVERY
 #define FV_POLY_EVERY 0
@@ -116,16 +124,20 @@ struct __align__(8) AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kNK], k_empty[kNK];
   uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[kNS];   // per S slot
-  uint64_t p_full[kNS];
-  uint64_t pv_done[kNS], o_empty;
+  uint64_t s_full[kNS];   // per S slot: written by the MMA ...
+  uint64_t s_empty[kNS];  //   ... and loaded into registers by its softmax group
+  uint64_t p_full[kNP];   // per P slot
+  uint64_t pv_done[3];    // P.V of block c commits [c % 3]: a group waiting for P.V c-1 or
+                          // c-2 has itself seen P.V c-4 complete, so no wait aliases a phase
+  uint64_t o_empty;
   uint64_t hb[2][4];      // reference hand-off, [writing group][TMEM lane quarter]
   uint64_t xbar[4];       // end-of-tile row-sum exchange, per TMEM lane quarter: written
   uint64_t xread[4];      //   ... and read by both warps of the quarter pair
   uint64_t t_full[kTR], t_empty[kTR];
-  uint64_t fin;
+  uint64_t fin[2];        // drain after an abort: S issuer, P.V issuer
   int tile[kTR];
-  uint32_t mrow[kTR][64]; // the tile's mask row (nB <= 2048), read by every role
+  int bcount[kTR];        // kept blocks of the tile
+  uint32_t blist[kTR][kMaxBlocks];  // the tile's kept blocks in ascending order (pack_blk)
   uint32_t tmem_base;
   int abort;
   float hv[2][128];       // [group][row] reference after the group's latest block, guarded by hb
@@ -144,29 +156,17 @@ __host__ __device__ constexpr int attn_smem_bytes() {
 }
 static_assert(attn_smem_bytes<128>() <= 232448, "attention kernel exceeds 227 KB of shared memory");
 
-// Iterates the set bits of a mask row in ascending order (or every block when dense).
-struct KvIter {
-  const uint32_t* row;
-  int nB, words, w, next;
-  uint32_t bits;
-  __device__ void init(const uint32_t* r, int nB_, int words_) {
-    row = r; nB = nB_; words = words_; w = -1; bits = 0; next = -1;
-  }
-  __device__ int advance() {      // returns the next block id, or -1
-    if (row == nullptr) {
-      ++next;
-      return next < nB ? next : -1;
-    }
-    while (bits == 0) {
-      ++w;
-      if (w >= words) return -1;
-      bits = row[w];
-    }
-    const int b = __ffs(bits) - 1;
-    bits &= bits - 1;
-    return w * 32 + b;
-  }
-};
+// One kept block of a tile as the consumers need it: block id (bits 0-11), npad / 16
+// (12-15), real token count (16-23), real tokens form a prefix of the box (24).
+__device__ __forceinline__ uint32_t pack_blk(const Geo& g, int kb) {
+  const BlkEnt e = blk_of(g, kb);
+  return static_cast<uint32_t>(kb) | (static_cast<uint32_t>(e.npad >> 4) << 12) |
+         (static_cast<uint32_t>(e.nvalid) << 16) | (e.prefix ? (1u << 24) : 0u);
+}
+__device__ __forceinline__ int blk_id(uint32_t e) { return static_cast<int>(e & 0xFFFu); }
+__device__ __forceinline__ int blk_npad(uint32_t e) { return static_cast<int>((e >> 12) & 0xFu) << 4; }
+__device__ __forceinline__ int blk_nvalid(uint32_t e) { return static_cast<int>((e >> 16) & 0xFFu); }
+__device__ __forceinline__ bool blk_prefix(uint32_t e) { return (e >> 24) & 1u; }
 
 __device__ __forceinline__ void decode_tile(const Geo& g, int tile, int& bhi, int& qb) {
   bhi = tile / g.nB;
@@ -208,9 +208,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kNV; ++i) { mbar_init(&bars.v_full[i], 1); mbar_init(&bars.v_empty[i], 1); }
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.p_full[i], kSoftWarps / 2);
-      mbar_init(&bars.pv_done[i], 1);
+      mbar_init(&bars.s_empty[i], kSoftWarps / 2);
     }
+    for (int i = 0; i < kNP; ++i) mbar_init(&bars.p_full[i], kSoftWarps / 2);
+    for (int i = 0; i < 3; ++i) mbar_init(&bars.pv_done[i], 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&bars.xbar[i], 2);
       mbar_init(&bars.xread[i], 2);
@@ -218,8 +219,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       mbar_init(&bars.hb[1][i], 1);
     }
     mbar_init(&bars.o_empty, kSoftWarps);
-    for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 1 + kSoftWarps); }
-    mbar_init(&bars.fin, 1);
+    for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 3 + kSoftWarps); }
+    mbar_init(&bars.fin[0], 1);
+    mbar_init(&bars.fin[1], 1);
     bars.abort = 0;
     fence_barrier_init();
   }
@@ -256,7 +258,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
      return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err));
    };
    if (warp == 0) {
-    // ------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------ tile queue, Q and K
+    // Takes the next tile, publishes it with its kept-block list (all 32 lanes: each
+    // lane expands two mask words, placed by a popcount scan), then loads Q and the K
+    // tiles.  V has its own loader (warp 3) so that the K ring never waits on a P.V.
     uint32_t tcount = 0;
     bool ok = true;
     while (ok) {
@@ -266,13 +271,33 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int tile = pos < prm.ntiles ? __ldg(prm.order + pos) : -1;
       const int slot = tcount % kTR;
       if (!wwait(&bars.t_empty[slot], ((tcount / kTR) & 1) ^ 1)) break;
-      if (tile >= 0 && prm.mask != nullptr) {
-        const uint32_t* src = prm.mask + static_cast<size_t>(tile) * g.words;
-        for (int w = lane; w < g.words; w += 32) bars.mrow[slot][w] = __ldg(src + w);
+      int nkv = 0;
+      if (tile >= 0) {
+        uint32_t* bl = bars.blist[slot];
+        if (prm.mask != nullptr) {
+          const uint32_t* src = prm.mask + static_cast<size_t>(tile) * g.words;
+          const uint32_t w0 = lane < g.words ? __ldg(src + lane) : 0u;
+          const uint32_t w1 = lane + 32 < g.words ? __ldg(src + lane + 32) : 0u;
+          int i0 = __popc(w0), i1 = __popc(w1);
+#pragma unroll
+          for (int o = 1; o < 32; o <<= 1) {
+            const int a0 = __shfl_up_sync(0xffffffffu, i0, o), a1 = __shfl_up_sync(0xffffffffu, i1, o);
+            if (lane >= o) { i0 += a0; i1 += a1; }
+          }
+          const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
+          int p0 = i0 - __popc(w0), p1 = tot0 + i1 - __popc(w1);
+          for (uint32_t bits = w0; bits; bits &= bits - 1) bl[p0++] = pack_blk(g, lane * 32 + __ffs(bits) - 1);
+          for (uint32_t bits = w1; bits; bits &= bits - 1) bl[p1++] = pack_blk(g, (lane + 32) * 32 + __ffs(bits) - 1);
+          nkv = tot0 + __shfl_sync(0xffffffffu, i1, 31);
+        } else {
+          for (int i = lane; i < g.nB; i += 32) bl[i] = pack_blk(g, i);
+          nkv = g.nB;
+        }
       }
       __syncwarp();
       if (lane == 0) {
         bars.tile[slot] = tile;
+        bars.bcount[slot] = nkv;
         mbar_arrive(&bars.t_full[slot]);
       }
       __syncwarp();
@@ -290,11 +315,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       }
       __syncwarp();
       ++qc;
-      KvIter it;
-      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
       const int full_rows = g.bt * g.bh * g.bw;
-      for (int kb = it.advance(); kb >= 0; kb = it.advance()) {
-        const BlkEnt ki = blk_of(g, kb);
+      for (int n = 0; n < nkv; ++n) {
+        const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][n]));
         const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
         const bool xedge = ki.rows != full_rows;
         const int ks = kc % kNK;
@@ -307,6 +330,26 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         __syncwarp();
         ++kc;
+      }
+    }
+   } else if (warp == 3) {
+    // ------------------------------------------------------------ V loader
+    uint32_t tcount = 0;
+    bool ok = true;
+    while (ok) {
+      const int slot = tcount % kTR;
+      if (!wwait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
+      const int tile = bars.tile[slot];
+      const int nkv = bars.bcount[slot];
+      ++tcount;
+      if (tile < 0) break;
+      int bhi, qb;
+      decode_tile(g, tile, bhi, qb);
+      const int full_rows = g.bt * g.bh * g.bw;
+      for (int n = 0; n < nkv; ++n) {
+        const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][n]));
+        const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
+        const bool xedge = ki.rows != full_rows;
         const int vs = vc % kNV;
         if (!wwait(&bars.v_empty[vs], ((vc / kNV) & 1) ^ 1)) { ok = false; break; }
         if (elect_one()) {
@@ -318,20 +361,19 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         __syncwarp();
         ++vc;
       }
+      if (!ok) break;
+      if (lane == 0) mbar_arrive(&bars.t_empty[slot]);   // done with the tile's block list
     }
    } else if (warp == 1) {
-    // ------------------------------------------------------------ MMA issuer
-    // Block j of the call's running block count c lives in S slot c mod kNS; S_c
-    // overwrites P_c-kNS, so it waits for that P.V.  O is one accumulator: the P.V
-    // products go in block order.  The S stream and the P.V stream are each issued in
-    // block order and interleave as their inputs become ready (non-blocking probes),
-    // which keeps every ring barrier at most one phase ahead of its probe.
-    uint32_t tcount = 0, mqc = 0, tiles = 0;
-    uint32_t gc = 0;                      // blocks issued so far (all tiles): ring position
-    const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+    // ------------------------------------------------------------ S issuer
+    // Block j of the call's running block count c: S_c = Q K_c^T into S slot c mod kNS,
+    // once the softmax group has loaded S_c-kNS out of it.  The S and the P.V products come
+    // from two warps: an MMA issue blocks while the tensor core's queue is full, so one
+    // warp's waits and bookkeeping overlap the other warp's issue.
+    uint32_t tcount = 0, mqc = 0;
+    uint32_t gc = 0;                      // blocks of all tiles so far: ring position
     const uint64_t dQ = sdesc_sw128(sQ, 16, 1024);
     const uint64_t dK0 = sdesc_sw128(sK(0), 16, 1024);
-    const uint64_t dV0 = sdesc_sw128(sV(0), kChunkBytes, 1024);
     bool ok = true;
     while (ok) {
       const int slot = tcount % kTR;
@@ -339,100 +381,79 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int tile = bars.tile[slot];
       ++tcount;
       if (tile < 0) break;
+      const int nkv = bars.bcount[slot];
       if (!wwait(&bars.q_full, mqc & 1)) break;
       ++mqc;
-      KvIter it;
-      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
-      uint32_t npk = 0;                 // npad/16 of blocks j..j+7, 4 bits each (ring)
-      int nknown = 0;
-      bool ended = false;
-      int sn = 0, vn = 0;               // next S / next P.V block index of the tile
-      uint64_t t_prog = globaltimer();
-      uint32_t idle = 0;
-      while (true) {
-        while (!ended && nknown <= sn) {
-          const int kb = it.advance();
-          if (kb < 0) { ended = true; break; }
-          const uint32_t sh = 4u * (nknown & 7);
-          npk = (npk & ~(0xFu << sh)) | (static_cast<uint32_t>(blk_of(g, kb).npad >> 4) << sh);
-          ++nknown;
-        }
-        bool progressed = false;
-        // ---- S_sn
-        if (sn < nknown && vn > sn - kNS) {
-          const uint32_t c = gc + sn;
-          const int ss = c % kNS;
-          const int ks = c % kNK;
-          bool rdy = mbar_test(&bars.k_full[ks], (c / kNK) & 1);
-          if (rdy && c >= kNS) rdy = mbar_test(&bars.pv_done[ss], ((c - kNS) / kNS) & 1);
-          if (__all_sync(0xffffffffu, rdy)) {
-            tc_fence_after();
-            const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
-            const uint32_t tS = tmem + kColS + ss * 128;
-            const uint32_t np = ((npk >> (4u * (sn & 7))) & 0xFu) << 4;
-            const uint32_t idesc_s = idesc_bf16_f32(128, np, 0, 0);
-            if (elect_one()) {
+      int n = 0;
+      for (; n < nkv; ++n) {
+        const uint32_t c = gc + n;
+        const int ss = c % kNS;
+        const int ks = c % kNK;
+        const uint32_t idesc_s = idesc_bf16_f32(128, blk_npad(bars.blist[slot][n]), 0, 0);
+        if (!wwait(&bars.k_full[ks], (c / kNK) & 1)) { ok = false; break; }
+        if (c >= kNS && !wwait(&bars.s_empty[ss], ((c - kNS) / kNS) & 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
+        const uint32_t tS = tmem + kColS + ss * 128;
+        if (elect_one()) {
 #pragma unroll
-              for (int q = 0; q < D / 16; ++q) {
-                const uint64_t off =
-                    static_cast<uint64_t>(((q >> 2) * kChunkBytes + (q & 3) * 32) >> 4);
-                mma_ss(tS, dQ + off, dK + off, idesc_s, q > 0 ? 1u : 0u);
-              }
-              mma_commit(&bars.s_full[ss]);
-              mma_commit(&bars.k_empty[ks]);
-            }
-            __syncwarp();
-            ++sn;
-            progressed = true;
+          for (int q = 0; q < D / 16; ++q) {
+            const uint64_t off = static_cast<uint64_t>(((q >> 2) * kChunkBytes + (q & 3) * 32) >> 4);
+            mma_ss(tS, dQ + off, dK + off, idesc_s, q > 0 ? 1u : 0u);
           }
+          mma_commit(&bars.s_full[ss]);
+          mma_commit(&bars.k_empty[ks]);
         }
-        // ---- O += P_vn V_vn
-        if (vn < sn) {
-          const uint32_t c = gc + vn;
-          const int ss = c % kNS;
-          const int vs = c % kNV;
-          bool rdy = mbar_test(&bars.p_full[ss], (c / kNS) & 1);
-          if (rdy) rdy = mbar_test(&bars.v_full[vs], (c / kNV) & 1);
-          if (rdy && vn == 0) rdy = mbar_test(&bars.o_empty, (tiles & 1) ^ 1);
-          if (__all_sync(0xffffffffu, rdy)) {
-            tc_fence_after();
-            const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
-            const uint32_t tP = tmem + kColS + ss * 128;
-            const int nk = (npk >> (4u * (vn & 7))) & 0xFu;
-            if (elect_one()) {
-#pragma unroll
-              for (int q = 0; q < 8; ++q) {
-                if (q < nk)
-                  mma_ts(tmem + kColO, tP + q * 8, dV + static_cast<uint64_t>((q * 2048) >> 4),
-                         idesc_pv, (vn == 0 && q == 0) ? 0u : 1u);
-              }
-              mma_commit(&bars.v_empty[vs]);
-              mma_commit(&bars.pv_done[ss]);
-            }
-            __syncwarp();
-            ++vn;
-            progressed = true;
-          }
-        }
-        if (ended && vn >= nknown) break;
-        if (progressed) {
-          idle = 0;
-          t_prog = globaltimer();
-        } else if ((++idle & 63u) == 0) {
-          if (*abort) { ok = false; break; }
-          if (globaltimer() - t_prog > 2000000000ull) {
-            *abort = 1;
-            if (lane == 0) atomicOr(err, kErrTimeout);
-            ok = false;
-            break;
-          }
-        }
+        __syncwarp();
       }
       if (!ok) break;
-      gc += nknown;
-      if (elect_one()) mma_commit(&bars.q_empty);
+      gc += n;
+      if (elect_one()) mma_commit(&bars.q_empty);      // the tile's last S has read Q
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.t_empty[slot]);   // done with the tile's mask row
+    }
+   } else if (warp == 2) {
+    // ------------------------------------------------------------ P.V issuer
+    // O += P_c V_c in block order (one accumulator), P_c from P slot c mod kNP.
+    uint32_t tcount = 0, tiles = 0;
+    uint32_t gc = 0;
+    const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
+    const uint64_t dV0 = sdesc_sw128(sV(0), kChunkBytes, 1024);
+    bool ok = true;
+    while (ok) {
+      const int slot = tcount % kTR;
+      if (!wwait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
+      const int tile = bars.tile[slot];
+      const int nkv = bars.bcount[slot];
+      ++tcount;
+      if (tile < 0) break;
+      int n = 0;
+      for (; n < nkv; ++n) {
+        const uint32_t c = gc + n;
+        const int ps = c % kNP;
+        const int vs = c % kNV;
+        const int nk = blk_npad(bars.blist[slot][n]) >> 4;
+        if (!wwait(&bars.p_full[ps], (c / kNP) & 1)) { ok = false; break; }
+        if (!wwait(&bars.v_full[vs], (c / kNV) & 1)) { ok = false; break; }
+        if (n == 0 && !wwait(&bars.o_empty, (tiles & 1) ^ 1)) { ok = false; break; }
+        tc_fence_after();
+        const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
+        const uint32_t tP = tmem + col_p<D>() + ps * 64;
+        if (elect_one()) {
+#pragma unroll
+          for (int q = 0; q < 8; ++q) {
+            if (q < nk)
+              mma_ts(tmem + kColO, tP + q * 8, dV + static_cast<uint64_t>((q * 2048) >> 4), idesc_pv,
+                     (n == 0 && q == 0) ? 0u : 1u);
+          }
+          mma_commit(&bars.v_empty[vs]);
+          mma_commit(&bars.pv_done[c % 3]);
+        }
+        __syncwarp();
+      }
+      if (!ok) break;
+      gc += n;
+      if (lane == 0) mbar_arrive(&bars.t_empty[slot]);
       ++tiles;
     }
    }
@@ -453,6 +474,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS0 = tmem + lane_off + kColS;
+    const uint32_t tP0 = tmem + lane_off + col_p<D>();
     const uint32_t tO = tmem + lane_off + kColO;
     uint32_t tcount = 0, xn = 0, hr = 0;
     uint32_t gc = 0;                    // blocks of all earlier tiles: S ring position
@@ -473,42 +495,52 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int token = box_row_token(g, qi, row);
 
       float m = -INFINITY, l = 0.f;     // this group's latest reference and its row sum
-      int j = 0;
+      const int nkv = bars.bcount[slot];
+      const uint32_t* bl = bars.blist[slot];
       bool ok = true;
-      KvIter it;
-      it.init(prm.mask ? bars.mrow[slot] : nullptr, g.nB, g.words);
-      for (int kb = it.advance(); kb >= 0; kb = it.advance(), ++j) {
-        if ((j & 1) != grp) continue;
+      for (int j = grp; j < nkv; j += 2) {
+        const uint32_t e = bl[j];
         const uint32_t c = gc + j;
         const int ss = c % kNS;
         const uint32_t tS = tS0 + ss * 128;
-        const BlkEnt ki = blk_of(g, kb);
-        const bool full = ki.prefix && ki.nvalid >= 128;
+        const uint32_t tP = tP0 + (c % kNP) * 64;
+        const int nvalid = blk_nvalid(e);
+        const bool full = blk_prefix(e) && nvalid >= 128;
+        const int nact = (blk_npad(e) + 31) >> 5;   // 32-column chunks below npad (uniform)
+        // valid keys of each chunk: a prefix of the box, or (time and height edge at
+        // once) read off the box geometry
         uint32_t vm[4];
-        if (ki.prefix) {
+        if (blk_prefix(e)) {
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4) {
-            const int nn = ki.nvalid - 32 * w4;
+            const int nn = nvalid - 32 * w4;
             vm[w4] = nn >= 32 ? 0xffffffffu : (nn <= 0 ? 0u : ((1u << nn) - 1u));
           }
         } else {
+          const BlockInfo bi = block_info(g, blk_id(e));
 #pragma unroll
           for (int w4 = 0; w4 < 4; ++w4)
-            vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, block_info(g, kb), 32 * w4 + lane) >= 0);
+            vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, bi, 32 * w4 + lane) >= 0);
         }
         if (!sync_wait(&bars.s_full[ss], (c / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
-        // The whole row of S in one TMEM round trip (loads are grouped, then one wait:
-        // a TMEM store issued after a load waits for it, so loads and stores are not
-        // interleaved).
+        // The whole row of S in one TMEM round trip (loads are grouped, then one wait).
         float s[128];
 #pragma unroll
         for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, reinterpret_cast<uint32_t*>(s + 32 * q));
         tmem_wait_ld();
-        const int nact = (ki.npad + 31) >> 5;    // 32-column chunks below npad (uniform)
-        if (!full) {
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(&bars.s_empty[ss]);    // the slot may take S_c+2
+        // Invalid keys to -inf in the chunks that hold some; chunks at or past npad (not
+        // written by this S) are left out of the maximum and of P.
 #pragma unroll
-          for (int q = 0; q < 128; ++q) s[q] = ((vm[q >> 5] >> (q & 31)) & 1u) ? s[q] : -INFINITY;
+        for (int r = 0; r < 4; ++r) {
+          if (r < nact && vm[r] != 0xffffffffu) {
+#pragma unroll
+            for (int q = 0; q < 32; ++q)
+              s[32 * r + q] = ((vm[r] >> q) & 1u) ? s[32 * r + q] : -INFINITY;
+          }
         }
         float mq[4];
 #pragma unroll
@@ -516,7 +548,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           float mm = max3f(s[32 * r], s[32 * r + 1], s[32 * r + 2]);
 #pragma unroll
           for (int q = 3; q < 31; q += 2) mm = max3f(mm, s[32 * r + q], s[32 * r + q + 1]);
-          mq[r] = fmaxf(mm, s[32 * r + 31]);
+          mq[r] = r < nact ? fmaxf(mm, s[32 * r + 31]) : -INFINITY;
         }
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
         // reference after block j-1, from the other group
@@ -541,7 +573,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // has finished; re-base it before P_j goes in.
         if (__any_sync(0xffffffffu, rebase)) {
           const uint32_t cp = c - 1;
-          if (!sync_wait(&bars.pv_done[cp % kNS], (cp / kNS) & 1)) { ok = false; break; }
+          if (!sync_wait(&bars.pv_done[cp % 3], (cp / 3) & 1)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
@@ -556,9 +588,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // this group's row sum follows the reference (unchanged unless a group re-based)
         if (mref != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mref);
         m = mref;
+        // P slot c mod kNP is free once P.V c-kNP has read it (long done: it is this
+        // group's previous block)
+        if (c >= kNP) {
+          const uint32_t cp = c - kNP;
+          if (!sync_wait(&bars.pv_done[cp % 3], (cp / 3) & 1)) { ok = false; break; }
+          tc_fence_after();
+        }
         // P = 2^(s * scale * log2 e - m), packed to bf16 pairs and stored 16 keys at a
-        // time over S columns already read (P column k/2 holds keys k, k+1).  Chunks at
-        // or past npad are neither computed nor stored: the P.V reads keys < npad only.
+        // time (P column k/2 holds keys k, k+1).  Chunks at or past npad are neither
+        // computed nor stored: the P.V reads keys < npad only.
         const uint64_t nmx2 = f32x2(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
 #pragma unroll
@@ -582,7 +621,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 acc[e & 3] = fadd2(acc[e & 3], f32x2(p0, p1));
                 pk[e] = pack_bf16x2(p0, p1);
               }
-              tmem_st8(tS + 16 * c32 + 8 * h, pk);
+              tmem_st8(tP + 16 * c32 + 8 * h, pk);
             }
           }
         }
@@ -593,11 +632,10 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[ss]);
+        if (lane == 0) mbar_arrive(&bars.p_full[c % kNP]);
       }
       if (!ok) break;
       // ---- epilogue
-      const int nkv = j;
       gc += nkv;
       float mf = m;                      // final reference of the tile
       if (nkv > 0 && ((nkv - 1) & 1) != grp) {
@@ -608,7 +646,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (mf != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mf);
       if (nkv > 0) {
         const uint32_t cl = gc - 1;      // the tile's last P.V
-        if (!sync_wait(&bars.pv_done[cl % kNS], (cl / kNS) & 1)) break;
+        if (!sync_wait(&bars.pv_done[cl % 3], (cl / 3) & 1)) break;
       }
       if (xn > 0 && !sync_wait(&bars.xread[quarter], (xn - 1) & 1)) break;
       bars.xl[grp][row] = l;
@@ -656,7 +694,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
   if (bars.abort) {
     // Drain: let every armed TMA copy land and every issued MMA finish before the
     // shared and tensor memory they touch is released.  Bounded, abort ignored.
-    if (warp == 0 && lane == 0) {
+    if ((warp == 0 || warp == 3) && lane == 0) {   // each loader's copies (Q, K / V)
       int never = 0;
       volatile int* nv = &never;
       if (qc > 0) mbar_wait(&bars.q_full, (qc - 1) & 1, nv, nullptr, 100000000ull);
@@ -665,11 +703,11 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       for (uint32_t i = (vc > kNV ? vc - kNV : 0); i < vc; ++i)
         mbar_wait(&bars.v_full[i % kNV], (i / kNV) & 1, nv, nullptr, 100000000ull);
     }
-    if (warp == 1 && lane == 0) {
+    if ((warp == 1 || warp == 2) && lane == 0) {   // each issuer's MMAs
       int never = 0;
       volatile int* nv = &never;
-      mma_commit(&bars.fin);
-      mbar_wait(&bars.fin, 0, nv, nullptr, 100000000ull);
+      mma_commit(&bars.fin[warp - 1]);
+      mbar_wait(&bars.fin[warp - 1], 0, nv, nullptr, 100000000ull);
     }
   }
   tc_fence_before();
