@@ -38,7 +38,7 @@ METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16
 
 # DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
 # `ncu --set full` capture; valid only for the kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "a686b3a7a8a5028d", "bytes": 390201344}
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "813a70c1c8f5e0e2", "bytes": 391571200}
 
 
 def attn_traffic():
