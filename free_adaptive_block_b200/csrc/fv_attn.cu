@@ -61,13 +61,6 @@ constexpr uint32_t kColO = 128 * kNS;  // O: columns [256, 256 + d)
 template <int D> __host__ __device__ constexpr uint32_t col_p() { return kColO + D; }   // P slot r: +64r
 static_assert(col_p<128>() + 64 * kNP <= 512, "tensor memory layout exceeds 512 columns");
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
-#ifndef FV_POLY_EVERY
-#define FV_POLY_EVERY 0
-#endif
-// When nonzero, one exponential pair in kPolyEvery (interior blocks) goes to the FMA
-// pipe (ex2_poly2) instead of the MUFU unit.  Off by default: measured slower so far.
-constexpr int kPolyEvery = FV_POLY_EVERY;
-
 // True in exactly one lane of the (converged) warp.
 __device__ __forceinline__ bool elect_one() {
   uint32_t pred;
@@ -81,31 +74,6 @@ __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
   asm("max.f32 %0, %1, %2, %3;" : "=f"(r) : "f"(a), "f"(b), "f"(c));
   return r;
-}
-
-// 2^x for a pair of x <= 8 on the FMA pipe (Blackwell f32x2 arithmetic), for the P
-// values of the online softmax.  Cody-Waite style range reduction x = j + f with
-// j = round(x), f in [-1/2, 1/2] (adding 1.5 * 2^23 leaves j in the low mantissa
-// bits), a degree-3 polynomial for 2^f whose coefficients are this file's own minimax
-// (Remez exchange) fit of the relative error on [-1/2, 1/2] (max relative error
-// 7.5e-5, far below the 2^-9 of the bf16 P it feeds), and 2^j added to the exponent
-// field with one integer multiply-add.  x is clamped at -125 so the exponent field
-// cannot underflow; 2^-125 is 2e-38, nothing next to the row's terms.
-__device__ __forceinline__ void ex2_poly2(float xa, float xb, float& ya, float& yb) {
-  const uint64_t x = f32x2(fmaxf(xa, -125.0f), fmaxf(xb, -125.0f));
-  const uint64_t magic = f32x2(12582912.0f, 12582912.0f);
-  const uint64_t t = fadd2(x, magic);
-  const uint64_t jf = fsub2(t, magic);
-  const uint64_t f = fsub2(x, jf);
-  uint64_t p = ffma2(f32x2(0.0551716685295105f, 0.0551716685295105f), f,
-                     f32x2(0.2426111251115799f, 0.2426111251115799f));
-  p = ffma2(p, f, f32x2(0.6932609677314758f, 0.6932609677314758f));
-  p = ffma2(p, f, f32x2(0.9999280571937561f, 0.9999280571937561f));
-  float pa, pb, ta, tb;
-  unpack_f32x2(p, pa, pb);
-  unpack_f32x2(t, ta, tb);
-  ya = __uint_as_float(__float_as_uint(ta) * 8388608u + __float_as_uint(pa));
-  yb = __uint_as_float(__float_as_uint(tb) * 8388608u + __float_as_uint(pb));
 }
 
 struct AttnParams {
@@ -157,16 +125,22 @@ __host__ __device__ constexpr int attn_smem_bytes() {
 static_assert(attn_smem_bytes<128>() <= 232448, "attention kernel exceeds 227 KB of shared memory");
 
 // One kept block of a tile as the consumers need it: block id (bits 0-11), npad / 16
-// (12-15), real token count (16-23), real tokens form a prefix of the box (24).
+// (12-15), real token count (16-23), real tokens form a prefix of the box (24), some
+// keys of the 32-key chunks the softmax reads (those below npad) are not real tokens
+// and must be masked (25): a box with gaps, or a real-token count that is not a
+// multiple of 32 (the S MMA writes npad columns; the rest of the last chunk is stale).
 __device__ __forceinline__ uint32_t pack_blk(const Geo& g, int kb) {
   const BlkEnt e = blk_of(g, kb);
+  const bool need_mask = !e.prefix || (e.nvalid & 31) != 0;
   return static_cast<uint32_t>(kb) | (static_cast<uint32_t>(e.npad >> 4) << 12) |
-         (static_cast<uint32_t>(e.nvalid) << 16) | (e.prefix ? (1u << 24) : 0u);
+         (static_cast<uint32_t>(e.nvalid) << 16) | (e.prefix ? (1u << 24) : 0u) |
+         (need_mask ? (1u << 25) : 0u);
 }
 __device__ __forceinline__ int blk_id(uint32_t e) { return static_cast<int>(e & 0xFFFu); }
 __device__ __forceinline__ int blk_npad(uint32_t e) { return static_cast<int>((e >> 12) & 0xFu) << 4; }
 __device__ __forceinline__ int blk_nvalid(uint32_t e) { return static_cast<int>((e >> 16) & 0xFFu); }
 __device__ __forceinline__ bool blk_prefix(uint32_t e) { return (e >> 24) & 1u; }
+__device__ __forceinline__ bool blk_needmask(uint32_t e) { return (e >> 25) & 1u; }
 
 __device__ __forceinline__ void decode_tile(const Geo& g, int tile, int& bhi, int& qb) {
   bhi = tile / g.nB;
@@ -504,24 +478,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const int ss = c % kNS;
         const uint32_t tS = tS0 + ss * 128;
         const uint32_t tP = tP0 + (c % kNP) * 64;
-        const int nvalid = blk_nvalid(e);
-        const bool full = blk_prefix(e) && nvalid >= 128;
         const int nact = (blk_npad(e) + 31) >> 5;   // 32-column chunks below npad (uniform)
-        // valid keys of each chunk: a prefix of the box, or (time and height edge at
-        // once) read off the box geometry
-        uint32_t vm[4];
-        if (blk_prefix(e)) {
-#pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4) {
-            const int nn = nvalid - 32 * w4;
-            vm[w4] = nn >= 32 ? 0xffffffffu : (nn <= 0 ? 0u : ((1u << nn) - 1u));
-          }
-        } else {
-          const BlockInfo bi = block_info(g, blk_id(e));
-#pragma unroll
-          for (int w4 = 0; w4 < 4; ++w4)
-            vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, bi, 32 * w4 + lane) >= 0);
-        }
         if (!sync_wait(&bars.s_full[ss], (c / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
         // The whole row of S in one TMEM round trip (loads are grouped, then one wait).
@@ -532,39 +489,56 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_empty[ss]);    // the slot may take S_c+2
-        // Invalid keys to -inf in the chunks that hold some; chunks at or past npad (not
-        // written by this S) are left out of the maximum and of P.
+        // Keys that are not real tokens (a partial last 16-key group, or the gaps of a box
+        // cut at the time and height edges at once) to -inf.  One warp-uniform branch,
+        // taken only by such blocks, so the common path carries none of this code.
+        if (blk_needmask(e)) {
+          uint32_t vm[4];
+          if (blk_prefix(e)) {
+            const int nvalid = blk_nvalid(e);
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          if (r < nact && vm[r] != 0xffffffffu) {
+            for (int w4 = 0; w4 < 4; ++w4) {
+              const int nn = nvalid - 32 * w4;
+              vm[w4] = nn >= 32 ? 0xffffffffu : (nn <= 0 ? 0u : ((1u << nn) - 1u));
+            }
+          } else {
+            const BlockInfo bi = block_info(g, blk_id(e));
 #pragma unroll
-            for (int q = 0; q < 32; ++q)
-              s[32 * r + q] = ((vm[r] >> q) & 1u) ? s[32 * r + q] : -INFINITY;
+            for (int w4 = 0; w4 < 4; ++w4)
+              vm[w4] = __ballot_sync(0xffffffffu, box_row_token(g, bi, 32 * w4 + lane) >= 0);
+          }
+#pragma unroll
+          for (int r = 0; r < 4; ++r) {
+            if (r < nact && vm[r] != 0xffffffffu) {
+#pragma unroll
+              for (int q = 0; q < 32; ++q)
+                s[32 * r + q] = ((vm[r] >> q) & 1u) ? s[32 * r + q] : -INFINITY;
+            }
           }
         }
+        // Row maximum of each chunk as a shallow tree (depth 4 instead of a 16-long chain).
         float mq[4];
 #pragma unroll
         for (int r = 0; r < 4; ++r) {
-          float mm = max3f(s[32 * r], s[32 * r + 1], s[32 * r + 2]);
+          const float* x = s + 32 * r;
+          float t[11];
 #pragma unroll
-          for (int q = 3; q < 31; q += 2) mm = max3f(mm, s[32 * r + q], s[32 * r + q + 1]);
-          mq[r] = r < nact ? fmaxf(mm, s[32 * r + 31]) : -INFINITY;
+          for (int k = 0; k < 10; ++k) t[k] = max3f(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+          t[10] = fmaxf(x[30], x[31]);
+          const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
+          const float u2 = max3f(t[6], t[7], t[8]), u3 = max3f(t[9], t[10], u0);
+          mq[r] = r < nact ? max3f(u1, u2, u3) : -INFINITY;
         }
         const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
         // reference after block j-1, from the other group
-        float mref = mx;
+        float mref = mx, mp = mx;
         bool rebase = false;
-        float alpha = 1.f;
         if (j > 0) {
           if (!sync_wait(&bars.hb[grp ^ 1][quarter], hr & 1)) { ok = false; break; }
           ++hr;
-          const float mp = bars.hv[grp ^ 1][row];
-          mref = mp;
-          if (mx > mp + kRebase) {
-            mref = mx;
-            alpha = ex2(mp - mx);
-            rebase = true;
-          }
+          mp = bars.hv[grp ^ 1][row];
+          rebase = mx > mp + kRebase;
+          mref = rebase ? mx : mp;
         }
         bars.hv[grp][row] = mref;
         __syncwarp();
@@ -572,6 +546,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // O holds P_0 V_0 + ... + P_j-1 V_j-1 against the old reference once P.V j-1
         // has finished; re-base it before P_j goes in.
         if (__any_sync(0xffffffffu, rebase)) {
+          const float alpha = rebase ? ex2(mp - mx) : 1.f;
           const uint32_t cp = c - 1;
           if (!sync_wait(&bars.pv_done[cp % 3], (cp / 3) & 1)) { ok = false; break; }
           tc_fence_after();
@@ -585,8 +560,12 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             tmem_st32(tO + 32 * q, o);
           }
         }
-        // this group's row sum follows the reference (unchanged unless a group re-based)
-        if (mref != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mref);
+        // this group's row sum follows the reference (unchanged unless a group re-based;
+        // l is still 0 before the group's first block of the tile)
+        const bool lscale = mref != m && m != -INFINITY;
+        if (__any_sync(0xffffffffu, lscale)) {
+          if (lscale) l *= ex2(m - mref);
+        }
         m = mref;
         // P slot c mod kNP is free once P.V c-kNP has read it (long done: it is this
         // group's previous block)
@@ -611,13 +590,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                 const int q = 32 * c32 + 16 * h + 2 * e;
                 float x0, x1;
                 unpack_f32x2(ffma2(f32x2(s[q], s[q + 1]), sl2x2, nmx2), x0, x1);
-                float p0, p1;
-                if (full && kPolyEvery > 0 && (e % kPolyEvery) == kPolyEvery - 1) {
-                  ex2_poly2(x0, x1, p0, p1);
-                } else {
-                  p0 = ex2(x0);
-                  p1 = ex2(x1);
-                }
+                const float p0 = ex2(x0), p1 = ex2(x1);
                 acc[e & 3] = fadd2(acc[e & 3], f32x2(p0, p1));
                 pk[e] = pack_bf16x2(p0, p1);
               }

@@ -40,7 +40,7 @@ struct BlockInfo {
   int tb, yb, xb;    // block coordinates
   int rt, ry, rx;    // real extents (clipped to the latent)
   int rows;          // rows of the loaded box: bt * bh * rx (x is loaded compactly)
-  int npad;          // rows rounded up to 16 (MMA N / K granularity)
+  int npad;          // rows the MMAs read, rounded up to 16 (MMA N / K granularity)
   int nvalid;        // when `prefix`: the real rows are exactly rows [0, nvalid)
   bool prefix;
   bool xedge;        // rx < bw: the block is loaded with the narrow tensor map
@@ -57,9 +57,11 @@ __host__ __device__ inline BlockInfo block_info(const Geo& g, int j) {
   b.ry = min(g.bh, g.Hs - b.yb * g.bh);
   b.rx = min(g.bw, g.Ws - b.xb * g.bw);
   b.rows = g.bt * g.bh * b.rx;
-  b.npad = (b.rows + 15) & ~15;
   b.prefix = (g.bt == 1) || (b.ry == g.bh);
   b.nvalid = b.rt * b.ry * b.rx;   // the real token count (a prefix of the box when `prefix`)
+  // Rows the MMAs use: when the real tokens are a prefix of the box, the rows past them
+  // (zero fill at the latent's H or T edge) are left out of S and P.V altogether.
+  b.npad = ((b.prefix ? b.nvalid : b.rows) + 15) & ~15;
   b.xedge = b.rx < g.bw;
   return b;
 }
@@ -172,18 +174,25 @@ __device__ __forceinline__ uint32_t smid() {
 enum : uint32_t { kErrTimeout = 1u, kErrLayout = 2u };
 
 // A bounded wait on an mbarrier phase.  Returns false (after raising *abort and the
-// global error word) when the phase has not completed within `limit_ns`, or when
-// another thread of the CTA has already raised *abort.
+// global error word) when the phase has not completed within about `limit_ns`, or when
+// another thread of the CTA has already raised *abort.  The deadline is kept in SM
+// cycles (clock64, counted at 2 cycles per ns so that it is never shorter than the
+// limit at clocks up to 2 GHz) and starts only after 64 unsuccessful probes: the
+// %globaltimer register is slow to read, and a wait that ends within a few probes
+// should pay nothing for the deadline.  A failed try_wait suspends the thread until
+// the phase completes or a hardware time limit (a few hundred cycles) passes.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volatile int* abort,
                                           uint32_t* err, uint64_t limit_ns = 2000000000ull) {
   const uint32_t a = smem_u32(bar);
   if (mbar_try_wait(a, parity)) return true;
-  const uint64_t t0 = globaltimer();
+  long long t0 = 0;
   for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(a, parity)) return true;
     if ((i & 63u) == 0) {
       if (*abort) return false;
-      if (globaltimer() - t0 > limit_ns) {
+      if (i == 64u) {
+        t0 = clock64();
+      } else if (static_cast<uint64_t>(clock64() - t0) > 2ull * limit_ns) {
         *abort = 1;
         if (err) atomicOr(err, kErrTimeout);
         return false;
