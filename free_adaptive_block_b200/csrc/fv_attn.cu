@@ -694,10 +694,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Schedule prep: one CTA.  Resets the queue counter, the error word and the SM busy
+// Schedule prep, two kernels.
+//
+// prep_cost_kernel (one warp per tile, many CTAs): a tile's cost is its issued work,
+// the sum over its kept blocks of (keys the MMAs read + a per-block overhead).  Blocks
+// are classed by whether they sit in the last block column, row and frame (8 classes;
+// the caller passes each class's cost, read off the block geometry), so a mask word
+// costs eight popcounts.
+//
+// prep_order_kernel (one CTA): resets the queue counter, the error word and the SM busy
 // record, then writes the tile order:
-//   * a tile's cost is its issued work, sum over kept blocks of (rows padded to 16 +
-//     a per-block overhead);
 //   * (b, h) slices are ranked by total cost, heaviest first, and a slice's tiles are
 //     contiguous in the order, heaviest first (counting sort on cost buckets).
 // Grouping by slice keeps the K/V tiles that concurrently running tiles read within a
@@ -706,18 +712,61 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
 // lightest).  Order inside a bucket is arbitrary: it changes timing, never results.
 // ----------------------------------------------------------------------------
 constexpr int kPrepThreads = 1024;
+constexpr int kCostWarps = 8;
 constexpr int kHistCells = 8192;       // slices x cost buckets
 constexpr int kMaxSlices = 1024;
 constexpr int kBlockOverhead = 64;
 
-__global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_t* __restrict__ mask,
-                                                            uint32_t* hdr, int* order, int* keys,
-                                                            int ntiles,
-                                                            unsigned long long* busy, int nsm) {
+struct ClassCost {
+  int c[8];                            // cost of a block of class (x_edge | y_edge << 1 | t_edge << 2)
+};
+
+__global__ void __launch_bounds__(32 * kCostWarps) prep_cost_kernel(Geo g, const uint32_t* __restrict__ mask,
+                                                                    int* cost_out, int ntiles, ClassCost cc) {
+  __shared__ uint32_t edge[3][kMaxBlocks / 32];   // per word: last column / row / frame bits
+  for (int w = threadIdx.x; w < g.words; w += 32 * kCostWarps) {
+    uint32_t ex = 0, ey = 0, et = 0;
+    for (int i = 0; i < 32; ++i) {
+      const int j = w * 32 + i;
+      if (j >= g.nB) break;
+      const int xb = j % g.nBx, r = j / g.nBx;
+      const int yb = r % g.nBy, tb = r / g.nBy;
+      ex |= (xb == g.nBx - 1 ? 1u : 0u) << i;
+      ey |= (yb == g.nBy - 1 ? 1u : 0u) << i;
+      et |= (tb == g.nBt - 1 ? 1u : 0u) << i;
+    }
+    edge[0][w] = ex;
+    edge[1][w] = ey;
+    edge[2][w] = et;
+  }
+  __syncthreads();
+  const int lane = threadIdx.x & 31;
+  const int warp = blockIdx.x * kCostWarps + (threadIdx.x >> 5);
+  for (int tile = warp; tile < ntiles; tile += gridDim.x * kCostWarps) {
+    const uint32_t* row = mask + static_cast<size_t>(tile) * g.words;
+    int cost = 0;
+    for (int w = lane; w < g.words; w += 32) {
+      const uint32_t m = __ldg(row + w);
+      const uint32_t ex = edge[0][w], ey = edge[1][w], et = edge[2][w];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        const uint32_t sel = ((k & 1) ? ex : ~ex) & ((k & 2) ? ey : ~ey) & ((k & 4) ? et : ~et);
+        cost += cc.c[k] * __popc(m & sel);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) cost += __shfl_xor_sync(0xffffffffu, cost, off);
+    if (lane == 0) cost_out[tile] = cost;
+  }
+}
+
+__global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const uint32_t* __restrict__ mask,
+                                                                  uint32_t* hdr, int* order, int* keys,
+                                                                  int ntiles, int maxcost,
+                                                                  unsigned long long* busy, int nsm) {
   __shared__ int hist[kHistCells];
   __shared__ unsigned long long total[kMaxSlices];
   __shared__ int rank[kMaxSlices];
-  __shared__ uint32_t edge[64];
   const int t = threadIdx.x;
   if (t == 0) { hdr[0] = 0; hdr[1] = 0; }
   if (busy)
@@ -726,39 +775,40 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
     for (int i = t; i < ntiles; i += kPrepThreads) order[i] = i;
     return;
   }
-  const int words = g.words;
   const int slices = g.B * g.H;
   // slices beyond the shared tables fall back to one group (plain LPT order)
   const bool grouped = slices <= kMaxSlices;
   const int ngroups = grouped ? slices : 1;
   int nbk = kHistCells / ngroups;
   nbk = nbk >= 256 ? 256 : (nbk >= 128 ? 128 : (nbk >= 64 ? 64 : (nbk >= 32 ? 32 : (nbk >= 16 ? 16 : 8))));
-  for (int w = t; w < words; w += kPrepThreads) {
-    uint32_t bits = 0;
-    for (int i = 0; i < 32; ++i) {
-      const int j = w * 32 + i;
-      if (j < g.nB && (j % g.nBx) == g.nBx - 1) bits |= 1u << i;
-    }
-    edge[w] = bits;
-  }
   for (int i = t; i < kHistCells; i += kPrepThreads) hist[i] = 0;
   for (int i = t; i < ngroups; i += kPrepThreads) total[i] = 0ull;
   __syncthreads();
-  const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
-  const long long full = ((g.bt * g.bh * g.bw + 15) & ~15) + kBlockOverhead;
-  const long long part = ((g.bt * g.bh * rx_edge + 15) & ~15) + kBlockOverhead;
-  const long long maxcost = full * g.nB;
-  for (int i = t; i < ntiles; i += kPrepThreads) {
-    const uint32_t* row = mask + static_cast<size_t>(i) * words;
-    long long cost = 0;
-    for (int w = 0; w < words; ++w) {
-      const uint32_t m = __ldg(row + w);
-      cost += full * __popc(m) - (full - part) * __popc(m & edge[w]);
-    }
-    int key = static_cast<int>(((maxcost - cost) * nbk) / (maxcost + 1));
+  // keys[] holds the tile costs on entry and the cost buckets on exit.  Shared-memory
+  // atomics are aggregated per warp (lanes with the same slice or bucket combine first):
+  // a warp's tiles are consecutive, so they mostly share a slice and many share a bucket.
+  const int lane = t & 31;
+  const int iters = (ntiles + kPrepThreads - 1) / kPrepThreads;
+  for (int it = 0; it < iters; ++it) {
+    const int i = it * kPrepThreads + t;
+    const bool valid = i < ntiles;
+    const long long cost = valid ? keys[i] : 0;
+    int key = static_cast<int>(((maxcost - cost) * nbk) / (static_cast<long long>(maxcost) + 1));
     key = min(max(key, 0), nbk - 1);
-    keys[i] = key;
-    atomicAdd(&total[grouped ? i / g.nB : 0], static_cast<unsigned long long>(cost));
+    if (valid) keys[i] = key;
+    const int grp = valid ? (grouped ? i / g.nB : 0) : -1;
+    // one warp reduction and one atomic per distinct slice among the warp's tiles
+    uint32_t remaining = __ballot_sync(0xffffffffu, valid);
+    while (remaining) {
+      const int leader = __ffs(remaining) - 1;
+      const int lg = __shfl_sync(0xffffffffu, grp, leader);
+      const bool mine = valid && grp == lg;
+      unsigned long long v = mine ? static_cast<unsigned long long>(cost) : 0ull;
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (lane == leader) atomicAdd(&total[lg], v);
+      remaining &= ~__ballot_sync(0xffffffffu, mine);
+    }
   }
   __syncthreads();
   for (int h = t; h < ngroups; h += kPrepThreads) {
@@ -771,8 +821,12 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
     rank[h] = r;
   }
   __syncthreads();
-  for (int i = t; i < ntiles; i += kPrepThreads)
-    atomicAdd(&hist[rank[grouped ? i / g.nB : 0] * nbk + keys[i]], 1);
+  for (int it = 0; it < iters; ++it) {
+    const int i = it * kPrepThreads + t;
+    const int cell = i < ntiles ? rank[grouped ? i / g.nB : 0] * nbk + keys[i] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, cell);
+    if (cell >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[cell], __popc(peers));
+  }
   __syncthreads();
   // exclusive scan of the histogram in (slice rank, bucket) order: warp 0, 256 cells per lane
   const int cells = ngroups * nbk;
@@ -800,9 +854,15 @@ __global__ void __launch_bounds__(kPrepThreads) prep_kernel(Geo g, const uint32_
     }
   }
   __syncthreads();
-  for (int i = t; i < ntiles; i += kPrepThreads) {
-    const int pos = atomicAdd(&hist[rank[grouped ? i / g.nB : 0] * nbk + keys[i]], 1);
-    order[pos] = i;
+  for (int it = 0; it < iters; ++it) {
+    const int i = it * kPrepThreads + t;
+    const int cell = i < ntiles ? rank[grouped ? i / g.nB : 0] * nbk + keys[i] : -1;
+    const uint32_t peers = __match_any_sync(0xffffffffu, cell);
+    const int leader = __ffs(peers) - 1;
+    int base = 0;
+    if (cell >= 0 && lane == leader) base = atomicAdd(&hist[cell], __popc(peers));
+    base = __shfl_sync(peers, base, leader);
+    if (cell >= 0) order[base + __popc(peers & ((1u << lane) - 1u))] = i;
   }
 }
 
@@ -823,7 +883,23 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
   uint32_t* hdr = static_cast<uint32_t*>(ws);
   int* order = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + kWsHeader);
   int* keys = order + ntiles;
-  prep_kernel<<<1, kPrepThreads, 0, st>>>(g, mask, hdr, order, keys, ntiles, busy, nsm);
+  int maxcost = 0;
+  if (mask != nullptr) {
+    // cost of each block class, from a block of that class (last column / row / frame)
+    ClassCost cc;
+    for (int k = 0; k < 8; ++k) {
+      const int xb = (k & 1) ? g.nBx - 1 : 0, yb = (k & 2) ? g.nBy - 1 : 0, tb = (k & 4) ? g.nBt - 1 : 0;
+      const BlockInfo bi = block_info(g, (tb * g.nBy + yb) * g.nBx + xb);
+      cc.c[k] = bi.npad + kBlockOverhead;
+      maxcost = cc.c[k] > maxcost ? cc.c[k] : maxcost;
+    }
+    maxcost *= g.nB;
+    const int ctas = (ntiles + kCostWarps - 1) / kCostWarps;
+    prep_cost_kernel<<<ctas, 32 * kCostWarps, 0, st>>>(g, mask, keys, ntiles, cc);
+    cudaError_t e0 = cudaGetLastError();
+    if (e0 != cudaSuccess) return e0;
+  }
+  prep_order_kernel<<<1, kPrepThreads, 0, st>>>(g, mask, hdr, order, keys, ntiles, maxcost, busy, nsm);
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   AttnParams prm;

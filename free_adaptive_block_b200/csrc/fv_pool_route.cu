@@ -15,97 +15,84 @@
 namespace fv {
 
 // ----------------------------------------------------------------------------
-// Pooling: one CTA per (b*h, block).  Thread t owns the 16-byte chunk t % (d/8) of
-// the tokens t / (d/8), t / (d/8) + 256 / (d/8), ...  of the block; partial sums
-// are folded with warp shuffles, then across warps through shared memory.
-// Loads are 16-byte vectors, and a warp reads whole 256-byte token rows.
+// Pooling: one CTA per (block, b*h, tensor), tensor 0 = Q, 1 = K.  A block is rt * ry
+// rows of rx tokens, and the tokens of a row are contiguous in memory; warp w takes
+// rows w, w + 8, ...  Lane l owns the 16-byte chunk l % (d/8) of tokens l / (d/8),
+// l / (d/8) + 32 / (d/8), ... of the row, all of a row's loads are issued before any is
+// used, and no address needs a division.  Partial sums are folded with warp shuffles,
+// then across warps through shared memory.
 // ----------------------------------------------------------------------------
 constexpr int kPoolThreads = 256;
 
 template <int D>
-__global__ void __launch_bounds__(kPoolThreads) pool_kernel(Geo g, const uint4* __restrict__ q,
-                                                            const uint4* __restrict__ k,
-                                                            float* __restrict__ qp,
-                                                            float* __restrict__ kp) {
-  constexpr int CH = D / 8;               // 16-byte chunks per token
-  constexpr int G = kPoolThreads / CH;     // tokens processed side by side
-  constexpr int MAXR = 128 / G;            // a block holds at most 128 tokens
-  __shared__ float red[2][kPoolThreads / 32][D];
+__global__ void __launch_bounds__(kPoolThreads, 4) pool_kernel(Geo g, const uint4* __restrict__ q,
+                                                               const uint4* __restrict__ k,
+                                                               float* __restrict__ qp,
+                                                               float* __restrict__ kp) {
+  constexpr int CH = D / 8;                // 16-byte chunks per token
+  constexpr int TPI = 32 / CH;             // tokens a warp covers per load instruction
+  constexpr int NW = kPoolThreads / 32;
+  constexpr int BATCH = 8;                 // loads in flight per lane
+  __shared__ float red[NW][D];
 
   const int j = blockIdx.x;
   const int bhi = blockIdx.y;
+  const uint4* __restrict__ src = blockIdx.z ? k : q;
+  float* __restrict__ dst = blockIdx.z ? kp : qp;
   const BlockInfo bi = block_info(g, j);
-  const int nreal = bi.nvalid;
-  const int plane = bi.ry * bi.rx;
-  const int ch = threadIdx.x % CH;
-  const int grp = threadIdx.x / CH;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int ch = lane % CH, tsub = lane / CH;
   const size_t base = static_cast<size_t>(bhi) * g.N;
   const int t0 = bi.tb * g.bt, y0 = bi.yb * g.bh, x0 = bi.xb * g.bw;
 
-  uint4 vq[MAXR], vk[MAXR];
+  float a[8];
 #pragma unroll
-  for (int i = 0; i < MAXR; ++i) {
-    const int r = grp + i * G;
-    if (r < nreal) {
-      const int tt = r / plane;
-      const int r2 = r - tt * plane;
-      const int yy = r2 / bi.rx;
-      const int xx = r2 - yy * bi.rx;
-      const size_t n = base + (static_cast<size_t>(t0 + tt) * g.Hs + (y0 + yy)) * g.Ws + (x0 + xx);
-      vq[i] = __ldg(q + n * CH + ch);
-      vk[i] = __ldg(k + n * CH + ch);
-    } else {
-      vq[i] = make_uint4(0, 0, 0, 0);
-      vk[i] = make_uint4(0, 0, 0, 0);
-    }
-  }
-  float aq[8], ak[8];
+  for (int e = 0; e < 8; ++e) a[e] = 0.f;
+  const int nrows = bi.rt * bi.ry;
+  for (int row = warp; row < nrows; row += NW) {
+    const int tt = row / bi.ry, yy = row - tt * bi.ry;
+    const uint4* p = src + (base + (static_cast<size_t>(t0 + tt) * g.Hs + (y0 + yy)) * g.Ws + x0) * CH + ch;
+    for (int x = tsub; x < bi.rx; x += BATCH * TPI) {
+      uint4 v[BATCH];
 #pragma unroll
-  for (int e = 0; e < 8; ++e) aq[e] = ak[e] = 0.f;
+      for (int u = 0; u < BATCH; ++u) {
+        const int xx = x + u * TPI;
+        v[u] = xx < bi.rx ? __ldg(p + static_cast<size_t>(xx) * CH) : make_uint4(0, 0, 0, 0);
+      }
 #pragma unroll
-  for (int i = 0; i < MAXR; ++i) {
-    const uint32_t wq[4] = {vq[i].x, vq[i].y, vq[i].z, vq[i].w};
-    const uint32_t wk[4] = {vk[i].x, vk[i].y, vk[i].z, vk[i].w};
+      for (int u = 0; u < BATCH; ++u) {
+        const uint32_t w[4] = {v[u].x, v[u].y, v[u].z, v[u].w};
 #pragma unroll
-    for (int e = 0; e < 4; ++e) {
-      aq[2 * e] += __uint_as_float(wq[e] << 16);
-      aq[2 * e + 1] += __uint_as_float(wq[e] & 0xFFFF0000u);
-      ak[2 * e] += __uint_as_float(wk[e] << 16);
-      ak[2 * e + 1] += __uint_as_float(wk[e] & 0xFFFF0000u);
+        for (int e = 0; e < 4; ++e) {
+          a[2 * e] += __uint_as_float(w[e] << 16);
+          a[2 * e + 1] += __uint_as_float(w[e] & 0xFFFF0000u);
+        }
+      }
     }
   }
   // lanes l, l + CH, ... of a warp hold the same chunk
 #pragma unroll
   for (int off = CH; off < 32; off <<= 1) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      aq[e] += __shfl_xor_sync(0xffffffffu, aq[e], off);
-      ak[e] += __shfl_xor_sync(0xffffffffu, ak[e], off);
-    }
+    for (int e = 0; e < 8; ++e) a[e] += __shfl_xor_sync(0xffffffffu, a[e], off);
   }
-  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   if (lane < CH) {
 #pragma unroll
-    for (int e = 0; e < 8; ++e) {
-      red[0][warp][lane * 8 + e] = aq[e];
-      red[1][warp][lane * 8 + e] = ak[e];
-    }
+    for (int e = 0; e < 8; ++e) red[warp][lane * 8 + e] = a[e];
   }
   __syncthreads();
-  const float inv = 1.f / static_cast<float>(nreal);
-  for (int t = threadIdx.x; t < 2 * D; t += kPoolThreads) {
-    const int which = t / D, dd = t - which * D;
-    float s = 0.f;
+  const float inv = 1.f / static_cast<float>(bi.nvalid);
+  for (int t = threadIdx.x; t < D; t += kPoolThreads) {
+    float sum = 0.f;
 #pragma unroll
-    for (int w = 0; w < kPoolThreads / 32; ++w) s += red[which][w][dd];
-    float* dst = which ? kp : qp;
-    dst[(static_cast<size_t>(bhi) * g.nB + j) * D + dd] = s * inv;
+    for (int w = 0; w < NW; ++w) sum += red[w][t];
+    dst[(static_cast<size_t>(bhi) * g.nB + j) * D + t] = sum * inv;
   }
 }
 
 cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, float* kp,
                         cudaStream_t st) {
-  dim3 grid(g.nB, g.B * g.H);
+  dim3 grid(g.nB, g.B * g.H, 2);
   if (g.d == 128)
     pool_kernel<128><<<grid, kPoolThreads, 0, st>>>(g, static_cast<const uint4*>(q),
                                                      static_cast<const uint4*>(k), qp, kp);
@@ -116,9 +103,11 @@ cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, f
 }
 
 // ----------------------------------------------------------------------------
-// Routing: one CTA per (b*h, 16 query blocks); warp w owns query blocks 2w and 2w+1
-// of the CTA.  Logits come from key tiles of 32 blocks staged in shared memory (lane =
-// key block, 16-byte loads along d).  Then, per query block, with the row's logits and
+// Routing: one CTA per (b*h, 8 query blocks); warp w owns query block w of the CTA.
+// Logits: pooled key rows are staged in shared memory 128 blocks x 32 channels at a
+// time (coalesced cp.async, two stages in flight) and each lane takes one key block
+// against 4 of the CTA's 8 pooled query rows.  Then, per query block, with the row's
+// logits and
 // scores held in registers: softmax over all key blocks, and a bitwise search for the
 // Top-p cut over an order-preserving integer key of the logits, so no sort is needed:
 //   u* = the largest key with mass(key >= u*) >= p  -> the key of the m_p-th block;
@@ -126,7 +115,7 @@ cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, f
 // prefix with a second search on counts.  Reductions are warp shuffles in a fixed
 // order, so the result is deterministic.
 // ----------------------------------------------------------------------------
-constexpr int kRouteRows = 16;
+constexpr int kRouteRows = 8;
 constexpr int kRouteThreads = 256;
 
 __device__ __forceinline__ uint32_t order_key(float x) {
@@ -193,10 +182,13 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
   } else {
     for (int bit = 31; bit >= 0; --bit) {
       const uint32_t cand = u | (1u << bit);
-      float m = 0.f;
+      float m0 = 0.f, m1 = 0.f;
 #pragma unroll
-      for (int c = 0; c < MAXW; ++c) m += key[c] >= cand ? sc[c] : 0.f;
-      if (warp_sum(m) >= p) u = cand;
+      for (int c = 0; c < MAXW; c += 2) {
+        m0 += key[c] >= cand ? sc[c] : 0.f;
+        if (c + 1 < MAXW) m1 += key[c + 1] >= cand ? sc[c + 1] : 0.f;
+      }
+      if (warp_sum(m0 + m1) >= p) u = cand;
     }
     int gt = 0, eq = 0;
     float gm = 0.f, es = 0.f;
@@ -257,6 +249,17 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
   if (lane == 0) *cnt_out = cnt;
 }
 
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
+
+constexpr int kRouteKT = 128;          // key blocks per staged tile
+constexpr int kRouteDC = 32;           // channels per staged tile
+constexpr int kRouteKSP = kRouteDC + 4;  // padded tile row (floats)
+
 template <int D, int MAXW>
 __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float* __restrict__ qp,
                                                               const float* __restrict__ kp, float p,
@@ -264,12 +267,12 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
                                                               uint32_t* __restrict__ mask,
                                                               int32_t* __restrict__ counts) {
   extern __shared__ __align__(16) unsigned char route_smem[];
-  constexpr int KS = D + 4;                                      // padded key row (floats)
+  constexpr int NDC = D / kRouteDC;    // channel tiles per key row
   const int words = g.words;
   const int nBpad = words * 32;
-  float* sQ = reinterpret_cast<float*>(route_smem);              // [16][D]
-  float* sK = sQ + kRouteRows * D;                               // [32][D + 4]
-  float* sL = sK + 32 * KS;                                      // [16][nBpad]
+  float* sQ = reinterpret_cast<float*>(route_smem);              // [8][D]
+  float* sL = sQ + kRouteRows * D;                               // [8][nBpad]
+  float* sK = sL + kRouteRows * nBpad;                           // [2][128][36]
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int bhi = blockIdx.y;
@@ -277,6 +280,21 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
   const int row0 = blockIdx.x * kRouteRows;
   const float* kph = kp + static_cast<size_t>(bhi) * nB * D;
 
+  // stage st = (round, channel tile): key blocks [128 round, +128) x channels
+  // [32 tile, +32), coalesced 16-byte copies, rows past nB zero-filled
+  const int nstage = ((nB + kRouteKT - 1) / kRouteKT) * NDC;
+  auto stage = [&](int st) {
+    const int round = st / NDC, ct = st - round * NDC;
+    float* dst = sK + (st & 1) * kRouteKT * kRouteKSP;
+    for (int e = threadIdx.x; e < kRouteKT * kRouteDC / 4; e += kRouteThreads) {
+      const int key = e / (kRouteDC / 4), q4 = e - key * (kRouteDC / 4);
+      const int j = round * kRouteKT + key;
+      cp_async16(smem_u32(dst + key * kRouteKSP + 4 * q4),
+                 kph + static_cast<size_t>(j < nB ? j : 0) * D + ct * kRouteDC + 4 * q4, j < nB ? 16u : 0u);
+    }
+    cp_async_commit();
+  };
+  stage(0);
   for (int e = threadIdx.x; e < kRouteRows * D / 4; e += kRouteThreads) {
     const int r = e / (D / 4), d4 = e - r * (D / 4);
     const int row = row0 + r;
@@ -284,46 +302,55 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
         row < nB ? reinterpret_cast<const float4*>(qp + (static_cast<size_t>(bhi) * nB + row) * D)[d4]
                  : make_float4(0.f, 0.f, 0.f, 0.f);
   }
-  const float4* q0 = reinterpret_cast<const float4*>(sQ + (2 * warp) * D);
-  const float4* q1 = reinterpret_cast<const float4*>(sQ + (2 * warp + 1) * D);
-  for (int kt = 0; kt < words; ++kt) {
-    __syncthreads();
-    for (int e = threadIdx.x; e < 32 * D / 4; e += kRouteThreads) {
-      const int key = e / (D / 4), d4 = e - key * (D / 4);
-      const int j = kt * 32 + key;
-      reinterpret_cast<float4*>(sK + key * KS)[d4] =
-          j < nB ? reinterpret_cast<const float4*>(kph + static_cast<size_t>(j) * D)[d4]
-                 : make_float4(0.f, 0.f, 0.f, 0.f);
+  // Logits: warp w takes key blocks 32 (w % 4) + lane of each round against query rows
+  // 4 (w / 4) .. + 3.  Per (row, key) the sum over d runs in two partial sums (even and
+  // odd components of each float4), in ascending d, added at the end.
+  const int kgrp = warp & 3, rgrp = warp >> 2;
+  float a0[4], a1[4];
+  for (int st = 0; st < nstage; ++st) {
+    if (st + 1 < nstage) {
+      stage(st + 1);
+      cp_async_wait<1>();
+    } else {
+      cp_async_wait<0>();
     }
     __syncthreads();
-    const float4* kr = reinterpret_cast<const float4*>(sK + lane * KS);
-    float a0 = 0.f, a1 = 0.f, b0 = 0.f, b1 = 0.f;
-#pragma unroll 8
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      const float4 k4 = kr[d4], x = q0[d4], y = q1[d4];
-      a0 = fmaf(x.x, k4.x, a0); a1 = fmaf(x.y, k4.y, a1);
-      a0 = fmaf(x.z, k4.z, a0); a1 = fmaf(x.w, k4.w, a1);
-      b0 = fmaf(y.x, k4.x, b0); b1 = fmaf(y.y, k4.y, b1);
-      b0 = fmaf(y.z, k4.z, b0); b1 = fmaf(y.w, k4.w, b1);
+    const int round = st / NDC, ct = st - round * NDC;
+    if (ct == 0) {
+#pragma unroll
+      for (int r = 0; r < 4; ++r) a0[r] = a1[r] = 0.f;
     }
-    sL[(2 * warp) * nBpad + kt * 32 + lane] = (a0 + a1) * scale;
-    sL[(2 * warp + 1) * nBpad + kt * 32 + lane] = (b0 + b1) * scale;
+    const float4* kr = reinterpret_cast<const float4*>(sK + (st & 1) * kRouteKT * kRouteKSP + (32 * kgrp + lane) * kRouteKSP);
+#pragma unroll
+    for (int u = 0; u < kRouteDC / 4; ++u) {
+      const float4 k4 = kr[u];
+#pragma unroll
+      for (int r = 0; r < 4; ++r) {
+        const float4 x = reinterpret_cast<const float4*>(sQ + (4 * rgrp + r) * D)[ct * (kRouteDC / 4) + u];
+        a0[r] = fmaf(x.x, k4.x, a0[r]); a1[r] = fmaf(x.y, k4.y, a1[r]);
+        a0[r] = fmaf(x.z, k4.z, a0[r]); a1[r] = fmaf(x.w, k4.w, a1[r]);
+      }
+    }
+    if (ct == NDC - 1) {
+      const int key = round * kRouteKT + 32 * kgrp + lane;
+      if (key < nB) {
+#pragma unroll
+        for (int r = 0; r < 4; ++r) sL[(4 * rgrp + r) * nBpad + key] = (a0[r] + a1[r]) * scale;
+      }
+    }
+    __syncthreads();   // this buffer is restaged by the next iteration's prefetch
   }
-  __syncwarp();
-  for (int r = 0; r < 2; ++r) {
-    const int lr = 2 * warp + r;
-    const int qb = row0 + lr;
-    if (qb >= nB) break;
-    select_row<MAXW>(sL + lr * nBpad, nB, words, qb, p, k_floor,
+  const int qb = row0 + warp;
+  if (qb < nB)
+    select_row<MAXW>(sL + warp * nBpad, nB, words, qb, p, k_floor,
                      mask + (static_cast<size_t>(bhi) * nB + qb) * words,
                      counts + static_cast<size_t>(bhi) * nB + qb, lane);
-  }
 }
 
 size_t route_smem_bytes(const Geo& g) {
   const size_t nBpad = static_cast<size_t>(g.words) * 32;
-  return (static_cast<size_t>(kRouteRows) * g.d + 32 * static_cast<size_t>(g.d + 4) +
-          static_cast<size_t>(kRouteRows) * nBpad) * 4;
+  return (static_cast<size_t>(kRouteRows) * g.d + static_cast<size_t>(kRouteRows) * nBpad +
+          2 * static_cast<size_t>(kRouteKT) * kRouteKSP) * 4;
 }
 
 template <int D, int MAXW>
@@ -341,8 +368,16 @@ static cudaError_t launch_route_t(const Geo& g, const float* qp, const float* kp
 template <int D>
 static cudaError_t launch_route_d(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
                                   float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
+  // a lane holds MAXW logits of the row; MAXW close to the word count keeps the 32-step
+  // threshold search from running over empty slots
+  if (g.words <= 4) return launch_route_t<D, 4>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 8) return launch_route_t<D, 8>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 12) return launch_route_t<D, 12>(g, qp, kp, p, k_floor, scale, mask, counts, st);
   if (g.words <= 16) return launch_route_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 20) return launch_route_t<D, 20>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 24) return launch_route_t<D, 24>(g, qp, kp, p, k_floor, scale, mask, counts, st);
   if (g.words <= 32) return launch_route_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, st);
+  if (g.words <= 48) return launch_route_t<D, 48>(g, qp, kp, p, k_floor, scale, mask, counts, st);
   return launch_route_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, st);
 }
 
