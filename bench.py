@@ -38,7 +38,7 @@ METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16
 
 # DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
 # `ncu --set full` capture; valid only for the kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "813a70c1c8f5e0e2", "bytes": 391571200}
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "adc1da1aba719505", "bytes": 389496576}
 
 
 def attn_traffic():
@@ -272,7 +272,7 @@ def run_ours(args, rank, world, local_rank):
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
         "e2e": {"value": round(eff * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 4 * args.steps,
+        "gpu_launches": 5 * args.steps,   # pool, route, prep_cost, prep_order, attention
         "clocks": clocks,
     }
     return line
