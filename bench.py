@@ -4,8 +4,10 @@ on the Wan2.1-1.3B 480p self-attention shape (12 heads, 21x30x52 latent = 32760 
 d = 128, 3D blocks 1x8x16, p = 0.9, k_floor = 4), seeded synthetic inputs.
 
 One step = fvattn_block_pool + fvattn_route + fvattn_block_sparse_attn over the whole
-layer, inputs resident in HBM.  Each step is timed on the device with CUDA events on the
-launching stream; L2 is flushed (256 MiB write) between steps, outside the events.
+layer, inputs resident in HBM, replayed from a CUDA graph captured once (LayerGraph;
+--no-graph makes the three calls directly).  Each step is timed on the device with CUDA
+events on the launching stream; L2 is flushed (256 MiB write) between steps, outside the
+events.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference] [--sweep]
 
@@ -148,8 +150,16 @@ def run_ours(args, rank, world, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream(dev)
 
+    # The layer step: pool -> route -> attention captured once in a CUDA graph (the
+    # library's LayerGraph), so a step is five kernel launches with no host work between
+    # them; --no-graph times the three direct calls instead.
+    lg = fv.LayerGraph(g, q, k, v, wl.p, wl.k_floor, scale, buf) if args.graph else None
+
     def step():
-        fv.attention_layer(g, q, k, v, wl.p, wl.k_floor, scale, buf, stream)
+        if lg is not None:
+            lg.replay()
+        else:
+            fv.attention_layer(g, q, k, v, wl.p, wl.k_floor, scale, buf, stream)
 
     # warm-up (also the mask used for the FLOP count)
     for _ in range(max(args.warmup, 3)):
@@ -163,7 +173,7 @@ def run_ours(args, rank, world, local_rank):
     eff = MX.effective_flops(keep, real, wl.d)
     kept_frac = float(keep.mean())
 
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
     if world > 1:
         torch.distributed.barrier()
@@ -172,24 +182,16 @@ def run_ours(args, rank, world, local_rank):
         sampler.start()
         time.sleep(0.3)
     for i in range(args.steps):
-        e = ev[i]
-        e[0].record(stream)
-        fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream)
-        e[1].record(stream)
-        fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts, stream)
-        e[2].record(stream)
-        fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse, buf.workspace,
-                                    buf.sm_busy_ns, stream)
-        e[3].record(stream)
+        ev[i][0].record(stream)
+        step()
+        ev[i][1].record(stream)
         flush.fill_(float(i))
     torch.cuda.synchronize(dev)
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
-    t_pool = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    t_route = [ev[i][1].elapsed_time(ev[i][2]) for i in range(args.steps)]
-    t_attn = [ev[i][2].elapsed_time(ev[i][3]) for i in range(args.steps)]
-    total_ms = sum(t_pool) + sum(t_route) + sum(t_attn)
+    t_layer = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
+    total_ms = sum(t_layer)
     if world > 1:
         t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
         torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
@@ -199,28 +201,75 @@ def run_ours(args, rank, world, local_rank):
     if fv.fvattn_device_status(buf.workspace, stream) != 0:
         raise RuntimeError("attention kernel reported a timeout")
 
+    def graph_of(fn):
+        side = torch.cuda.Stream(dev)
+        side.wait_stream(stream)
+        with torch.cuda.stream(side):
+            fn()
+        stream.wait_stream(side)
+        gr = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(gr):
+            fn()
+        return gr
+
+    def per_call(gr, reps):
+        """Device time of one replay in its place in the layer (median): L2 flushed, then
+        pool and route (untimed; they also absorb the write-back of the flush's dirty
+        lines), then the timed replay."""
+        ts = []
+        for i in range(3 + reps):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            flush.fill_(float(i))
+            fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream)
+            fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts, stream)
+            a.record(stream)
+            gr.replay()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 3:
+                ts.append(a.elapsed_time(b))
+        return statistics.median(ts)
+
+    def back_to_back(fn, reps=20):
+        """Device time per launch of `reps` launches in a row (no host gaps)."""
+        for _ in range(3):
+            fn()
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        flush.fill_(0.5)
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b) / reps
+
+    # Per-stage device times (not added to the layer time above).  Pool streams 201 MB
+    # (more than L2); route reads the pooled rows pool has just written.
+    t_pool = back_to_back(lambda: fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream))
+    t_route = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
+                                                   buf.mask, buf.counts, stream))
+    # (inside a capture the calls must use the capturing stream: stream=None = current)
+    attn_graph = graph_of(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
+                                                              buf.workspace, buf.sm_busy_ns))
+    attn_ms = per_call(attn_graph, min(max(args.steps, 5), 20))
+
     if args.layer_only:
         ms_step = total_ms / args.steps
         return {"metric": METRIC, "value": round(eff * world / (ms_step * 1e-3) / 1e12, 3), "unit": UNIT,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
-                "ms_per_step": round(ms_step, 4), "attn_ms": round(statistics.mean(t_attn), 4),
+                "ms_per_step": round(ms_step, 4), "attn_ms": round(attn_ms, 4),
                 "layer_only": True}
 
     # dense baseline (p = 1 through the same kernel), same protocol
-    dense_t = []
-    for i in range(max(args.warmup, 3) + min(args.steps, 10)):
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
-        fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace, None, stream)
-        b.record(stream)
-        flush.fill_(float(i))
-        torch.cuda.synchronize(dev)
-        if i >= max(args.warmup, 3):
-            dense_t.append(a.elapsed_time(b))
-    dense_ms = statistics.median(dense_t)
+    dense_graph = graph_of(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace,
+                                                        None))
+    dense_ms = per_call(dense_graph, min(args.steps, 10))
 
-    # end to end through the public API with host buffers (pinned), copies timed
+    # end to end through the public API with host buffers (pinned), copies timed: each
+    # step copies Q/K/V into the captured input buffers, replays the layer, reads
+    # out and lse back
     pinned = {n: host[n].pin_memory() for n in ("q", "k", "v")}
     out_h = torch.empty(buf.out.shape, dtype=torch.bfloat16).pin_memory()
     lse_h = torch.empty(buf.lse.shape, dtype=torch.float32).pin_memory()
@@ -230,8 +279,10 @@ def run_ours(args, rank, world, local_rank):
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         a.record(stream)
-        qd, kd, vd = (pinned[n].to(dev, non_blocking=True) for n in ("q", "k", "v"))
-        fv.attention_layer(g, qd, kd, vd, wl.p, wl.k_floor, scale, buf, stream)
+        q.copy_(pinned["q"], non_blocking=True)
+        k.copy_(pinned["k"], non_blocking=True)
+        v.copy_(pinned["v"], non_blocking=True)
+        step()
         out_h.copy_(buf.out, non_blocking=True)
         lse_h.copy_(buf.lse, non_blocking=True)
         b.record(stream)
@@ -243,11 +294,10 @@ def run_ours(args, rank, world, local_rank):
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
     ms_step = total_ms / args.steps
-    attn_ms = statistics.mean(t_attn)
     value = eff * world / (ms_step * 1e-3) / 1e12
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
     pr_bytes = MX.pool_route_bytes(wl.B, wl.H, wl.N, g.nB, wl.d, g.words)
-    pr_ms = statistics.mean(t_pool) + statistics.mean(t_route)
+    pr_ms = t_pool + t_route
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -257,7 +307,10 @@ def run_ours(args, rank, world, local_rank):
         "attn_ms": round(attn_ms, 4),
         "attn_effective_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
-        "pool_ms": round(statistics.mean(t_pool), 4), "route_ms": round(statistics.mean(t_route), 4),
+        "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
+        "stage_timing": "pool, route: device time per launch over 20 back-to-back launches; attention: "
+                        "one captured call after L2 flush + pool + route (median)",
+        "layer_step": "CUDA graph of pool -> route -> attention (LayerGraph)" if args.graph else "direct calls",
         "pool_route_gbs": round(pr_bytes / (pr_ms * 1e-3) / 1e9, 1),
         "pool_route_frac_of_hbm": round(pr_bytes / (pr_ms * 1e-3) / 1e9 / peaks["hbm"], 4),
         "dense_attn_ms": round(dense_ms, 4),
@@ -271,6 +324,7 @@ def run_ours(args, rank, world, local_rank):
                      "frac": round(attn_tflops / peaks["bf16"], 4), "traffic": attn_traffic(),
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
         "e2e": {"value": round(eff * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+                "how": "pinned host Q/K/V -> device, layer step, out/lse -> pinned host, one stream",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 5 * args.steps,   # pool, route, prep_cost, prep_order, attention
         "clocks": clocks,
@@ -400,6 +454,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", action="store_true", help="also time the 15 p/k points (config 5)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-graph", dest="graph", action="store_false",
+                    help="time the layer as three direct calls instead of a captured CUDA graph")
     ap.add_argument("--layer-only", action="store_true",
                     help="time the layer steps only (no dense, e2e or CPU legs); for profilers")
     args = ap.parse_args()

@@ -11,7 +11,8 @@ Entry points mirror the C ABI in ``include/fvattn.h``:
 * ``fvattn_block_sparse_attn``  attention over the kept key blocks -> out, lse
 * ``fvattn_dense_attn``   the same kernel with every key block kept
 
-and ``attention_layer`` strings the three steps together for one layer.
+and ``attention_layer`` strings the three steps together for one layer; ``LayerGraph``
+captures that layer once in a CUDA graph and replays it.
 """
 from __future__ import annotations
 
@@ -25,7 +26,7 @@ __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
-    "LayerBuffers",
+    "LayerBuffers", "LayerGraph",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -273,3 +274,38 @@ def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optiona
     fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
     fvattn_block_sparse_attn(g, q, k, v, b.mask, scale, b.out, b.lse, b.workspace, b.sm_busy_ns, stream)
     return b
+
+
+class LayerGraph:
+    """One attention layer (pool -> route -> block-sparse attention) captured once in a
+    CUDA graph and replayed.
+
+    A replay launches the layer's kernels (pool, route, the two schedule-prep kernels and
+    attention) with no host work in between: argument checks, tensor-map encoding and the
+    launch configuration happen once, at capture.  Everything the calls were given is
+    fixed in the graph: q, k, v and the buffers must stay allocated, at the same
+    addresses, with the same shapes; to run on new inputs, copy them into ``q``, ``k``,
+    ``v`` (for instance from pinned host memory on the same stream) before ``replay``.
+    p, k_floor and scale are fixed as well."""
+
+    def __init__(self, g: Geometry, q, k, v, p: float, k_floor: int, scale: Optional[float] = None,
+                 buffers: Optional[LayerBuffers] = None):
+        import torch
+        self.g, self.q, self.k, self.v = g, q, k, v
+        self.p, self.k_floor = float(p), int(k_floor)
+        self.scale = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+        self.buffers = buffers if buffers is not None else LayerBuffers.allocate(g, q.device)
+        # one uncaptured run on a side stream first (module loading, kernel attributes)
+        side = torch.cuda.Stream(q.device)
+        side.wait_stream(torch.cuda.current_stream(q.device))
+        with torch.cuda.stream(side):
+            attention_layer(g, q, k, v, self.p, self.k_floor, self.scale, self.buffers)
+        torch.cuda.current_stream(q.device).wait_stream(side)
+        self.graph = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(self.graph):
+            attention_layer(g, q, k, v, self.p, self.k_floor, self.scale, self.buffers)
+
+    def replay(self) -> LayerBuffers:
+        """Launches the captured layer on the current stream; returns its buffers."""
+        self.graph.replay()
+        return self.buffers
