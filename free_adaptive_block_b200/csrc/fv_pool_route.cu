@@ -139,6 +139,23 @@ __device__ __forceinline__ float warp_max(float v) {
   return v;
 }
 
+// When exactly one valid key of the row has the high 16 bits of u, sets u to that key
+// and returns true (uniform over the warp).
+template <int MAXW>
+__device__ __forceinline__ bool unique_prefix(const uint32_t* key, uint32_t& u) {
+  int n = 0;
+  uint32_t kmax = 0;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    const bool in = key[c] != 0u && (key[c] >> 16) == (u >> 16);
+    n += in ? 1 : 0;
+    kmax = in ? max(kmax, key[c]) : kmax;
+  }
+  if (warp_sum_i(n) != 1) return false;
+  u = __reduce_max_sync(0xffffffffu, kmax);
+  return true;
+}
+
 // Selection for one query block; the row's logits are in sL[i], i = c*32 + lane.
 template <int MAXW>
 __device__ __forceinline__ void select_row(const float* sL, int nB, int words, int qb, float p,
@@ -180,7 +197,10 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
   if (p >= 1.f || total < p) {
     m_p = nB;
   } else {
-    for (int bit = 31; bit >= 0; --bit) {
+    // The high 16 bits first.  The answer is the key of one logit (the m_p-th in the
+    // order), so when a single logit carries the 16-bit prefix found, its key is the
+    // answer and the low 16 steps are skipped; otherwise they run as usual.
+    auto mass_step = [&](int bit) {
       const uint32_t cand = u | (1u << bit);
       float m0 = 0.f, m1 = 0.f;
 #pragma unroll
@@ -189,6 +209,10 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
         if (c + 1 < MAXW) m1 += key[c + 1] >= cand ? sc[c + 1] : 0.f;
       }
       if (warp_sum(m0 + m1) >= p) u = cand;
+    };
+    for (int bit = 31; bit >= 16; --bit) mass_step(bit);
+    if (!unique_prefix<MAXW>(key, u)) {
+      for (int bit = 15; bit >= 0; --bit) mass_step(bit);
     }
     int gt = 0, eq = 0;
     float gm = 0.f, es = 0.f;
@@ -216,12 +240,16 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
     ties_needed = nB;     // every block (keys of real blocks are nonzero)
   } else if (M > m_p) {
     uint32_t v = 0;
-    for (int bit = 31; bit >= 0; --bit) {
+    auto count_step = [&](int bit) {
       const uint32_t cand = v | (1u << bit);
       int n = 0;
 #pragma unroll
       for (int c = 0; c < MAXW; ++c) n += key[c] >= cand ? 1 : 0;
       if (warp_sum_i(n) >= M) v = cand;
+    };
+    for (int bit = 31; bit >= 16; --bit) count_step(bit);
+    if (!unique_prefix<MAXW>(key, v)) {
+      for (int bit = 15; bit >= 0; --bit) count_step(bit);
     }
     int gt = 0;
 #pragma unroll
@@ -306,7 +334,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
   // 4 (w / 4) .. + 3.  Per (row, key) the sum over d runs in two partial sums (even and
   // odd components of each float4), in ascending d, added at the end.
   const int kgrp = warp & 3, rgrp = warp >> 2;
-  float a0[4], a1[4];
+  uint64_t acc[4];   // (a0, a1) per query row as an f32x2 pair
   for (int st = 0; st < nstage; ++st) {
     if (st + 1 < nstage) {
       stage(st + 1);
@@ -318,24 +346,29 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
     const int round = st / NDC, ct = st - round * NDC;
     if (ct == 0) {
 #pragma unroll
-      for (int r = 0; r < 4; ++r) a0[r] = a1[r] = 0.f;
+      for (int r = 0; r < 4; ++r) acc[r] = 0ull;
     }
     const float4* kr = reinterpret_cast<const float4*>(sK + (st & 1) * kRouteKT * kRouteKSP + (32 * kgrp + lane) * kRouteKSP);
 #pragma unroll
     for (int u = 0; u < kRouteDC / 4; ++u) {
       const float4 k4 = kr[u];
+      const uint64_t kxy = f32x2(k4.x, k4.y), kzw = f32x2(k4.z, k4.w);
 #pragma unroll
       for (int r = 0; r < 4; ++r) {
         const float4 x = reinterpret_cast<const float4*>(sQ + (4 * rgrp + r) * D)[ct * (kRouteDC / 4) + u];
-        a0[r] = fmaf(x.x, k4.x, a0[r]); a1[r] = fmaf(x.y, k4.y, a1[r]);
-        a0[r] = fmaf(x.z, k4.z, a0[r]); a1[r] = fmaf(x.w, k4.w, a1[r]);
+        acc[r] = ffma2(f32x2(x.x, x.y), kxy, acc[r]);   // a0 += x.x k.x, a1 += x.y k.y
+        acc[r] = ffma2(f32x2(x.z, x.w), kzw, acc[r]);   // a0 += x.z k.z, a1 += x.w k.w
       }
     }
     if (ct == NDC - 1) {
       const int key = round * kRouteKT + 32 * kgrp + lane;
       if (key < nB) {
 #pragma unroll
-        for (int r = 0; r < 4; ++r) sL[(4 * rgrp + r) * nBpad + key] = (a0[r] + a1[r]) * scale;
+        for (int r = 0; r < 4; ++r) {
+          float a0, a1;
+          unpack_f32x2(acc[r], a0, a1);
+          sL[(4 * rgrp + r) * nBpad + key] = (a0 + a1) * scale;
+        }
       }
     }
     __syncthreads();   // this buffer is restaged by the next iteration's prefetch
