@@ -132,13 +132,13 @@ class ClockSampler:
 
 
 # ----------------------------------------------------------------------------- GPU arm
-def run_ours(args, rank, world, local_rank):
+def run_ours(args, rank, world, local_rank, wl=None):
     import torch
     import free_adaptive_block_b200 as fv
 
     torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    wl = W.WAN21_480P
+    wl = wl or W.WAN21_480P
     g = fv.Geometry(**wl.geom())
     scale = float(np.float32(1.0 / math.sqrt(wl.d)))
     peaks = load_peaks()
@@ -454,6 +454,8 @@ def main():
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", action="store_true", help="also time the 15 p/k points (config 5)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--all-configs", action="store_true",
+                    help="after the 480p line, one line per other workload (tiny, 720p, 6x horizon)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the layer as three direct calls instead of a captured CUDA graph")
     ap.add_argument("--layer-only", action="store_true",
@@ -480,6 +482,11 @@ def main():
             if world == 1 and not (args.no_cpu_baseline or args.layer_only):
                 line["cpu_baseline"] = cpu_baseline(W.WAN21_480P, W.generate(W.WAN21_480P))
             print(json.dumps(line), flush=True)
+        if args.all_configs and rank == 0:
+            for wl in (W.TINY, W.WAN22_720P, W.WAN21_6X):
+                extra = run_ours(args, 0, 1, local_rank, wl)
+                extra["metric"] = f"same measurements on the {wl.name} workload (not the headline)"
+                print(json.dumps(extra), flush=True)
         if args.sweep and rank == 0:
             run_sweep(args, local_rank)
     finally:
