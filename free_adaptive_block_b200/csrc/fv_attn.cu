@@ -5,7 +5,8 @@
 // the selected KV blocks.  Here it is one persistent kernel per call:
 //
 //   * a (b, h, query block) "tile" is one query block of up to 128 tokens against
-//     its kept key blocks, visited in ascending block order with an online softmax;
+//     its kept key blocks with an online softmax: the wide blocks in ascending order,
+//     then the narrow W-edge blocks packed up to 128 / rows_e per 128-row K/V slot;
 //   * tiles come from an atomic queue ordered by decreasing cost (longest processing
 //     time first); the order is built by prep_kernel from the mask;
 //   * warp 0 loads Q / K / V boxes with TMA (5D tensor maps over
@@ -86,6 +87,8 @@ struct AttnParams {
   const int* order;
   int ntiles;
   unsigned long long* busy;
+  int pack;               // narrow (W-edge) key blocks packed per 128-row K/V slot (1: none)
+  int rows_e;             // box rows of a W-edge block (bt * bh * (Ws mod bw))
 };
 
 struct __align__(8) AttnBars {
@@ -104,8 +107,11 @@ struct __align__(8) AttnBars {
   uint64_t t_full[kTR], t_empty[kTR];
   uint64_t fin[2];        // drain after an abort: S issuer, P.V issuer
   int tile[kTR];
-  int bcount[kTR];        // kept blocks of the tile
-  uint32_t blist[kTR][kMaxBlocks];  // the tile's kept blocks in ascending order (pack_blk)
+  int bcount[kTR];        // kept wide blocks of the tile
+  int ncount[kTR];        // kept narrow (packed) blocks of the tile
+  uint32_t blist[kTR][kMaxBlocks];  // the tile's kept blocks (pack_blk): wide ones in
+                                    // ascending order, then narrow ones in ascending order
+  uint32_t edgew[kMaxBlocks / 32];  // per mask word: bits of the blocks that are packed
   uint32_t tmem_base;
   int abort;
   float hv[2][128];       // [group][row] reference after the group's latest block, guarded by hb
@@ -141,6 +147,29 @@ __device__ __forceinline__ int blk_npad(uint32_t e) { return static_cast<int>((e
 __device__ __forceinline__ int blk_nvalid(uint32_t e) { return static_cast<int>((e >> 16) & 0xFFu); }
 __device__ __forceinline__ bool blk_prefix(uint32_t e) { return (e >> 24) & 1u; }
 __device__ __forceinline__ bool blk_needmask(uint32_t e) { return (e >> 25) & 1u; }
+
+// The work items of a tile: each kept wide block on its own, then the narrow blocks
+// (W-edge blocks whose box has rows_e = 16, 32 or 64 rows) in groups of up to
+// pack = 128 / rows_e that share one 128-row K/V slot, one S and one P.V product.
+// Sub-block s of a group occupies rows [s * rows_e, (s + 1) * rows_e) of the slot.
+struct ItemRange {
+  int first, cnt;
+};
+__device__ __forceinline__ int num_items(int nw, int nn, int pack) { return nw + (nn + pack - 1) / pack; }
+__device__ __forceinline__ ItemRange item_range(int i, int nw, int nn, int pack) {
+  if (i < nw) return ItemRange{i, 1};
+  const int k = i - nw;
+  return ItemRange{nw + k * pack, min(pack, nn - k * pack)};
+}
+__device__ __forceinline__ int item_npad(const uint32_t* bl, int i, int nw, const ItemRange& r, int rows_e) {
+  return i < nw ? blk_npad(bl[i]) : r.cnt * rows_e;
+}
+__device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
+  const int a = min(max(lo - base, 0), 32), b = min(max(hi - base, 0), 32);
+  const uint32_t hib = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
+  const uint32_t lob = a >= 32 ? 0xffffffffu : ((1u << a) - 1u);
+  return hib & ~lob;
+}
 
 __device__ __forceinline__ void decode_tile(const Geo& g, int tile, int& bhi, int& qb) {
   bhi = tile / g.nB;
@@ -199,6 +228,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     bars.abort = 0;
     fence_barrier_init();
   }
+  // Which blocks are packed narrow blocks: the last block column, when packing is on.
+  for (int w = threadIdx.x; w < kMaxBlocks / 32; w += kAttnThreads) {
+    uint32_t bits = 0;
+    if (prm.pack > 1 && w < g.words) {
+      for (int i = 0; i < 32; ++i) {
+        const int j = w * 32 + i;
+        if (j < g.nB && (j % g.nBx) == g.nBx - 1) bits |= 1u << i;
+      }
+    }
+    bars.edgew[w] = bits;
+  }
   // Rows past a box are read by the MMAs (multiplied by zero P or masked): start
   // from zeros so they are finite.
   {
@@ -245,33 +285,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int tile = pos < prm.ntiles ? __ldg(prm.order + pos) : -1;
       const int slot = tcount % kTR;
       if (!wwait(&bars.t_empty[slot], ((tcount / kTR) & 1) ^ 1)) break;
-      int nkv = 0;
+      int nw = 0, nn = 0;
       if (tile >= 0) {
         uint32_t* bl = bars.blist[slot];
+        uint32_t w0, w1;
         if (prm.mask != nullptr) {
           const uint32_t* src = prm.mask + static_cast<size_t>(tile) * g.words;
-          const uint32_t w0 = lane < g.words ? __ldg(src + lane) : 0u;
-          const uint32_t w1 = lane + 32 < g.words ? __ldg(src + lane + 32) : 0u;
-          int i0 = __popc(w0), i1 = __popc(w1);
-#pragma unroll
-          for (int o = 1; o < 32; o <<= 1) {
-            const int a0 = __shfl_up_sync(0xffffffffu, i0, o), a1 = __shfl_up_sync(0xffffffffu, i1, o);
-            if (lane >= o) { i0 += a0; i1 += a1; }
-          }
-          const int tot0 = __shfl_sync(0xffffffffu, i0, 31);
-          int p0 = i0 - __popc(w0), p1 = tot0 + i1 - __popc(w1);
-          for (uint32_t bits = w0; bits; bits &= bits - 1) bl[p0++] = pack_blk(g, lane * 32 + __ffs(bits) - 1);
-          for (uint32_t bits = w1; bits; bits &= bits - 1) bl[p1++] = pack_blk(g, (lane + 32) * 32 + __ffs(bits) - 1);
-          nkv = tot0 + __shfl_sync(0xffffffffu, i1, 31);
+          w0 = lane < g.words ? __ldg(src + lane) : 0u;
+          w1 = lane + 32 < g.words ? __ldg(src + lane + 32) : 0u;
         } else {
-          for (int i = lane; i < g.nB; i += 32) bl[i] = pack_blk(g, i);
-          nkv = g.nB;
+          const int tail = g.nB & 31;
+          auto full_word = [&](int w) -> uint32_t {
+            return w < g.words - 1 ? 0xffffffffu : (w == g.words - 1 ? (tail ? (1u << tail) - 1u : 0xffffffffu) : 0u);
+          };
+          w0 = full_word(lane);
+          w1 = full_word(lane + 32);
+        }
+        const uint32_t n0 = w0 & bars.edgew[lane], n1 = w1 & bars.edgew[lane + 32];
+        const uint32_t d0 = w0 & ~n0, d1 = w1 & ~n1;
+        int i0 = __popc(d0), i1 = __popc(d1), j0 = __popc(n0), j1 = __popc(n1);
+#pragma unroll
+        for (int o = 1; o < 32; o <<= 1) {
+          const int a0 = __shfl_up_sync(0xffffffffu, i0, o), a1 = __shfl_up_sync(0xffffffffu, i1, o);
+          const int b0 = __shfl_up_sync(0xffffffffu, j0, o), b1 = __shfl_up_sync(0xffffffffu, j1, o);
+          if (lane >= o) { i0 += a0; i1 += a1; j0 += b0; j1 += b1; }
+        }
+        const int tw0 = __shfl_sync(0xffffffffu, i0, 31), tn0 = __shfl_sync(0xffffffffu, j0, 31);
+        nw = tw0 + __shfl_sync(0xffffffffu, i1, 31);
+        nn = tn0 + __shfl_sync(0xffffffffu, j1, 31);
+        int p0 = i0 - __popc(d0), p1 = tw0 + i1 - __popc(d1);
+        int q0 = nw + j0 - __popc(n0), q1 = nw + tn0 + j1 - __popc(n1);
+        // one placement loop over the four (word, kind) sets keeps a single copy of pack_blk
+#pragma unroll 1
+        for (int set = 0; set < 4; ++set) {
+          uint32_t bits = set == 0 ? d0 : (set == 1 ? d1 : (set == 2 ? n0 : n1));
+          const int wbase = ((set & 1) ? lane + 32 : lane) * 32;
+          int pos = set == 0 ? p0 : (set == 1 ? p1 : (set == 2 ? q0 : q1));
+          for (; bits; bits &= bits - 1) bl[pos++] = pack_blk(g, wbase + __ffs(bits) - 1);
         }
       }
       __syncwarp();
       if (lane == 0) {
         bars.tile[slot] = tile;
-        bars.bcount[slot] = nkv;
+        bars.bcount[slot] = nw;
+        bars.ncount[slot] = nn;
         mbar_arrive(&bars.t_full[slot]);
       }
       __syncwarp();
@@ -290,17 +347,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       ++qc;
       const int full_rows = g.bt * g.bh * g.bw;
-      for (int n = 0; n < nkv; ++n) {
-        const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][n]));
-        const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
-        const bool xedge = ki.rows != full_rows;
+      const int nitems = num_items(nw, nn, prm.pack);
+      for (int n = 0; n < nitems; ++n) {
+        const ItemRange ir = item_range(n, nw, nn, prm.pack);
         const int ks = kc % kNK;
         if (!wwait(&bars.k_empty[ks], ((kc / kNK) & 1) ^ 1)) { ok = false; break; }
         if (elect_one()) {
-          mbar_arrive_expect_tx(&bars.k_full[ks], bytes);
-          for (int c = 0; c < NCH; ++c)
-            tma_load_5d(sK(ks) + c * kChunkBytes, xedge ? &tmKe : &tmK, &bars.k_full[ks],
-                        c * 64, ki.x0, ki.y0, ki.t0, bhi);
+          // every box of an item has the same rows (a wide block, or narrow blocks)
+          const uint32_t rows0 = blk_of(g, blk_id(bars.blist[slot][ir.first])).rows;
+          mbar_arrive_expect_tx(&bars.k_full[ks], rows0 * 128 * NCH * ir.cnt);
+#pragma unroll 1
+          for (int sb = 0; sb < ir.cnt; ++sb) {
+            const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][ir.first + sb]));
+            const bool xedge = ki.rows != full_rows;
+            const uint32_t off = static_cast<uint32_t>(sb * prm.rows_e * 128);
+#pragma unroll 1
+            for (int c = 0; c < NCH; ++c)
+              tma_load_5d(sK(ks) + c * kChunkBytes + off, xedge ? &tmKe : &tmK, &bars.k_full[ks],
+                          c * 64, ki.x0, ki.y0, ki.t0, bhi);
+          }
         }
         __syncwarp();
         ++kc;
@@ -314,23 +379,31 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int slot = tcount % kTR;
       if (!wwait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
       const int tile = bars.tile[slot];
-      const int nkv = bars.bcount[slot];
+      const int nw = bars.bcount[slot], nn = bars.ncount[slot];
       ++tcount;
       if (tile < 0) break;
       int bhi, qb;
       decode_tile(g, tile, bhi, qb);
       const int full_rows = g.bt * g.bh * g.bw;
-      for (int n = 0; n < nkv; ++n) {
-        const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][n]));
-        const uint32_t bytes = static_cast<uint32_t>(ki.rows * 128 * NCH);
-        const bool xedge = ki.rows != full_rows;
+      const int nitems = num_items(nw, nn, prm.pack);
+      for (int n = 0; n < nitems; ++n) {
+        const ItemRange ir = item_range(n, nw, nn, prm.pack);
         const int vs = vc % kNV;
         if (!wwait(&bars.v_empty[vs], ((vc / kNV) & 1) ^ 1)) { ok = false; break; }
         if (elect_one()) {
-          mbar_arrive_expect_tx(&bars.v_full[vs], bytes);
-          for (int c = 0; c < NCH; ++c)
-            tma_load_5d(sV(vs) + c * kChunkBytes, xedge ? &tmVe : &tmV, &bars.v_full[vs],
-                        c * 64, ki.x0, ki.y0, ki.t0, bhi);
+          // every box of an item has the same rows (a wide block, or narrow blocks)
+          const uint32_t rows0 = blk_of(g, blk_id(bars.blist[slot][ir.first])).rows;
+          mbar_arrive_expect_tx(&bars.v_full[vs], rows0 * 128 * NCH * ir.cnt);
+#pragma unroll 1
+          for (int sb = 0; sb < ir.cnt; ++sb) {
+            const BlkEnt ki = blk_of(g, blk_id(bars.blist[slot][ir.first + sb]));
+            const bool xedge = ki.rows != full_rows;
+            const uint32_t off = static_cast<uint32_t>(sb * prm.rows_e * 128);
+#pragma unroll 1
+            for (int c = 0; c < NCH; ++c)
+              tma_load_5d(sV(vs) + c * kChunkBytes + off, xedge ? &tmVe : &tmV, &bars.v_full[vs],
+                          c * 64, ki.x0, ki.y0, ki.t0, bhi);
+          }
         }
         __syncwarp();
         ++vc;
@@ -355,15 +428,17 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int tile = bars.tile[slot];
       ++tcount;
       if (tile < 0) break;
-      const int nkv = bars.bcount[slot];
+      const int nw = bars.bcount[slot], nn = bars.ncount[slot];
+      const int nitems = num_items(nw, nn, prm.pack);
       if (!wwait(&bars.q_full, mqc & 1)) break;
       ++mqc;
       int n = 0;
-      for (; n < nkv; ++n) {
+      for (; n < nitems; ++n) {
         const uint32_t c = gc + n;
         const int ss = c % kNS;
         const int ks = c % kNK;
-        const uint32_t idesc_s = idesc_bf16_f32(128, blk_npad(bars.blist[slot][n]), 0, 0);
+        const ItemRange ir = item_range(n, nw, nn, prm.pack);
+        const uint32_t idesc_s = idesc_bf16_f32(128, item_npad(bars.blist[slot], n, nw, ir, prm.rows_e), 0, 0);
         if (!wwait(&bars.k_full[ks], (c / kNK) & 1)) { ok = false; break; }
         if (c >= kNS && !wwait(&bars.s_empty[ss], ((c - kNS) / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
@@ -398,15 +473,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int slot = tcount % kTR;
       if (!wwait(&bars.t_full[slot], (tcount / kTR) & 1)) break;
       const int tile = bars.tile[slot];
-      const int nkv = bars.bcount[slot];
+      const int nw = bars.bcount[slot], nn = bars.ncount[slot];
+      const int nitems = num_items(nw, nn, prm.pack);
       ++tcount;
       if (tile < 0) break;
       int n = 0;
-      for (; n < nkv; ++n) {
+      for (; n < nitems; ++n) {
         const uint32_t c = gc + n;
         const int ps = c % kNP;
         const int vs = c % kNV;
-        const int nk = blk_npad(bars.blist[slot][n]) >> 4;
+        const int nk = item_npad(bars.blist[slot], n, nw, item_range(n, nw, nn, prm.pack), prm.rows_e) >> 4;
         if (!wwait(&bars.p_full[ps], (c / kNP) & 1)) { ok = false; break; }
         if (!wwait(&bars.v_full[vs], (c / kNV) & 1)) { ok = false; break; }
         if (n == 0 && !wwait(&bars.o_empty, (tiles & 1) ^ 1)) { ok = false; break; }
@@ -469,16 +545,25 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int token = box_row_token(g, qi, row);
 
       float m = -INFINITY, l = 0.f;     // this group's latest reference and its row sum
-      const int nkv = bars.bcount[slot];
+      const int nw = bars.bcount[slot], nn = bars.ncount[slot];
+      const int nkv = num_items(nw, nn, prm.pack);
       const uint32_t* bl = bars.blist[slot];
       bool ok = true;
       for (int j = grp; j < nkv; j += 2) {
-        const uint32_t e = bl[j];
+        const ItemRange ir = item_range(j, nw, nn, prm.pack);
+        const uint32_t e = bl[ir.first];
         const uint32_t c = gc + j;
         const int ss = c % kNS;
         const uint32_t tS = tS0 + ss * 128;
         const uint32_t tP = tP0 + (c % kNP) * 64;
-        const int nact = (blk_npad(e) + 31) >> 5;   // 32-column chunks below npad (uniform)
+        const int npad = item_npad(bl, j, nw, ir, prm.rows_e);
+        const int nact = (npad + 31) >> 5;          // 32-column chunks below npad (uniform)
+        bool need_mask = blk_needmask(e);
+        if (j >= nw) {
+          need_mask = (npad & 31) != 0;
+#pragma unroll 1
+          for (int sb = 0; sb < ir.cnt; ++sb) need_mask |= blk_nvalid(bl[ir.first + sb]) < prm.rows_e;
+        }
         if (!sync_wait(&bars.s_full[ss], (c / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
         // The whole row of S in one TMEM round trip (loads are grouped, then one wait).
@@ -492,9 +577,18 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // Keys that are not real tokens (a partial last 16-key group, or the gaps of a box
         // cut at the time and height edges at once) to -inf.  One warp-uniform branch,
         // taken only by such blocks, so the common path carries none of this code.
-        if (blk_needmask(e)) {
+        if (need_mask) {
           uint32_t vm[4];
-          if (blk_prefix(e)) {
+          if (j >= nw) {
+#pragma unroll
+            for (int w4 = 0; w4 < 4; ++w4) vm[w4] = 0u;
+#pragma unroll 1
+            for (int sb = 0; sb < ir.cnt; ++sb) {
+              const int lo = sb * prm.rows_e, hi = lo + blk_nvalid(bl[ir.first + sb]);
+#pragma unroll
+              for (int w4 = 0; w4 < 4; ++w4) vm[w4] |= range_bits(lo, hi, 32 * w4);
+            }
+          } else if (blk_prefix(e)) {
             const int nvalid = blk_nvalid(e);
 #pragma unroll
             for (int w4 = 0; w4 < 4; ++w4) {
@@ -887,10 +981,14 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
   if (mask != nullptr) {
     // cost of each block class, from a block of that class (last column / row / frame)
     ClassCost cc;
+    // a packed W-edge block costs its rows plus a 1/pack share of one item's overhead
+    const int rx_e = g.Ws - (g.nBx - 1) * g.bw, rows_e = g.bt * g.bh * rx_e;
+    const int pack = (rx_e < g.bw && (rows_e == 16 || rows_e == 32 || rows_e == 64) &&
+                      (g.bt == 1 || g.Hs % g.bh == 0)) ? 128 / rows_e : 1;
     for (int k = 0; k < 8; ++k) {
       const int xb = (k & 1) ? g.nBx - 1 : 0, yb = (k & 2) ? g.nBy - 1 : 0, tb = (k & 4) ? g.nBt - 1 : 0;
       const BlockInfo bi = block_info(g, (tb * g.nBy + yb) * g.nBx + xb);
-      cc.c[k] = bi.npad + kBlockOverhead;
+      cc.c[k] = (pack > 1 && (k & 1)) ? rows_e + kBlockOverhead / pack : bi.npad + kBlockOverhead;
       maxcost = cc.c[k] > maxcost ? cc.c[k] : maxcost;
     }
     maxcost *= g.nB;
@@ -912,6 +1010,11 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
   prm.order = order;
   prm.ntiles = ntiles;
   prm.busy = busy;
+  const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
+  prm.rows_e = g.bt * g.bh * rx_edge;
+  const bool narrow_ok = rx_edge < g.bw && (prm.rows_e == 16 || prm.rows_e == 32 || prm.rows_e == 64) &&
+                         (g.bt == 1 || g.Hs % g.bh == 0);
+  prm.pack = narrow_ok ? 128 / prm.rows_e : 1;
   const int grid = ntiles < nsm ? ntiles : nsm;
   return g.d == 128 ? launch_attn_d<128>(g, maps, prm, grid, st)
                     : launch_attn_d<64>(g, maps, prm, grid, st);
