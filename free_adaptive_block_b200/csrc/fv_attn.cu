@@ -89,6 +89,8 @@ struct AttnParams {
   unsigned long long* busy;
   int pack;               // narrow (W-edge) key blocks packed per 128-row K/V slot (1: none)
   int rows_e;             // box rows of a W-edge block (bt * bh * (Ws mod bw))
+  int qg;                 // narrow query blocks grouped per 128-row tile (1: none)
+  int qps;                // lane quarters per grouped query block (rows_e / 32)
 };
 
 struct __align__(8) AttnBars {
@@ -112,6 +114,7 @@ struct __align__(8) AttnBars {
   uint32_t blist[kTR][kMaxBlocks];  // the tile's kept blocks (pack_blk): wide ones in
                                     // ascending order, then narrow ones in ascending order
   uint32_t edgew[kMaxBlocks / 32];  // per mask word: bits of the blocks that are packed
+  uint32_t gmask[kTR][4][kMaxBlocks / 32];  // a query group's member mask rows (tile list slot)
   uint32_t tmem_base;
   int abort;
   float hv[2][128];       // [group][row] reference after the group's latest block, guarded by hb
@@ -169,6 +172,27 @@ __device__ __forceinline__ uint32_t range_bits(int lo, int hi, int base) {
   const uint32_t hib = b >= 32 ? 0xffffffffu : ((1u << b) - 1u);
   const uint32_t lob = a >= 32 ? 0xffffffffu : ((1u << a) - 1u);
   return hib & ~lob;
+}
+
+// Query groups: when qg > 1, the narrow (W-edge) query blocks of a slice are taken qg at
+// a time, in ascending order, as one tile.  Query block s of a group fills rows
+// [s * rows_e, (s + 1) * rows_e) of the 128-row tile (lane quarters s * qps, ...).  The
+// tile's list is the union of the members' kept blocks; each member's own mask row is
+// kept next to the list, and a member's warps skip the items it does not keep.  The
+// tile is named by its first query block; the others are not tiles of their own.
+__host__ __device__ inline bool q_narrow(const Geo& g, int qb) { return (qb % g.nBx) == g.nBx - 1; }
+__host__ __device__ inline int q_group_cnt(const Geo& g, int qb, int qg) {
+  if (qg <= 1 || !q_narrow(g, qb)) return 1;
+  const int r = qb / g.nBx, rows = g.nBt * g.nBy;
+  return min(qg, rows - r);
+}
+__host__ __device__ inline bool q_member_only(const Geo& g, int qb, int qg) {
+  return qg > 1 && q_narrow(g, qb) && ((qb / g.nBx) % qg) != 0;
+}
+__host__ inline int query_group_size(const Geo& g) {
+  const int rx_e = g.Ws - (g.nBx - 1) * g.bw, rows_e = g.bt * g.bh * rx_e;
+  const bool ok = rx_e < g.bw && (rows_e == 32 || rows_e == 64) && (g.bt == 1 || g.Hs % g.bh == 0);
+  return ok ? 128 / rows_e : 1;
 }
 
 __device__ __forceinline__ void decode_tile(const Geo& g, int tile, int& bhi, int& qb) {
@@ -278,28 +302,37 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     // tiles.  V has its own loader (warp 3) so that the K ring never waits on a P.V.
     uint32_t tcount = 0;
     bool ok = true;
+    // work tiles in the order (grouped narrow query blocks count once), from the prep
+    const int nwork = *reinterpret_cast<volatile const int*>(prm.hdr + 2);
     while (ok) {
       int pos = 0;
       if (lane == 0) pos = static_cast<int>(atomicAdd(prm.hdr, 1u));
       pos = __shfl_sync(0xffffffffu, pos, 0);
-      const int tile = pos < prm.ntiles ? __ldg(prm.order + pos) : -1;
+      const int tile = pos < nwork ? __ldg(prm.order + pos) : -1;
       const int slot = tcount % kTR;
       if (!wwait(&bars.t_empty[slot], ((tcount / kTR) & 1) ^ 1)) break;
       int nw = 0, nn = 0;
       if (tile >= 0) {
         uint32_t* bl = bars.blist[slot];
-        uint32_t w0, w1;
-        if (prm.mask != nullptr) {
-          const uint32_t* src = prm.mask + static_cast<size_t>(tile) * g.words;
-          w0 = lane < g.words ? __ldg(src + lane) : 0u;
-          w1 = lane + 32 < g.words ? __ldg(src + lane + 32) : 0u;
-        } else {
-          const int tail = g.nB & 31;
-          auto full_word = [&](int w) -> uint32_t {
-            return w < g.words - 1 ? 0xffffffffu : (w == g.words - 1 ? (tail ? (1u << tail) - 1u : 0xffffffffu) : 0u);
-          };
-          w0 = full_word(lane);
-          w1 = full_word(lane + 32);
+        // the tile's members (1, or a query group): the list is the union of their kept
+        // blocks; the members' own mask rows go to gmask for the softmax warps
+        const int gcnt = q_group_cnt(g, tile - (tile / g.nB) * g.nB, prm.qg);
+        const int tail = g.nB & 31;
+        uint32_t w0 = 0u, w1 = 0u;
+#pragma unroll 1
+        for (int s4 = 0; s4 < 4; ++s4) {
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            const int w = lane + 32 * h;
+            uint32_t m = 0u;
+            if (s4 < gcnt && w < g.words) {
+              m = prm.mask != nullptr
+                      ? __ldg(prm.mask + static_cast<size_t>(tile + s4 * g.nBx) * g.words + w)
+                      : (w < g.words - 1 ? 0xffffffffu : (tail ? (1u << tail) - 1u : 0xffffffffu));
+            }
+            bars.gmask[slot][s4][w] = m;
+            if (h == 0) w0 |= m; else w1 |= m;
+          }
         }
         const uint32_t n0 = w0 & bars.edgew[lane], n1 = w1 & bars.edgew[lane + 32];
         const uint32_t d0 = w0 & ~n0, d1 = w1 & ~n1;
@@ -336,13 +369,20 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (tile < 0) break;
       int bhi, qb;
       decode_tile(g, tile, bhi, qb);
-      const BlockInfo qi = block_info(g, qb);
+      const int gq = prm.qg > 1 && q_narrow(g, qb) ? q_group_cnt(g, qb, prm.qg) : 0;   // 0: not a group
       if (!wwait(&bars.q_empty, (qc & 1) ^ 1)) break;
       if (elect_one()) {
-        mbar_arrive_expect_tx(&bars.q_full, static_cast<uint32_t>(qi.rows * 128 * NCH));
-        for (int c = 0; c < NCH; ++c)
-          tma_load_5d(sQ + c * kChunkBytes, qi.xedge ? &tmQe : &tmQ, &bars.q_full, c * 64,
-                      qi.xb * g.bw, qi.yb * g.bh, qi.tb * g.bt, bhi);
+        const BlockInfo qi0 = block_info(g, qb);
+        mbar_arrive_expect_tx(&bars.q_full, static_cast<uint32_t>(qi0.rows * 128 * NCH * (gq > 0 ? gq : 1)));
+#pragma unroll 1
+        for (int s4 = 0; s4 < (gq > 0 ? gq : 1); ++s4) {
+          const BlockInfo qi = block_info(g, qb + s4 * g.nBx);
+          const uint32_t off = static_cast<uint32_t>(s4 * prm.rows_e * 128);
+#pragma unroll 1
+          for (int c = 0; c < NCH; ++c)
+            tma_load_5d(sQ + c * kChunkBytes + off, qi.xedge ? &tmQe : &tmQ, &bars.q_full, c * 64,
+                        qi.xb * g.bw, qi.yb * g.bh, qi.tb * g.bt, bhi);
+        }
       }
       __syncwarp();
       ++qc;
@@ -541,8 +581,16 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (tile < 0) break;
       int bhi, qb;
       decode_tile(g, tile, bhi, qb);
-      const BlockInfo qi = block_info(g, qb);
-      const int token = box_row_token(g, qi, row);
+      // in a query group this warp's rows belong to member `sub` (none past the group)
+      const bool qgrp = prm.qg > 1 && q_narrow(g, qb);
+      const int sub = qgrp ? quarter / prm.qps : 0;
+      const int gcnt = qgrp ? q_group_cnt(g, qb, prm.qg) : 1;
+      const uint32_t* gm = bars.gmask[slot][qgrp && sub < 4 ? sub : 0];
+      int token = -1;
+      if (sub < gcnt) {
+        const BlockInfo qi = block_info(g, qb + sub * g.nBx);
+        token = box_row_token(g, qi, qgrp ? row - sub * prm.rows_e : row);
+      }
 
       float m = -INFINITY, l = 0.f;     // this group's latest reference and its row sum
       const int nw = bars.bcount[slot], nn = bars.ncount[slot];
@@ -558,33 +606,50 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t tP = tP0 + (c % kNP) * 64;
         const int npad = item_npad(bl, j, nw, ir, prm.rows_e);
         const int nact = (npad + 31) >> 5;          // 32-column chunks below npad (uniform)
+        // member: this warp's query block keeps the item (some sub-block of a packed item)
+        auto kept = [&](uint32_t es) -> bool {
+          const int kb = blk_id(es);
+          return !qgrp || (sub < gcnt && ((gm[kb >> 5] >> (kb & 31)) & 1u));
+        };
         bool need_mask = blk_needmask(e);
+        bool member = kept(e);
         if (j >= nw) {
           need_mask = (npad & 31) != 0;
+          member = false;
 #pragma unroll 1
-          for (int sb = 0; sb < ir.cnt; ++sb) need_mask |= blk_nvalid(bl[ir.first + sb]) < prm.rows_e;
+          for (int sb = 0; sb < ir.cnt; ++sb) {
+            const uint32_t es = bl[ir.first + sb];
+            const bool k = kept(es);
+            need_mask |= blk_nvalid(es) < prm.rows_e || !k;
+            member |= k;
+          }
         }
         if (!sync_wait(&bars.s_full[ss], (c / kNS) & 1)) { ok = false; break; }
         tc_fence_after();
-        // The whole row of S in one TMEM round trip (loads are grouped, then one wait).
+        // The whole row of S in one TMEM round trip (loads are grouped, then one wait).  A
+        // warp whose query block does not keep the item takes no part in it: P = 0 for its
+        // rows, and its reference carries over unchanged.
         float s[128];
+        if (member) {
 #pragma unroll
-        for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, reinterpret_cast<uint32_t*>(s + 32 * q));
-        tmem_wait_ld();
+          for (int q = 0; q < 4; ++q) tmem_ld32(tS + 32 * q, reinterpret_cast<uint32_t*>(s + 32 * q));
+          tmem_wait_ld();
+        }
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(&bars.s_empty[ss]);    // the slot may take S_c+2
         // Keys that are not real tokens (a partial last 16-key group, or the gaps of a box
         // cut at the time and height edges at once) to -inf.  One warp-uniform branch,
         // taken only by such blocks, so the common path carries none of this code.
-        if (need_mask) {
+        if (member && need_mask) {
           uint32_t vm[4];
           if (j >= nw) {
 #pragma unroll
             for (int w4 = 0; w4 < 4; ++w4) vm[w4] = 0u;
 #pragma unroll 1
             for (int sb = 0; sb < ir.cnt; ++sb) {
-              const int lo = sb * prm.rows_e, hi = lo + blk_nvalid(bl[ir.first + sb]);
+              const uint32_t es = bl[ir.first + sb];
+              const int lo = sb * prm.rows_e, hi = lo + (kept(es) ? blk_nvalid(es) : 0);
 #pragma unroll
               for (int w4 = 0; w4 < 4; ++w4) vm[w4] |= range_bits(lo, hi, 32 * w4);
             }
@@ -611,19 +676,22 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           }
         }
         // Row maximum of each chunk as a shallow tree (depth 4 instead of a 16-long chain).
-        float mq[4];
+        float mx = -INFINITY;
+        if (member) {
+          float mq[4];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) {
-          const float* x = s + 32 * r;
-          float t[11];
+          for (int r = 0; r < 4; ++r) {
+            const float* x = s + 32 * r;
+            float t[11];
 #pragma unroll
-          for (int k = 0; k < 10; ++k) t[k] = max3f(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
-          t[10] = fmaxf(x[30], x[31]);
-          const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
-          const float u2 = max3f(t[6], t[7], t[8]), u3 = max3f(t[9], t[10], u0);
-          mq[r] = r < nact ? max3f(u1, u2, u3) : -INFINITY;
+            for (int k = 0; k < 10; ++k) t[k] = max3f(x[3 * k], x[3 * k + 1], x[3 * k + 2]);
+            t[10] = fmaxf(x[30], x[31]);
+            const float u0 = max3f(t[0], t[1], t[2]), u1 = max3f(t[3], t[4], t[5]);
+            const float u2 = max3f(t[6], t[7], t[8]), u3 = max3f(t[9], t[10], u0);
+            mq[r] = r < nact ? max3f(u1, u2, u3) : -INFINITY;
+          }
+          mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
         }
-        const float mx = fmaxf(fmaxf(mq[0], mq[1]), fmaxf(mq[2], mq[3])) * sl2;
         // reference after block j-1, from the other group
         float mref = mx, mp = mx;
         bool rebase = false;
@@ -673,9 +741,14 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // computed nor stored: the P.V reads keys < npad only.
         const uint64_t nmx2 = f32x2(-m, -m);
         uint64_t acc[4] = {0ull, 0ull, 0ull, 0ull};
+        if (!member) {
+          const uint32_t zero8[8] = {0u, 0u, 0u, 0u, 0u, 0u, 0u, 0u};
+#pragma unroll 1
+          for (int h = 0; h < 2 * nact; ++h) tmem_st8(tP + 8 * h, zero8);
+        }
 #pragma unroll
         for (int c32 = 0; c32 < 4; ++c32) {
-          if (c32 < nact) {
+          if (member && c32 < nact) {
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               uint32_t pk[8];
@@ -816,7 +889,8 @@ struct ClassCost {
 };
 
 __global__ void __launch_bounds__(32 * kCostWarps) prep_cost_kernel(Geo g, const uint32_t* __restrict__ mask,
-                                                                    int* cost_out, int ntiles, ClassCost cc) {
+                                                                    int* cost_out, int ntiles, ClassCost cc,
+                                                                    int qg) {
   __shared__ uint32_t edge[3][kMaxBlocks / 32];   // per word: last column / row / frame bits
   for (int w = threadIdx.x; w < g.words; w += 32 * kCostWarps) {
     uint32_t ex = 0, ey = 0, et = 0;
@@ -837,10 +911,19 @@ __global__ void __launch_bounds__(32 * kCostWarps) prep_cost_kernel(Geo g, const
   const int lane = threadIdx.x & 31;
   const int warp = blockIdx.x * kCostWarps + (threadIdx.x >> 5);
   for (int tile = warp; tile < ntiles; tile += gridDim.x * kCostWarps) {
+    // a query group is one tile (its first member), costed by the union of its masks;
+    // the other members get cost -1 and are left out of the order
+    const int qb = tile - (tile / g.nB) * g.nB;
+    if (q_member_only(g, qb, qg)) {
+      if (lane == 0) cost_out[tile] = -1;
+      continue;
+    }
+    const int gcnt = q_group_cnt(g, qb, qg);
     const uint32_t* row = mask + static_cast<size_t>(tile) * g.words;
     int cost = 0;
     for (int w = lane; w < g.words; w += 32) {
-      const uint32_t m = __ldg(row + w);
+      uint32_t m = 0u;
+      for (int s4 = 0; s4 < gcnt; ++s4) m |= __ldg(row + static_cast<size_t>(s4) * g.nBx * g.words + w);
       const uint32_t ex = edge[0][w], ey = edge[1][w], et = edge[2][w];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {
@@ -857,16 +940,29 @@ __global__ void __launch_bounds__(32 * kCostWarps) prep_cost_kernel(Geo g, const
 __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const uint32_t* __restrict__ mask,
                                                                   uint32_t* hdr, int* order, int* keys,
                                                                   int ntiles, int maxcost,
-                                                                  unsigned long long* busy, int nsm) {
+                                                                  unsigned long long* busy, int nsm, int qg) {
   __shared__ int hist[kHistCells];
   __shared__ unsigned long long total[kMaxSlices];
   __shared__ int rank[kMaxSlices];
+  __shared__ int nwork;
   const int t = threadIdx.x;
-  if (t == 0) { hdr[0] = 0; hdr[1] = 0; }
+  if (t == 0) { hdr[0] = 0; hdr[1] = 0; nwork = 0; }
   if (busy)
     for (int i = t; i < nsm; i += kPrepThreads) busy[i] = 0ull;
+  __syncthreads();
   if (mask == nullptr) {
-    for (int i = t; i < ntiles; i += kPrepThreads) order[i] = i;
+    // every tile but the non-first members of query groups, in any order
+    for (int i0 = 0; i0 < ntiles; i0 += kPrepThreads) {
+      const int i = i0 + t;
+      const bool v = i < ntiles && !q_member_only(g, i - (i / g.nB) * g.nB, qg);
+      const uint32_t bal = __ballot_sync(0xffffffffu, v);
+      int base = 0;
+      if ((t & 31) == 0 && bal) base = atomicAdd(&nwork, __popc(bal));
+      base = __shfl_sync(0xffffffffu, base, 0);
+      if (v) order[base + __popc(bal & ((1u << (t & 31)) - 1u))] = i;
+    }
+    __syncthreads();
+    if (t == 0) hdr[2] = static_cast<uint32_t>(nwork);
     return;
   }
   const int slices = g.B * g.H;
@@ -885,11 +981,13 @@ __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const u
   const int iters = (ntiles + kPrepThreads - 1) / kPrepThreads;
   for (int it = 0; it < iters; ++it) {
     const int i = it * kPrepThreads + t;
-    const bool valid = i < ntiles;
-    const long long cost = valid ? keys[i] : 0;
+    const long long cost0 = i < ntiles ? keys[i] : -1;
+    const bool valid = cost0 >= 0;                     // -1: a non-first query-group member
+    const long long cost = valid ? cost0 : 0;
+    if (valid) atomicAdd(&nwork, 1);
     int key = static_cast<int>(((maxcost - cost) * nbk) / (static_cast<long long>(maxcost) + 1));
     key = min(max(key, 0), nbk - 1);
-    if (valid) keys[i] = key;
+    if (i < ntiles) keys[i] = valid ? key : -1;
     const int grp = valid ? (grouped ? i / g.nB : 0) : -1;
     // one warp reduction and one atomic per distinct slice among the warp's tiles
     uint32_t remaining = __ballot_sync(0xffffffffu, valid);
@@ -917,7 +1015,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const u
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
     const int i = it * kPrepThreads + t;
-    const int cell = i < ntiles ? rank[grouped ? i / g.nB : 0] * nbk + keys[i] : -1;
+    const int key = i < ntiles ? keys[i] : -1;
+    const int cell = key >= 0 ? rank[grouped ? i / g.nB : 0] * nbk + key : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, cell);
     if (cell >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[cell], __popc(peers));
   }
@@ -950,7 +1049,8 @@ __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const u
   __syncthreads();
   for (int it = 0; it < iters; ++it) {
     const int i = it * kPrepThreads + t;
-    const int cell = i < ntiles ? rank[grouped ? i / g.nB : 0] * nbk + keys[i] : -1;
+    const int key = i < ntiles ? keys[i] : -1;
+    const int cell = key >= 0 ? rank[grouped ? i / g.nB : 0] * nbk + key : -1;
     const uint32_t peers = __match_any_sync(0xffffffffu, cell);
     const int leader = __ffs(peers) - 1;
     int base = 0;
@@ -958,6 +1058,7 @@ __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const u
     base = __shfl_sync(peers, base, leader);
     if (cell >= 0) order[base + __popc(peers & ((1u << lane) - 1u))] = i;
   }
+  if (t == 0) hdr[2] = static_cast<uint32_t>(nwork);
 }
 
 template <int D>
@@ -993,11 +1094,12 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
     }
     maxcost *= g.nB;
     const int ctas = (ntiles + kCostWarps - 1) / kCostWarps;
-    prep_cost_kernel<<<ctas, 32 * kCostWarps, 0, st>>>(g, mask, keys, ntiles, cc);
+    prep_cost_kernel<<<ctas, 32 * kCostWarps, 0, st>>>(g, mask, keys, ntiles, cc, query_group_size(g));
     cudaError_t e0 = cudaGetLastError();
     if (e0 != cudaSuccess) return e0;
   }
-  prep_order_kernel<<<1, kPrepThreads, 0, st>>>(g, mask, hdr, order, keys, ntiles, maxcost, busy, nsm);
+  prep_order_kernel<<<1, kPrepThreads, 0, st>>>(g, mask, hdr, order, keys, ntiles, maxcost, busy, nsm,
+                                                query_group_size(g));
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   AttnParams prm;
@@ -1015,6 +1117,8 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
   const bool narrow_ok = rx_edge < g.bw && (prm.rows_e == 16 || prm.rows_e == 32 || prm.rows_e == 64) &&
                          (g.bt == 1 || g.Hs % g.bh == 0);
   prm.pack = narrow_ok ? 128 / prm.rows_e : 1;
+  prm.qg = query_group_size(g);
+  prm.qps = prm.qg > 1 ? prm.rows_e / 32 : 1;
   const int grid = ntiles < nsm ? ntiles : nsm;
   return g.d == 128 ? launch_attn_d<128>(g, maps, prm, grid, st)
                     : launch_attn_d<64>(g, maps, prm, grid, st);
