@@ -40,7 +40,7 @@ METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16
 
 # DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
 # `ncu --set full` capture; valid only for the kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "adc1da1aba719505", "bytes": 389496576}
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "cd81ce7b57cb48de", "bytes": 389637888}
 
 
 def attn_traffic():
