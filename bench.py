@@ -222,7 +222,8 @@ def run_ours(args, rank, world, local_rank, wl=None):
             b = torch.cuda.Event(enable_timing=True)
             flush.fill_(float(i))
             fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream)
-            fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts, stream)
+            fv.fvattn_route_ws(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts,
+                               buf.route_ws, stream)
             a.record(stream)
             gr.replay()
             b.record(stream)
@@ -248,8 +249,10 @@ def run_ours(args, rank, world, local_rank, wl=None):
     # Per-stage device times (not added to the layer time above).  Pool streams 201 MB
     # (more than L2); route reads the pooled rows pool has just written.
     t_pool = back_to_back(lambda: fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream))
-    t_route = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
-                                                   buf.mask, buf.counts, stream))
+    t_route = back_to_back(lambda: fv.fvattn_route_ws(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
+                                                      buf.mask, buf.counts, buf.route_ws, stream))
+    t_route1 = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
+                                                    buf.mask, buf.counts, stream))
     # (inside a capture the calls must use the capturing stream: stream=None = current)
     attn_graph = graph_of(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
                                                               buf.workspace, buf.sm_busy_ns))
@@ -308,8 +311,9 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "attn_effective_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
-        "stage_timing": "pool, route: device time per launch over 20 back-to-back launches; attention: "
-                        "one captured call after L2 flush + pool + route (median)",
+        "route_one_kernel_ms": round(t_route1, 4),
+        "stage_timing": "pool, route (fvattn_route_ws, the layer's route): device time per launch over 20 "
+                        "back-to-back launches; attention: one captured call after L2 flush + pool + route (median)",
         "layer_step": "CUDA graph of pool -> route -> attention (LayerGraph)" if args.graph else "direct calls",
         "pool_route_gbs": round(pr_bytes / (pr_ms * 1e-3) / 1e9, 1),
         "pool_route_frac_of_hbm": round(pr_bytes / (pr_ms * 1e-3) / 1e9 / peaks["hbm"], 4),

@@ -8,6 +8,7 @@ Entry points mirror the C ABI in ``include/fvattn.h``:
 
 * ``fvattn_block_pool``   3D block mean-pooling of Q and K
 * ``fvattn_route``        per-head Top-p routing with a Top-k floor -> packed mask, counts
+* ``fvattn_route_ws``     the same routing in two kernels through a caller-owned workspace
 * ``fvattn_block_sparse_attn``  attention over the kept key blocks -> out, lse
 * ``fvattn_dense_attn``   the same kernel with every key block kept
 
@@ -25,6 +26,7 @@ from typing import Optional
 __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
+    "fvattn_route_workspace_size", "fvattn_route_ws",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
     "LayerBuffers", "LayerGraph",
 ]
@@ -88,6 +90,10 @@ _SIGS = {
                                     ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                     ctypes.c_void_p]),
     "fvattn_attn_workspace_size": (ctypes.c_size_t, [ctypes.c_void_p]),
+    "fvattn_route_workspace_size": (ctypes.c_size_t, [ctypes.c_void_p]),
+    "fvattn_route_ws": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                       ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fvattn_num_sms": (ctypes.c_int, []),
     "fvattn_block_sparse_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
@@ -183,6 +189,24 @@ def fvattn_route(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: flo
         _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"), _stream(stream)))
 
 
+def fvattn_route_workspace_size(g: Geometry) -> int:
+    cg = g.c()
+    return int(lib().fvattn_route_workspace_size(ctypes.byref(cg)))
+
+
+def fvattn_route_ws(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: float, mask, counts,
+                    workspace, stream=None) -> None:
+    import torch
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_route_ws", lib().fvattn_route_ws(
+        ctypes.byref(cg), _ptr(q_pool, torch.float32, pooled, "q_pool"),
+        _ptr(k_pool, torch.float32, pooled, "k_pool"), float(p), int(k_floor), float(scale),
+        _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"),
+        _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
+
+
 def fvattn_attn_workspace_size(g: Geometry) -> int:
     cg = g.c()
     return int(lib().fvattn_attn_workspace_size(ctypes.byref(cg)))
@@ -248,6 +272,7 @@ class LayerBuffers:
     lse: "object"
     workspace: "object"
     sm_busy_ns: "object"
+    route_ws: "object" = None   # workspace of fvattn_route_ws (None: the one-kernel route)
 
     @classmethod
     def allocate(cls, g: Geometry, device="cuda") -> "LayerBuffers":
@@ -260,7 +285,8 @@ class LayerBuffers:
                    out=torch.empty(g.B, g.H, g.N, g.d, dtype=torch.bfloat16, device=device),
                    lse=torch.empty(g.B, g.H, g.N, dtype=torch.float32, device=device),
                    workspace=ws,
-                   sm_busy_ns=torch.zeros(max(1, fvattn_num_sms()), dtype=torch.int64, device=device))
+                   sm_busy_ns=torch.zeros(max(1, fvattn_num_sms()), dtype=torch.int64, device=device),
+                   route_ws=torch.empty(fvattn_route_workspace_size(g), dtype=torch.uint8, device=device))
 
 
 def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optional[float] = None,
@@ -271,7 +297,10 @@ def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optiona
         scale = 1.0 / math.sqrt(g.d)
     b = buffers if buffers is not None else LayerBuffers.allocate(g, q.device)
     fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
-    fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
+    if b.route_ws is not None:
+        fvattn_route_ws(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, b.route_ws, stream)
+    else:
+        fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
     fvattn_block_sparse_attn(g, q, k, v, b.mask, scale, b.out, b.lse, b.workspace, b.sm_busy_ns, stream)
     return b
 

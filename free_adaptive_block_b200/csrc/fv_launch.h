@@ -20,6 +20,11 @@ cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, f
                         cudaStream_t st);
 cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
                          float scale, uint32_t* mask, int32_t* counts, cudaStream_t st);
+// The same routing in two kernels (logits into `ws`, then selection); ws holds
+// route_ws_bytes(g) bytes.
+size_t route_ws_bytes(const Geo& g);
+cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st);
 
 struct AttnMaps {
   CUtensorMap q, qe, k, ke, v, ve;   // full-width and x-edge boxes of Q, K, V

@@ -420,4 +420,134 @@ cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p
                     : launch_route_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, st);
 }
 
+// ----------------------------------------------------------------------------
+// Routing in two kernels, for callers that pass a workspace (fvattn_route_ws): the
+// logits of every (query block, key block) pair go to the workspace as an fp32 matrix
+// per (b, h), rows padded to words * 32; then one warp per query block runs the same
+// selection as route_kernel from its row.  The per-logit arithmetic is the fused
+// kernel's (two partial sums over the even and odd components of each float4 of d, in
+// ascending d, added at the end, times scale), so both paths give the same mask.
+// ----------------------------------------------------------------------------
+constexpr int kLogitTile = 64;         // query x key blocks per CTA
+
+template <int D>
+__global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restrict__ qp,
+                                                     const float* __restrict__ kp, float scale,
+                                                     float* __restrict__ logits) {
+  constexpr int RS = D + 4;            // padded row (floats)
+  extern __shared__ __align__(16) unsigned char lg_smem[];
+  float* sQ = reinterpret_cast<float*>(lg_smem);   // [64][D + 4]
+  float* sK = sQ + kLogitTile * RS;                // [64][D + 4]
+  const int nB = g.nB, nBpad = g.words * 32;
+  const int bhi = blockIdx.z;
+  const int q0 = blockIdx.x * kLogitTile, k0 = blockIdx.y * kLogitTile;
+  const float* qh = qp + static_cast<size_t>(bhi) * nB * D;
+  const float* kh = kp + static_cast<size_t>(bhi) * nB * D;
+  for (int e = threadIdx.x; e < kLogitTile * D / 4; e += 256) {
+    const int r = e / (D / 4), d4 = e - r * (D / 4);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(sQ + r * RS)[d4] =
+        q0 + r < nB ? reinterpret_cast<const float4*>(qh + static_cast<size_t>(q0 + r) * D)[d4] : z;
+    reinterpret_cast<float4*>(sK + r * RS)[d4] =
+        k0 + r < nB ? reinterpret_cast<const float4*>(kh + static_cast<size_t>(k0 + r) * D)[d4] : z;
+  }
+  __syncthreads();
+  // thread (ty, tx) takes query rows ty + 16 i and key blocks tx + 16 j, i, j < 4
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  uint64_t acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
+#pragma unroll 4
+  for (int d4 = 0; d4 < D / 4; ++d4) {
+    uint64_t qxy[4], qzw[4], kxy[4], kzw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = reinterpret_cast<const float4*>(sQ + (ty + 16 * i) * RS)[d4];
+      qxy[i] = f32x2(x.x, x.y);
+      qzw[i] = f32x2(x.z, x.w);
+      const float4 k4 = reinterpret_cast<const float4*>(sK + (tx + 16 * i) * RS)[d4];
+      kxy[i] = f32x2(k4.x, k4.y);
+      kzw[i] = f32x2(k4.z, k4.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = ffma2(qxy[i], kxy[j], acc[i][j]);   // a0 += x.x k.x, a1 += x.y k.y
+        acc[i][j] = ffma2(qzw[i], kzw[j], acc[i][j]);   // a0 += x.z k.z, a1 += x.w k.w
+      }
+  }
+  float* out = logits + static_cast<size_t>(bhi) * nB * nBpad;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int qr = q0 + ty + 16 * i;
+    if (qr >= nB) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int kc = k0 + tx + 16 * j;
+      if (kc >= nB) continue;
+      float a0, a1;
+      unpack_f32x2(acc[i][j], a0, a1);
+      out[static_cast<size_t>(qr) * nBpad + kc] = (a0 + a1) * scale;
+    }
+  }
+}
+
+template <int MAXW>
+__global__ void __launch_bounds__(256) select_kernel(Geo g, const float* __restrict__ logits, float p,
+                                                     int k_floor, uint32_t* __restrict__ mask,
+                                                     int32_t* __restrict__ counts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nB = g.nB, nBpad = g.words * 32;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + warp;   // (b*h) * nB + qb
+  if (row >= static_cast<long long>(g.B) * g.H * nB) return;
+  const int qb = static_cast<int>(row % nB);
+  select_row<MAXW>(logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
+                   mask + static_cast<size_t>(row) * g.words, counts + row, lane);
+}
+
+size_t route_ws_bytes(const Geo& g) {
+  return static_cast<size_t>(g.B) * g.H * g.nB * (static_cast<size_t>(g.words) * 32) * 4;
+}
+
+template <int D, int MAXW>
+static cudaError_t launch_route2_t(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                                   float scale, uint32_t* mask, int32_t* counts, float* logits,
+                                   cudaStream_t st) {
+  const int tiles = (g.nB + kLogitTile - 1) / kLogitTile;
+  const int smem = 2 * kLogitTile * (D + 4) * 4;
+  cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  logits_kernel<D><<<dim3(tiles, tiles, g.B * g.H), 256, smem, st>>>(g, qp, kp, scale, logits);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const long long rows = static_cast<long long>(g.B) * g.H * g.nB;
+  select_kernel<MAXW><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(g, logits, p, k_floor, mask, counts);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_route2_d(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                                   float scale, uint32_t* mask, int32_t* counts, float* logits,
+                                   cudaStream_t st) {
+  if (g.words <= 4) return launch_route2_t<D, 4>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 8) return launch_route2_t<D, 8>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 12) return launch_route2_t<D, 12>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 16) return launch_route2_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 20) return launch_route2_t<D, 20>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 24) return launch_route2_t<D, 24>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 32) return launch_route2_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  if (g.words <= 48) return launch_route2_t<D, 48>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+  return launch_route2_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+}
+
+cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st) {
+  float* logits = static_cast<float*>(ws);
+  return g.d == 128 ? launch_route2_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st)
+                    : launch_route2_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+}
+
 }  // namespace fv

@@ -99,6 +99,29 @@ FVATTN_API fvattn_status_t fvattn_route(const fvattn_geom_t* g, const float* q_p
                              float p, int k_floor, float scale,
                              uint32_t* mask, int32_t* counts, fvattn_stream_t stream);
 
+/* Bytes of device workspace fvattn_route_ws needs: one fp32 logit per (query block, key
+ * block) pair of every (b, h), rows padded to words * 32 entries
+ * (B * H * nB * words * 32 * 4 bytes; 5.4 MB at 21x30x52 with 1x8x16 blocks and 12
+ * heads, 181 MB at 121x30x52).  0 for an invalid geometry. */
+FVATTN_API size_t fvattn_route_workspace_size(const fvattn_geom_t* g);
+
+/* fvattn_route, computed in two kernels through a caller-owned workspace: the logits of
+ * all block pairs first (a tiled fp32 product written to `workspace`), then the
+ * selection, one query block per warp.  Same definition, inputs, outputs, argument
+ * domains and error behaviour as fvattn_route (FVATTN 稀疏路由前端 §1: Top-p with a Top-k
+ * floor and the own block over softmax(pooled q . pooled k * scale)).  The per-logit
+ * arithmetic is the same as fvattn_route's, so the two calls give the same mask and
+ * counts.  This form spreads the logits over many more CTAs, which matters most when nB
+ * is large.
+ *   workspace, ws_bytes : >= fvattn_route_workspace_size(g) bytes of device memory,
+ *                         16-byte aligned, owned by the caller; its contents on entry
+ *                         do not matter and on return are the logits (scaled).
+ * Returns FVATTN_ERR_WORKSPACE when the workspace is missing or too small. */
+FVATTN_API fvattn_status_t fvattn_route_ws(const fvattn_geom_t* g, const float* q_pool, const float* k_pool,
+                                           float p, int k_floor, float scale, uint32_t* mask,
+                                           int32_t* counts, void* workspace, size_t ws_bytes,
+                                           fvattn_stream_t stream);
+
 /* Bytes of device workspace fvattn_block_sparse_attn / fvattn_dense_attn need
  * for geometry g (a tile queue and a status word).  0 for a malformed geometry. */
 FVATTN_API size_t fvattn_attn_workspace_size(const fvattn_geom_t* g);

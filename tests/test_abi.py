@@ -71,6 +71,15 @@ def test_host_side_argument_checks(L):
                                0x6000, 64, None, None) == E["FVATTN_ERR_WORKSPACE"]
     assert L.fvattn_block_pool(ctypes.byref(cg), 0x1000, None, 0x3000, 0x4000, None) == E["FVATTN_ERR_INVALID_ARG"]
     assert L.fvattn_device_status(None, None) == E["FVATTN_ERR_INVALID_ARG"]
+    # two-kernel route: the route checks, then a missing / short / misaligned workspace
+    need = fv.fvattn_route_workspace_size(G480)
+    assert need == 12 * 336 * 11 * 32 * 4
+    args = (ctypes.byref(cg), 0x1000, 0x2000, 0.9, 4, 0.088, 0x3000, 0x4000)
+    assert L.fvattn_route_ws(*args, None, need, None) == E["FVATTN_ERR_WORKSPACE"]
+    assert L.fvattn_route_ws(*args, 0x10000, need - 1, None) == E["FVATTN_ERR_WORKSPACE"]
+    assert L.fvattn_route_ws(*args, 0x10008, need, None) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert L.fvattn_route_ws(ctypes.byref(cg), 0x1000, 0x2000, -1.0, 4, 0.088, 0x3000, 0x4000,
+                             0x10000, need, None) == E["FVATTN_ERR_INVALID_ARG"]
 
 
 def test_status_strings(L):

@@ -121,3 +121,27 @@ def test_repeat_bitwise(wl, reps, inputs):
             continue
         nbad = int((o != ref_out).any(-1).sum())
         assert nbad == 0 and bool((lse == ref_lse).all()), f"call {r}: {nbad} rows differ from the first call"
+
+
+@pytest.mark.parametrize("wl", SMALL + [W.WAN21_480P], ids=lambda w: w.name)
+@pytest.mark.parametrize("p,k", [(None, None), (0.5, 1), (1.0, 0), (0.0, 0)])
+def test_route_ws_equals_route(wl, p, k, inputs):
+    """The two-kernel route (logits through a workspace, then selection) gives exactly
+    the mask and counts of the one-kernel route."""
+    import torch
+    import free_adaptive_block_b200 as fv
+    p = wl.p if p is None else p
+    k = wl.k_floor if k is None else k
+    x = inputs(wl)
+    g = P.geometry(wl)
+    sc = P.scale_of(wl.d)
+    q, kk = P.to_dev(x["q"]), P.to_dev(x["k"])
+    b = fv.LayerBuffers.allocate(g)
+    fv.fvattn_block_pool(g, q, kk, b.q_pool, b.k_pool)
+    fv.fvattn_route(g, b.q_pool, b.k_pool, p, k, sc, b.mask, b.counts)
+    m1, c1 = b.mask.clone(), b.counts.clone()
+    b.mask.fill_(-1)
+    b.counts.fill_(-1)
+    fv.fvattn_route_ws(g, b.q_pool, b.k_pool, p, k, sc, b.mask, b.counts, b.route_ws)
+    torch.cuda.synchronize()
+    assert torch.equal(b.mask, m1) and torch.equal(b.counts, c1)

@@ -49,3 +49,23 @@ def test_sweep_480p():
     f = np.asarray(fracs).reshape(len(W.SWEEP_P), len(W.SWEEP_K))
     assert (np.diff(f, axis=0) >= -1e-12).all() and (np.diff(f, axis=1) >= -1e-12).all()
     assert f[-1].min() == 1.0          # p = 1 keeps everything
+
+
+def test_route_ws_equals_route_720p():
+    """The two-kernel route gives exactly the one-kernel route's mask at 720p (20 mask
+    words, 630 blocks)."""
+    import torch
+    import free_adaptive_block_b200 as fv
+    wl = W.WAN22_720P
+    x = W.generate(wl)
+    g = P.geometry(wl)
+    sc = P.scale_of(wl.d)
+    q, k = P.to_dev(x["q"]), P.to_dev(x["k"])
+    b = fv.LayerBuffers.allocate(g)
+    fv.fvattn_block_pool(g, q, k, b.q_pool, b.k_pool)
+    fv.fvattn_route(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts)
+    m1, c1 = b.mask.clone(), b.counts.clone()
+    b.mask.fill_(-1)
+    fv.fvattn_route_ws(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts, b.route_ws)
+    torch.cuda.synchronize()
+    assert torch.equal(b.mask, m1) and torch.equal(b.counts, c1)
