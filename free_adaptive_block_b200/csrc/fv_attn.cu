@@ -1021,29 +1021,42 @@ __global__ void __launch_bounds__(kPrepThreads) prep_order_kernel(Geo g, const u
     if (cell >= 0 && lane == __ffs(peers) - 1) atomicAdd(&hist[cell], __popc(peers));
   }
   __syncthreads();
-  // exclusive scan of the histogram in (slice rank, bucket) order: warp 0, 256 cells per lane
+  // exclusive scan of the histogram in (slice rank, bucket) order over the whole block:
+  // thread t owns `per` consecutive cells; warp scans, then a scan of the warp totals
   const int cells = ngroups * nbk;
-  const int per = (cells + 31) / 32;
+  const int per = (cells + kPrepThreads - 1) / kPrepThreads;
+  __shared__ int wsum[kPrepThreads / 32];
+  int run = 0;
+  for (int i = 0; i < per; ++i) {
+    const int idx = t * per + i;
+    if (idx < cells) run += hist[idx];
+  }
+  int incl = run;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const int v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  if (lane == 31) wsum[t >> 5] = incl;
+  __syncthreads();
   if (t < 32) {
-    int run = 0;
-    for (int i = 0; i < per; ++i) {
-      const int idx = t * per + i;
-      if (idx < cells) run += hist[idx];
-    }
-    int incl = run;
+    const int w = wsum[t];
+    int wi = w;
 #pragma unroll
     for (int off = 1; off < 32; off <<= 1) {
-      const int v = __shfl_up_sync(0xffffffffu, incl, off);
-      if (t >= off) incl += v;
+      const int v = __shfl_up_sync(0xffffffffu, wi, off);
+      if (t >= off) wi += v;
     }
-    int acc = incl - run;
-    for (int i = 0; i < per; ++i) {
-      const int idx = t * per + i;
-      if (idx < cells) {
-        const int c = hist[idx];
-        hist[idx] = acc;
-        acc += c;
-      }
+    wsum[t] = wi - w;   // exclusive prefix of the warp totals
+  }
+  __syncthreads();
+  int acc = wsum[t >> 5] + incl - run;
+  for (int i = 0; i < per; ++i) {
+    const int idx = t * per + i;
+    if (idx < cells) {
+      const int c = hist[idx];
+      hist[idx] = acc;
+      acc += c;
     }
   }
   __syncthreads();
