@@ -39,8 +39,9 @@ from free_adaptive_block_b200 import workloads as W  # noqa: E402
 METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16 peak"
 
 # DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
-# `ncu --set full` capture; valid only for the kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "cd81ce7b57cb48de", "bytes": 389637888}
+# ncu capture of dram__bytes_read.sum + dram__bytes_write.sum; valid only for the
+# kernel source it was taken from.
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "d1a9d3edfb431bc0", "bytes": 388617984}
 
 
 def attn_traffic():
@@ -76,35 +77,71 @@ def config_of(wl, extra=None):
 
 # ----------------------------------------------------------------------------- clocks
 class ClockSampler:
-    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs."""
+    """Samples nvidia-smi SM clocks and throttle reasons while the timed region runs.
+
+    nvidia-smi takes a while to start, and a timed region can be shorter than its
+    sampling interval, so the bench waits for the first sample before it opens the
+    timed region, marks the region's ends, and after it closes waits for the next
+    sample; the report keeps the samples that arrived inside the region plus that
+    one (reasons are sticky per interval, so it still covers the region's tail).
+    """
     FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
               "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
               "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+    INTERVAL_MS = 50
 
-    def __init__(self, index: int):
-        self.index = index
+    def __init__(self, local_rank: int):
+        vis = os.environ.get("CUDA_VISIBLE_DEVICES", "").split(",")
+        vis = [v.strip() for v in vis if v.strip()]
+        # nvidia-smi numbers GPUs physically; CUDA_VISIBLE_DEVICES maps the rank's
+        # device to that numbering when it is set, else the local rank is the index.
+        self.ids = [str(local_rank)]
+        if local_rank < len(vis) and vis[local_rank] != str(local_rank):
+            self.ids.insert(0, vis[local_rank])
+        self.index = self.ids[0]
         self.proc = None
-        self.lines = []
+        self.lines = []          # (arrival time, csv line)
         self.thread = None
+        self.t_begin = self.t_end = None
 
-    def start(self):
-        try:
-            self.proc = subprocess.Popen(
-                ["nvidia-smi", f"--id={self.index}", f"--query-gpu={self.FIELDS}",
-                 "--format=csv,noheader,nounits", "-lms", "200"],
-                stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+    def start(self, wait_s: float = 5.0):
+        for idx in self.ids:
+            self.index = idx
+            try:
+                self.proc = subprocess.Popen(
+                    ["nvidia-smi", f"--id={idx}", f"--query-gpu={self.FIELDS}",
+                     "--format=csv,noheader,nounits", "-lms", str(self.INTERVAL_MS)],
+                    stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            except Exception:
+                self.proc = None
+                return
             self.thread = threading.Thread(target=self._read, daemon=True)
             self.thread.start()
-        except Exception:
-            self.proc = None
+            deadline = time.monotonic() + wait_s
+            while not self.lines and time.monotonic() < deadline and self.proc.poll() is None:
+                time.sleep(0.01)
+            if self.lines or self.proc.poll() is None:
+                return
+            self.thread.join(timeout=2)      # this id was refused: try the next one
 
     def _read(self):
         for line in self.proc.stdout:
-            self.lines.append(line.strip())
+            self.lines.append((time.monotonic(), line.strip()))
+
+    def begin(self):
+        self.t_begin = time.monotonic()
+
+    def end(self):
+        self.t_end = time.monotonic()
 
     def stop(self):
         if self.proc is None:
             return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        t_end = self.t_end if self.t_end is not None else time.monotonic()
+        deadline = time.monotonic() + 2.0
+        while (not any(t > t_end for t, _ in self.lines) and time.monotonic() < deadline
+               and self.proc.poll() is None):
+            time.sleep(0.01)
         self.proc.terminate()
         try:
             self.proc.wait(timeout=5)
@@ -112,9 +149,12 @@ class ClockSampler:
             self.proc.kill()
         if self.thread:
             self.thread.join(timeout=2)
+        t_begin = self.t_begin if self.t_begin is not None else 0.0
+        inside = [ln for t, ln in self.lines if t_begin <= t <= t_end]
+        after = [ln for t, ln in self.lines if t > t_end][:1]
         sm, smax, reasons = [], [], set()
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for ln in self.lines:
+        for ln in inside + after:
             parts = [p.strip() for p in ln.split(",")]
             if len(parts) < 8:
                 continue
@@ -128,7 +168,9 @@ class ClockSampler:
                     reasons.add(nm)
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(smax) if smax else None,
-                "reasons": sorted(reasons), "samples": len(sm)}
+                "reasons": sorted(reasons), "samples": len(sm),
+                "samples_inside_timed_region": len(inside),
+                "interval_ms": self.INTERVAL_MS}
 
 
 # ----------------------------------------------------------------------------- GPU arm
@@ -175,18 +217,21 @@ def run_ours(args, rank, world, local_rank, wl=None):
 
     ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
     sampler = ClockSampler(local_rank) if rank == 0 else None
+    if sampler:
+        sampler.start()
     if world > 1:
         torch.distributed.barrier()
     torch.cuda.synchronize(dev)
     if sampler:
-        sampler.start()
-        time.sleep(0.3)
+        sampler.begin()
     for i in range(args.steps):
         ev[i][0].record(stream)
         step()
         ev[i][1].record(stream)
         flush.fill_(float(i))
     torch.cuda.synchronize(dev)
+    if sampler:
+        sampler.end()
     if world > 1:
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
@@ -417,21 +462,27 @@ def run_sweep(args, local_rank):
     real = MX.real_counts(wl0.T, wl0.Hs, wl0.Ws, wl0.bt, wl0.bh, wl0.bw)
     peaks = load_peaks()
 
-    def timed(fn, reps):
+    def timed(fn, p, k_floor, reps):
+        """Median device time of one call in its place in the layer, as on the headline
+        line: L2 flushed, then pool and route for this point (untimed; they also absorb
+        the write-back of the flush's dirty lines), then the timed call."""
         ts = []
         for i in range(3 + reps):
             a = torch.cuda.Event(enable_timing=True)
             b = torch.cuda.Event(enable_timing=True)
+            flush.fill_(float(i))
+            fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
+            fv.fvattn_route(g, buf.q_pool, buf.k_pool, p, k_floor, scale, buf.mask, buf.counts)
             a.record()
             fn()
             b.record()
-            flush.fill_(float(i))
             torch.cuda.synchronize()
             if i >= 3:
                 ts.append(a.elapsed_time(b))
         return statistics.median(ts)
 
-    dense_ms = timed(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace), args.steps)
+    dense_ms = timed(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace),
+                     wl0.p, wl0.k_floor, args.steps)
     for wl in W.sweep():
         fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
         fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts)
@@ -439,7 +490,8 @@ def run_sweep(args, local_rank):
         keep = MX.unpack_words(buf.mask.cpu().numpy().view(np.uint32), g.nB)
         eff = MX.effective_flops(keep, real, wl.d)
         ms = timed(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
-                                                        buf.workspace, buf.sm_busy_ns), args.steps)
+                                                        buf.workspace, buf.sm_busy_ns),
+                   wl.p, wl.k_floor, args.steps)
         busy = buf.sm_busy_ns.cpu().numpy()
         busy = busy[busy > 0]
         print(json.dumps({"sweep_point": wl.name, "p": wl.p, "k_floor": wl.k_floor,
