@@ -173,6 +173,25 @@ class ClockSampler:
                 "interval_ms": self.INTERVAL_MS}
 
 
+# ----------------------------------------------------------------------------- ranks
+def max_over_ranks(x: float, world: int, device=None) -> float:
+    """The largest x over all ranks (x itself at world size 1). Every rank must call it
+    at the same point: it is one all-reduce. `device` is where the reduced tensor lives:
+    the rank's GPU under NCCL, the CPU under gloo."""
+    if world <= 1:
+        return float(x)
+    import torch
+    t = torch.tensor([float(x)], device=device, dtype=torch.float64)
+    torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+    return float(t.item())
+
+
+def whole_job_tflops(eff_flop_per_rank: float, world: int, ms_per_step: float) -> float:
+    """Whole-job throughput: every rank processes the same workload (replicas), so the
+    job's FLOPs per step are world x one rank's, over the slowest rank's step time."""
+    return eff_flop_per_rank * world / (ms_per_step * 1e-3) / 1e12
+
+
 # ----------------------------------------------------------------------------- GPU arm
 def run_ours(args, rank, world, local_rank, wl=None):
     import torch
@@ -236,11 +255,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
         torch.distributed.barrier()
     clocks = sampler.stop() if sampler else None
     t_layer = [ev[i][0].elapsed_time(ev[i][1]) for i in range(args.steps)]
-    total_ms = sum(t_layer)
-    if world > 1:
-        t = torch.tensor([total_ms], device=dev, dtype=torch.float64)
-        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
-        total_ms = float(t.item())
+    total_ms = max_over_ranks(sum(t_layer), world, dev)
     busy = buf.sm_busy_ns.cpu().numpy()
     busy = busy[busy > 0]
     if fv.fvattn_device_status(buf.workspace, stream) != 0:
@@ -305,7 +320,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
 
     if args.layer_only:
         ms_step = total_ms / args.steps
-        return {"metric": METRIC, "value": round(eff * world / (ms_step * 1e-3) / 1e12, 3), "unit": UNIT,
+        return {"metric": METRIC, "value": round(whole_job_tflops(eff, world, ms_step), 3), "unit": UNIT,
                 "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
                 "ms_per_step": round(ms_step, 4), "attn_ms": round(attn_ms, 4),
                 "layer_only": True}
@@ -337,12 +352,12 @@ def run_ours(args, rank, world, local_rank, wl=None):
         torch.cuda.synchronize(dev)
         if i >= 2:
             e2e_t.append(a.elapsed_time(b))
-    e2e_ms = statistics.mean(e2e_t)
+    e2e_ms = max_over_ranks(statistics.mean(e2e_t), world, dev)
     h2d = sum(pinned[n].numel() * 2 for n in ("q", "k", "v"))
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
     ms_step = total_ms / args.steps
-    value = eff * world / (ms_step * 1e-3) / 1e12
+    value = whole_job_tflops(eff, world, ms_step)
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
     pr_bytes = MX.pool_route_bytes(wl.B, wl.H, wl.N, g.nB, wl.d, g.words)
     pr_ms = t_pool + t_route
@@ -372,7 +387,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
                      "achieved": round(attn_tflops, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
                      "frac": round(attn_tflops / peaks["bf16"], 4), "traffic": attn_traffic(),
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
-        "e2e": {"value": round(eff * world / (e2e_ms * 1e-3) / 1e12, 3), "unit": UNIT,
+        "e2e": {"value": round(whole_job_tflops(eff, world, e2e_ms), 3), "unit": UNIT,
                 "how": "pinned host Q/K/V -> device, layer step, out/lse -> pinned host, one stream",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
         "gpu_launches": 5 * args.steps,   # pool, route, prep_cost, prep_order, attention
