@@ -108,7 +108,7 @@ FVATTN_API size_t fvattn_route_workspace_size(const fvattn_geom_t* g);
 /* fvattn_route, computed in two kernels through a caller-owned workspace: the logits of
  * all block pairs first (a tiled fp32 product written to `workspace`), then the
  * selection, one query block per warp.  Same definition, inputs, outputs, argument
- * domains and error behaviour as fvattn_route (FVATTN 稀疏路由前端 §1: Top-p with a Top-k
+ * domains and error behaviour as fvattn_route (FVAttn explainer 核心方法 §1: Top-p with a Top-k
  * floor and the own block over softmax(pooled q . pooled k * scale)).  The per-logit
  * arithmetic is the same as fvattn_route's, so the two calls give the same mask and
  * counts.  This form spreads the logits over many more CTAs, which matters most when nB
