@@ -356,6 +356,9 @@ def run_ours(args, rank, world, local_rank, wl=None):
     h2d = sum(pinned[n].numel() * 2 for n in ("q", "k", "v"))
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
+    # the library's kernels one layer step launches: pool; route (logits + select through
+    # the route workspace, else the one-kernel route); prep_cost, prep_order, attention
+    launches_per_step = 1 + (2 if buf.route_ws is not None else 1) + 3
     ms_step = total_ms / args.steps
     value = whole_job_tflops(eff, world, ms_step)
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
@@ -390,7 +393,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "e2e": {"value": round(whole_job_tflops(eff, world, e2e_ms), 3), "unit": UNIT,
                 "how": "pinned host Q/K/V -> device, layer step, out/lse -> pinned host, one stream",
                 "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
-        "gpu_launches": 5 * args.steps,   # pool, route, prep_cost, prep_order, attention
+        "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
     return line
