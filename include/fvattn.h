@@ -27,7 +27,12 @@
  *   before anything is launched.  Launch failures return FVATTN_ERR_CUDA;
  *   faults during execution surface at the caller's next synchronisation.
  * - No C++ exception crosses this interface.
- * - Supported: d in {64, 128}; 1 <= bt*bh*bw <= 128; nB <= 2048; B*H*nB < 2^24.
+ * - Every extent of the geometry (B, H, T, Hs, Ws, bt, bh, bw) must be >= 1: an
+ *   empty batch, head set or latent is FVATTN_ERR_INVALID_ARG (a caller with nothing
+ *   to compute makes no call).
+ * - Supported: d in {64, 128}; 1 <= bt*bh*bw <= 128; nB <= 2048; B*H*nB < 2^24;
+ *   N < 2^31; B*H*N*d < 2^40; Ws, Hs <= 65535 and T <= 32767 (tensor-map extents).
+ *   Other valid geometries return FVATTN_ERR_UNSUPPORTED.
  */
 #ifndef FVATTN_H_
 #define FVATTN_H_

@@ -60,6 +60,18 @@ def test_host_side_argument_checks(L):
     assert call_route(L, big_block) == E["FVATTN_ERR_UNSUPPORTED"]
     zero = fv.Geometry(1, 0, 4, 16, 16, 128, 1, 8, 16)
     assert call_route(L, zero) == E["FVATTN_ERR_INVALID_ARG"]
+    # every empty extent is an argument error, for every entry point's geometry check
+    for i in range(9):
+        ext = [1, 12, 21, 30, 52, 128, 1, 8, 16]
+        ext[i] = 0
+        assert call_route(L, fv.Geometry(*ext)) == E["FVATTN_ERR_INVALID_ARG"], i
+        ext[i] = -3
+        assert call_route(L, fv.Geometry(*ext)) == E["FVATTN_ERR_INVALID_ARG"], i
+    # limits of the tensor maps and index types
+    assert call_route(L, fv.Geometry(1, 1, 1, 8, 65536, 128, 1, 8, 16)) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert call_route(L, fv.Geometry(1, 1, 32768, 1, 16, 128, 1, 1, 16)) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert call_route(L, fv.Geometry(1, 1, 16, 65535, 2049, 128, 16, 8, 1)) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert call_route(L, fv.Geometry(1, 1, 1, 2, 2049 * 64, 64, 1, 2, 64)) == E["FVATTN_ERR_UNSUPPORTED"]
     assert L.fvattn_route(None, 0x1000, 0x2000, 0.9, 4, 0.1, 0x3000, 0x4000, None) == E["FVATTN_ERR_INVALID_ARG"]
     cg = G480.c()
     # attention: missing mask, missing / short workspace
