@@ -374,6 +374,9 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "bf16",
         "data": "synthetic", "config": config_of(wl),
         "ms_per_layer": round(ms_step, 4),
+        # this rank's per-step spread (the headline above is the mean, max over ranks)
+        "ms_per_layer_median": round(statistics.median(t_layer), 4),
+        "ms_per_layer_min": round(min(t_layer), 4), "ms_per_layer_max": round(max(t_layer), 4),
         "attn_ms": round(attn_ms, 4),
         "attn_ms_mean": round(attn_ms_mean, 4),
         "attn_effective_tflops": round(attn_tflops, 2),
