@@ -145,11 +145,20 @@ def _stream(stream) -> Optional[int]:
     return getattr(stream, "cuda_stream", stream)
 
 
+def _current_device() -> int:
+    import torch
+    return torch.cuda.current_device()
+
+
 def _ptr(t, dtype, shape, name):
     if t is None:
         return None
     if not t.is_cuda:
         raise ValueError(f"{name} must be a CUDA tensor")
+    dev = _current_device()
+    if t.device.index != dev:
+        # the kernels run on the current device and would fault on another GPU's memory
+        raise ValueError(f"{name} is on cuda:{t.device.index}, but the current device is cuda:{dev}")
     if t.dtype != dtype:
         raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
     if shape is not None and tuple(t.shape) != tuple(shape):
@@ -216,9 +225,17 @@ def fvattn_num_sms() -> int:
     return int(lib().fvattn_num_sms())
 
 
+def _check_busy(sm_busy_ns) -> None:
+    """The kernel writes one entry per CTA, up to one per SM."""
+    if sm_busy_ns is not None and sm_busy_ns.numel() < fvattn_num_sms():
+        raise ValueError(f"sm_busy_ns needs fvattn_num_sms() = {fvattn_num_sms()} entries, "
+                         f"got {sm_busy_ns.numel()}")
+
+
 def fvattn_block_sparse_attn(g: Geometry, q, k, v, mask, scale: float, out, lse, workspace,
                              sm_busy_ns=None, stream=None) -> None:
     import torch
+    _check_busy(sm_busy_ns)
     tok = (g.B, g.H, g.N, g.d)
     cg = g.c()
     _ok("fvattn_block_sparse_attn", lib().fvattn_block_sparse_attn(
@@ -232,6 +249,7 @@ def fvattn_block_sparse_attn(g: Geometry, q, k, v, mask, scale: float, out, lse,
 def fvattn_dense_attn(g: Geometry, q, k, v, scale: float, out, lse, workspace, sm_busy_ns=None,
                       stream=None) -> None:
     import torch
+    _check_busy(sm_busy_ns)
     tok = (g.B, g.H, g.N, g.d)
     cg = g.c()
     _ok("fvattn_dense_attn", lib().fvattn_dense_attn(
@@ -246,6 +264,7 @@ def fvattn_block_sparse_attn_noalloc(g: Geometry, q, k, v, mask, scale: float, o
     """fvattn_block_sparse_attn without a workspace argument: for callers that cannot
     allocate device memory; the library uses its own static scratch area instead."""
     import torch
+    _check_busy(sm_busy_ns)
     tok = (g.B, g.H, g.N, g.d)
     cg = g.c()
     _ok("fvattn_block_sparse_attn_noalloc", lib().fvattn_block_sparse_attn_noalloc(
