@@ -327,6 +327,16 @@ def run_ours(args, rank, world, local_rank, wl=None):
                 "ms_per_step": round(ms_step, 4), "attn_ms": round(attn_ms, 4),
                 "layer_only": True}
 
+    # Host time of one direct call (Python binding, C entry point, three launches), with
+    # the GPU kept busy by the calls queued before it; outside every timed region.
+    torch.cuda.synchronize(dev)
+    h0 = time.perf_counter()
+    for _ in range(20):
+        fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse, buf.workspace,
+                                    buf.sm_busy_ns, stream)
+    attn_host_us = (time.perf_counter() - h0) / 20 * 1e6
+    torch.cuda.synchronize(dev)
+
     # dense baseline (p = 1 through the same kernel), same protocol
     dense_graph = graph_of(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace,
                                                         None))
@@ -379,6 +389,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "ms_per_layer_min": round(min(t_layer), 4), "ms_per_layer_max": round(max(t_layer), 4),
         "attn_ms": round(attn_ms, 4),
         "attn_ms_mean": round(attn_ms_mean, 4),
+        "attn_call_host_us": round(attn_host_us, 1),
         "attn_effective_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
