@@ -1,6 +1,8 @@
-"""The oracle's route against exhaustive search, on many random rows (hypothesis).
+"""Property tests of the oracle (hypothesis): the route against exhaustive search on many
+random rows, and masked attention against torch's scaled_dot_product_attention in fp64
+on random ragged geometries and block masks.
 
-The oracle keeps the shortest prefix of the (score desc, index asc) order whose mass is
+The route: the oracle keeps the shortest prefix of the (score desc, index asc) order whose mass is
 >= p, lengthened to the Top-k floor, plus the own block.  The exhaustive search finds,
 over all subsets, the smallest size whose best subset reaches p, then the heaviest subset
 of size max(that, k) with ties to the lexicographically smallest, plus the own block: the
@@ -54,3 +56,38 @@ def test_route_row_equals_exhaustive_search(case):
     if p >= 1.0 or k >= nB:
         assert want.all()
     assert math.isclose(float(s.sum()), 1.0, rel_tol=0, abs_tol=1e-12)
+
+
+@st.composite
+def attn_cases(draw):
+    T, Hs, Ws = draw(st.integers(1, 3)), draw(st.integers(1, 7)), draw(st.integers(1, 9))
+    bt, bh, bw = draw(st.integers(1, 2)), draw(st.integers(1, 4)), draw(st.integers(1, 5))
+    d = draw(st.sampled_from([4, 8, 16]))
+    seed = draw(st.integers(0, 2**31 - 1))
+    density = draw(st.sampled_from([0.1, 0.4, 0.8]))
+    return T, Hs, Ws, bt, bh, bw, d, seed, density
+
+
+@settings(max_examples=60, derandomize=True, deadline=None)
+@given(attn_cases())
+def test_masked_attention_equals_sdpa_with_token_mask(case):
+    """masked_attn on random ragged geometries and block masks (each row keeps its own
+    block) equals scaled_dot_product_attention in fp64 with the token-level mask."""
+    import torch
+    T, Hs, Ws, bt, bh, bw, d, seed, density = case
+    g = O.block_geometry(T, Hs, Ws, bt, bh, bw)
+    rng = np.random.default_rng(seed)
+    N = T * Hs * Ws
+    Q, K, V = (rng.standard_normal((1, 2, N, d)) * s for s in (1.5, 1.0, 1.0))
+    keep = rng.random((1, 2, g.nB, g.nB)) < density
+    keep[..., np.arange(g.nB), np.arange(g.nB)] = True
+    scale = 1.0 / math.sqrt(d)
+    tokens, out, lse = O.masked_attn(Q, K, V, keep, g, scale)
+    bt_of = g.block_of_token
+    tok_mask = torch.from_numpy(keep[:, :, bt_of][:, :, :, bt_of])
+    tq, tk, tv = (torch.from_numpy(a) for a in (Q, K, V))
+    ref = torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, attn_mask=tok_mask, scale=scale)
+    np.testing.assert_allclose(out, ref.numpy()[:, :, tokens], atol=1e-12)
+    logits = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
+    ref_lse = torch.logsumexp(logits.masked_fill(~tok_mask, float("-inf")), dim=-1)
+    np.testing.assert_allclose(lse, ref_lse.numpy()[:, :, tokens], atol=1e-12)
