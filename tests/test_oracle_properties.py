@@ -91,3 +91,31 @@ def test_masked_attention_equals_sdpa_with_token_mask(case):
     logits = torch.einsum("bhid,bhjd->bhij", tq, tk) * scale
     ref_lse = torch.logsumexp(logits.masked_fill(~tok_mask, float("-inf")), dim=-1)
     np.testing.assert_allclose(lse, ref_lse.numpy()[:, :, tokens], atol=1e-12)
+
+
+@st.composite
+def pool_cases(draw):
+    return (draw(st.integers(1, 4)), draw(st.integers(1, 9)), draw(st.integers(1, 11)),
+            draw(st.integers(1, 3)), draw(st.integers(1, 5)), draw(st.integers(1, 6)),
+            draw(st.integers(0, 2**31 - 1)))
+
+
+@settings(max_examples=80, derandomize=True, deadline=None)
+@given(pool_cases())
+def test_pool_equals_mean_over_latent_ranges(case):
+    """pool on random ragged geometries equals, for every block (tb, yb, xb), the mean of
+    the tokens at t in [tb bt, min(T, tb bt + bt)), y and x likewise, taken from the
+    latent grid."""
+    T, Hs, Ws, bt, bh, bw, seed = case
+    g = O.block_geometry(T, Hs, Ws, bt, bh, bw)
+    X = np.random.default_rng(seed).standard_normal((1, 2, T * Hs * Ws, 3))
+    got = O.pool(X, g)
+    grid = X.reshape(1, 2, T, Hs, Ws, 3)
+    nBt, nBy, nBx = -(-T // bt), -(-Hs // bh), -(-Ws // bw)
+    for tb in range(nBt):
+        for yb in range(nBy):
+            for xb in range(nBx):
+                j = (tb * nBy + yb) * nBx + xb
+                sub = grid[:, :, tb * bt:(tb + 1) * bt, yb * bh:(yb + 1) * bh, xb * bw:(xb + 1) * bw]
+                want = sub.reshape(1, 2, -1, 3).mean(axis=2)
+                np.testing.assert_allclose(got[:, :, j], want, rtol=0, atol=1e-13)
