@@ -142,11 +142,10 @@ FVATTN_API int fvattn_num_sms(void);
  *   out[n] = sum_{m in kept(i)} exp((q_n . k_m) * scale - lse[n]) v_m,
  * where m runs over the real tokens of the key blocks whose mask bit is set.
  *   q, k, v : bf16 [B][H][N][d]      (read)
- *   mask    : uint32 [B][H][nB][words], as written by fvattn_route: every row has
- *             at least one bit set (fvattn_route always sets bit i) and no bit at
- *             j >= nB (fvattn_route clears them).  The kernel checks neither on the
- *             device: a row with no bit set gives lse = -inf and unspecified out for
- *             its tokens, and a set bit at j >= nB is undefined behaviour.
+ *   mask    : uint32 [B][H][nB][words], as written by fvattn_route (bit j of a row:
+ *             key block j kept).  Bits at j >= nB are ignored.  A row with no bit set
+ *             (fvattn_route always sets bit i) gives out = 0 and lse = -inf for its
+ *             tokens.
  *   out     : bf16 [B][H][N][d]      (written, every token)
  *   lse     : fp32 [B][H][N]         (written, every token)
  *   workspace, ws_bytes : >= fvattn_attn_workspace_size(g) bytes, 16-byte aligned,
