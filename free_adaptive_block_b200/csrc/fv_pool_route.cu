@@ -718,10 +718,19 @@ static cudaError_t launch_pool_route_t(const Geo& g, const void* q, const void* 
   const int smem = 2 * kLogitTile * (D + 4) * 4;
   e = cudaFuncSetAttribute(pool_route_kernel<D, MAXW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  int per_sm = 0;
-  e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_route_kernel<D, MAXW>, kFusedThreads, smem);
+  // resident CTAs per SM, queried once per device (the first call, normally outside any
+  // stream capture) and reused
+  static int per_sm_of[64] = {};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  if (per_sm < 1) return cudaErrorInvalidConfiguration;
+  int per_sm = dev >= 0 && dev < 64 ? per_sm_of[dev] : 0;
+  if (per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_route_kernel<D, MAXW>, kFusedThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) per_sm_of[dev] = per_sm;
+  }
   const long long want = static_cast<long long>(nsm) * per_sm;
   const int grid = static_cast<int>(pl.total < want ? pl.total : want);
   uint32_t* hdr = static_cast<uint32_t*>(ws);
