@@ -313,6 +313,11 @@ def run_ours(args, rank, world, local_rank, wl=None):
                                                       buf.mask, buf.counts, buf.route_ws, stream))
     t_route1 = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
                                                     buf.mask, buf.counts, stream))
+    # the layer's pool and route: one persistent kernel when the mask row has <= 24 words
+    fused = buf.pool_route_ws is not None and g.words <= 24
+    t_pool_route = back_to_back(lambda: fv.fvattn_pool_route(g, q, k, wl.p, wl.k_floor, scale, buf.q_pool,
+                                                             buf.k_pool, buf.mask, buf.counts,
+                                                             buf.pool_route_ws, stream))
     # (inside a capture the calls must use the capturing stream: stream=None = current)
     attn_graph = graph_of(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
                                                               buf.workspace, buf.sm_busy_ns))
@@ -370,14 +375,14 @@ def run_ours(args, rank, world, local_rank, wl=None):
 
     # the library's kernels one layer step launches: pool; route (logits + select through
     # the route workspace, else the one-kernel route); prep_cost, prep_order, attention
-    launches_per_step = 1 + (2 if buf.route_ws is not None else 1) + 3
+    launches_per_step = (1 if fused else 1 + (2 if buf.route_ws is not None else 1)) + 3
     ms_step = total_ms / args.steps
     value = whole_job_tflops(eff, world, ms_step)
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
     # the roofline divides by the average duration of the same timed calls
     attn_tflops_avg = eff / (attn_ms_mean * 1e-3) / 1e12
     pr_bytes = MX.pool_route_bytes(wl.B, wl.H, wl.N, g.nB, wl.d, g.words)
-    pr_ms = t_pool + t_route
+    pr_ms = t_pool_route if buf.pool_route_ws is not None else t_pool + t_route
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -393,8 +398,11 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "attn_effective_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
+        "pool_route_ms": round(t_pool_route, 4),
+        "pool_route_kernel": "fused (one persistent kernel)" if fused else "pool + two-kernel route",
         "route_one_kernel_ms": round(t_route1, 4),
-        "stage_timing": "pool, route (fvattn_route_ws, the layer's route): device time per launch over 20 "
+        "stage_timing": "pool, route (fvattn_route_ws), pool_route (fvattn_pool_route, the layer's): device "
+                        "time per launch over 20 "
                         "back-to-back launches; attention: one captured call after L2 flush + pool + route "
                         "(attn_ms median, attn_ms_mean and roofline mean)",
         "layer_step": "CUDA graph of pool -> route -> attention (LayerGraph)" if args.graph else "direct calls",

@@ -26,7 +26,8 @@ from typing import Optional
 __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
-    "fvattn_route_workspace_size", "fvattn_route_ws",
+    "fvattn_route_workspace_size", "fvattn_route_ws", "fvattn_pool_route_workspace_size",
+    "fvattn_pool_route",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
     "LayerBuffers", "LayerGraph",
 ]
@@ -95,6 +96,11 @@ _SIGS = {
                                        ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fvattn_num_sms": (ctypes.c_int, []),
+    "fvattn_pool_route_workspace_size": (ctypes.c_size_t, [ctypes.c_void_p]),
+    "fvattn_pool_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                         ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p]),
     "fvattn_block_sparse_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -216,6 +222,27 @@ def fvattn_route_ws(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: 
         _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
 
 
+def fvattn_pool_route_workspace_size(g: Geometry) -> int:
+    cg = g.c()
+    return int(lib().fvattn_pool_route_workspace_size(ctypes.byref(cg)))
+
+
+def fvattn_pool_route(g: Geometry, q, k, p: float, k_floor: int, scale: float, q_pool, k_pool, mask,
+                      counts, workspace, stream=None) -> None:
+    """fvattn_block_pool then fvattn_route_ws, in one persistent kernel; same results."""
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_pool_route", lib().fvattn_pool_route(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        float(p), int(k_floor), float(scale), _ptr(q_pool, torch.float32, pooled, "q_pool"),
+        _ptr(k_pool, torch.float32, pooled, "k_pool"),
+        _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"),
+        _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
+
+
 def fvattn_attn_workspace_size(g: Geometry) -> int:
     cg = g.c()
     return int(lib().fvattn_attn_workspace_size(ctypes.byref(cg)))
@@ -292,6 +319,7 @@ class LayerBuffers:
     workspace: "object"
     sm_busy_ns: "object"
     route_ws: "object" = None   # workspace of fvattn_route_ws (None: the one-kernel route)
+    pool_route_ws: "object" = None   # workspace of fvattn_pool_route (used when present)
 
     @classmethod
     def allocate(cls, g: Geometry, device="cuda") -> "LayerBuffers":
@@ -305,7 +333,9 @@ class LayerBuffers:
                    lse=torch.empty(g.B, g.H, g.N, dtype=torch.float32, device=device),
                    workspace=ws,
                    sm_busy_ns=torch.zeros(max(1, fvattn_num_sms()), dtype=torch.int64, device=device),
-                   route_ws=torch.empty(fvattn_route_workspace_size(g), dtype=torch.uint8, device=device))
+                   route_ws=torch.empty(fvattn_route_workspace_size(g), dtype=torch.uint8, device=device),
+                   pool_route_ws=torch.empty(fvattn_pool_route_workspace_size(g), dtype=torch.uint8,
+                                             device=device))
 
 
 def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optional[float] = None,
@@ -315,11 +345,15 @@ def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optiona
     if scale is None:
         scale = 1.0 / math.sqrt(g.d)
     b = buffers if buffers is not None else LayerBuffers.allocate(g, q.device)
-    fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
-    if b.route_ws is not None:
-        fvattn_route_ws(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, b.route_ws, stream)
+    if b.pool_route_ws is not None:
+        fvattn_pool_route(g, q, k, p, k_floor, scale, b.q_pool, b.k_pool, b.mask, b.counts, b.pool_route_ws,
+                          stream)
     else:
-        fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
+        fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
+        if b.route_ws is not None:
+            fvattn_route_ws(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, b.route_ws, stream)
+        else:
+            fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
     fvattn_block_sparse_attn(g, q, k, v, b.mask, scale, b.out, b.lse, b.workspace, b.sm_busy_ns, stream)
     return b
 

@@ -79,6 +79,8 @@ fv.fvattn_route_ws = keep_all
 fv.fvattn_block_sparse_attn = lambda *a, **k: None
 fv.fvattn_dense_attn = lambda *a, **k: None
 fv.fvattn_device_status = lambda *a, **k: 0
+fv.fvattn_pool_route_workspace_size = lambda g: 1024
+fv.fvattn_pool_route = lambda g, q, k, p, kf, sc, qp, kp, mask, counts, ws, stream=None: mask.fill_(-1)
 
 
 class FakeLayerGraph:
