@@ -29,7 +29,7 @@ __all__ = [
     "fvattn_route_workspace_size", "fvattn_route_ws", "fvattn_pool_route_workspace_size",
     "fvattn_pool_route",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
-    "LayerBuffers", "LayerGraph",
+    "LayerBuffers", "LayerGraph", "HostPipeline",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -391,3 +391,96 @@ class LayerGraph:
         """Launches the captured layer on the current stream; returns its buffers."""
         self.graph.replay()
         return self.buffers
+
+
+class HostPipeline:
+    """One attention layer on inputs in (pinned) host memory, with the transfers overlapped
+    with the kernels.
+
+    The (b, h) slices run in ``chunks`` groups of consecutive slices.  A copy stream sends
+    every group's Q, K and V to the device in turn; the current stream runs pool, route and
+    attention on group c as soon as its inputs have arrived, while group c + 1 is still in
+    transit; a second copy stream brings group c's out and lse back while group c + 1
+    computes.  Pooling, routing and attention of a slice depend on that slice alone, so
+    the results equal one ``attention_layer`` call on the whole layer, bit for bit.
+
+    ``run`` is asynchronous on the current stream: the host inputs must stay unchanged, and
+    the host outputs are valid, once the current stream has passed the call (for instance
+    after ``torch.cuda.current_stream().synchronize()``)."""
+
+    def __init__(self, g: Geometry, p: float, k_floor: int, scale: Optional[float] = None,
+                 chunks: int = 4, device=None):
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.g = g
+        self.p, self.k_floor = float(p), int(k_floor)
+        self.scale = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+        S = g.B * g.H
+        n = max(1, min(int(chunks), S))
+        edges = [round(i * S / n) for i in range(n + 1)]
+        self.ranges = [(a, b) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+        tok = (g.B, g.H, g.N, g.d)
+        self.q = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        self.k = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        full = LayerBuffers.allocate(g, dev)
+        self.buffers = full
+        widest = max(b - a for a, b in self.ranges)
+        gw = dataclasses.replace(g, B=1, H=widest)
+        ws = torch.empty(fvattn_attn_workspace_size(gw), dtype=torch.uint8, device=dev)
+        rws = torch.empty(fvattn_route_workspace_size(gw), dtype=torch.uint8, device=dev)
+        self.workspace = ws
+
+        def rows(t, a, b):
+            # slices [a, b) of a [B][H][...] tensor as a [1][b - a][...] view
+            flat = t.reshape((S,) + tuple(t.shape[2:]))
+            return flat[a:b].reshape((1, b - a) + tuple(t.shape[2:]))
+
+        self._rows = rows
+        self.sub = []
+        for a, b in self.ranges:
+            gc = dataclasses.replace(g, B=1, H=b - a)
+            bc = LayerBuffers(q_pool=rows(full.q_pool, a, b), k_pool=rows(full.k_pool, a, b),
+                              mask=rows(full.mask, a, b), counts=rows(full.counts, a, b),
+                              out=rows(full.out, a, b), lse=rows(full.lse, a, b), workspace=ws,
+                              sm_busy_ns=full.sm_busy_ns, route_ws=rws)
+            self.sub.append((gc, bc, rows(self.q, a, b), rows(self.k, a, b), rows(self.v, a, b)))
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.ev_in = [torch.cuda.Event() for _ in self.ranges]
+        self.ev_done = [torch.cuda.Event() for _ in self.ranges]
+
+    def run(self, q_h, k_h, v_h, out_h, lse_h) -> LayerBuffers:
+        """q_h, k_h, v_h: bf16 [B][H][N][d] host tensors (pinned for overlap); out_h: bf16
+        [B][H][N][d] and lse_h: fp32 [B][H][N] host tensors that receive the results.
+        Returns the device buffers (mask, counts, pooled rows, out, lse)."""
+        import torch
+        g = self.g
+        tok = (g.B, g.H, g.N, g.d)
+        for t, name, dt, shape in ((q_h, "q", torch.bfloat16, tok), (k_h, "k", torch.bfloat16, tok),
+                                   (v_h, "v", torch.bfloat16, tok), (out_h, "out", torch.bfloat16, tok),
+                                   (lse_h, "lse", torch.float32, tok[:3])):
+            if t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous host tensor of {dt} and shape {shape}")
+        cur = torch.cuda.current_stream(self.q.device)
+        # the previous run's kernels read q, k, v and wrote out, lse: wait for them
+        self.s_in.wait_stream(cur)
+        self.s_out.wait_stream(cur)
+        with torch.cuda.stream(self.s_in):
+            for (a, b), (gc, bc, qd, kd, vd), ev in zip(self.ranges, self.sub, self.ev_in):
+                qd.copy_(self._rows(q_h, a, b), non_blocking=True)
+                kd.copy_(self._rows(k_h, a, b), non_blocking=True)
+                vd.copy_(self._rows(v_h, a, b), non_blocking=True)
+                ev.record(self.s_in)
+        for (a, b), (gc, bc, qd, kd, vd), e_in, e_done in zip(self.ranges, self.sub, self.ev_in, self.ev_done):
+            cur.wait_event(e_in)
+            attention_layer(gc, qd, kd, vd, self.p, self.k_floor, self.scale, bc, cur)
+            e_done.record(cur)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(e_done)
+                self._rows(out_h, a, b).copy_(bc.out, non_blocking=True)
+                self._rows(lse_h, a, b).copy_(bc.lse, non_blocking=True)
+        cur.wait_stream(self.s_out)
+        cur.wait_stream(self.s_in)
+        return self.buffers
+

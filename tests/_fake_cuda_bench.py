@@ -37,6 +37,9 @@ class FakeStream:
     def wait_stream(self, other):
         pass
 
+    def wait_event(self, event):
+        pass
+
 
 class FakeGraph:
     def replay(self):
@@ -53,6 +56,7 @@ def fake_device(*a, **k):
 
 
 torch.cuda.set_device = lambda d: None
+torch.cuda.current_device = lambda: 0
 torch.cuda.synchronize = lambda d=None: None
 torch.cuda.Event = FakeEvent
 torch.cuda.current_stream = lambda d=None: FakeStream()
