@@ -429,7 +429,9 @@ class HostPipeline:
         gw = dataclasses.replace(g, B=1, H=widest)
         ws = torch.empty(fvattn_attn_workspace_size(gw), dtype=torch.uint8, device=dev)
         rws = torch.empty(fvattn_route_workspace_size(gw), dtype=torch.uint8, device=dev)
+        prws = torch.empty(fvattn_pool_route_workspace_size(gw), dtype=torch.uint8, device=dev)
         self.workspace = ws
+        self.pool_route_ws = prws
 
         def rows(t, a, b):
             # slices [a, b) of a [B][H][...] tensor as a [1][b - a][...] view
@@ -443,7 +445,7 @@ class HostPipeline:
             bc = LayerBuffers(q_pool=rows(full.q_pool, a, b), k_pool=rows(full.k_pool, a, b),
                               mask=rows(full.mask, a, b), counts=rows(full.counts, a, b),
                               out=rows(full.out, a, b), lse=rows(full.lse, a, b), workspace=ws,
-                              sm_busy_ns=full.sm_busy_ns, route_ws=rws)
+                              sm_busy_ns=full.sm_busy_ns, route_ws=rws, pool_route_ws=prws)
             self.sub.append((gc, bc, rows(self.q, a, b), rows(self.k, a, b), rows(self.v, a, b)))
         self.s_in = torch.cuda.Stream(dev)
         self.s_out = torch.cuda.Stream(dev)

@@ -39,3 +39,4 @@ def test_pipeline_equals_layer(wl, chunks):
         assert torch.equal(b.mask.cpu(), want["mask"])
         assert torch.equal(b.counts.cpu(), want["counts"])
         assert fv.fvattn_device_status(pipe.workspace) == 0
+        assert fv.fvattn_device_status(pipe.pool_route_ws) == 0

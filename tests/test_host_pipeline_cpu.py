@@ -44,6 +44,7 @@ def cpu_cuda(monkeypatch):
     monkeypatch.setattr(torch.cuda, "stream", lambda s: contextlib.nullcontext())
     monkeypatch.setattr(fv, "fvattn_attn_workspace_size", lambda g: 64)
     monkeypatch.setattr(fv, "fvattn_route_workspace_size", lambda g: 64)
+    monkeypatch.setattr(fv, "fvattn_pool_route_workspace_size", lambda g: 64)
     monkeypatch.setattr(fv, "fvattn_num_sms", lambda: 4)
     monkeypatch.setattr(fv, "attention_layer", stand_in_layer)
 
