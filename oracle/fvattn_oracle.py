@@ -38,6 +38,7 @@ from __future__ import annotations
 
 import dataclasses
 import itertools
+from fractions import Fraction
 from typing import Dict, List, Optional, Sequence, Tuple
 
 import numpy as np
@@ -230,21 +231,26 @@ def brute_force_route_row(s_row: np.ndarray, own: int, p: float, k_floor: int) -
     """Exhaustive reference for one row (tiny nB only): the smallest cardinality c* of
     any subset with mass >= p (nB if none, or if p >= 1); then among all subsets of size
     max(c*, min(k, nB)) the one of largest mass, ties to the lexicographically smallest
-    index tuple; plus the own block."""
+    index tuple; plus the own block.  Subset masses are exact rational sums of the fp64
+    scores, so subsets of exactly equal mass tie and fall to the index rule, whatever
+    order a floating-point sum would take them in."""
     nB = s_row.shape[0]
     assert nB <= 12, "brute force is for tiny rows only"
+    exact = [Fraction(float(v)) for v in s_row]
+    mass_of = lambda S: sum((exact[j] for j in S), Fraction(0))   # noqa: E731
     if p >= 1.0:
         c_star = nB
     else:
+        target = Fraction(float(p))
         c_star = nB
         for c in range(1, nB + 1):
-            if any(sum(s_row[list(S)]) >= p for S in itertools.combinations(range(nB), c)):
+            if any(mass_of(S) >= target for S in itertools.combinations(range(nB), c)):
                 c_star = c
                 break
     m = max(c_star, min(int(k_floor), nB))
-    best, best_mass = None, -1.0
+    best, best_mass = None, Fraction(-1)
     for S in itertools.combinations(range(nB), m):      # lexicographic order
-        mass = float(sum(s_row[list(S)]))
+        mass = mass_of(S)
         if mass > best_mass:
             best, best_mass = S, mass
     keep = np.zeros(nB, dtype=bool)
