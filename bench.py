@@ -313,6 +313,11 @@ def run_ours(args, rank, world, local_rank, wl=None):
                                                       buf.mask, buf.counts, buf.route_ws, stream))
     t_route1 = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
                                                     buf.mask, buf.counts, stream))
+    # the layer's pool and route: one persistent kernel when the mask row has <= 24 words
+    fused = buf.pool_route_ws is not None and g.words <= 24
+    t_pool_route = back_to_back(lambda: fv.fvattn_pool_route(g, q, k, wl.p, wl.k_floor, scale, buf.q_pool,
+                                                             buf.k_pool, buf.mask, buf.counts,
+                                                             buf.pool_route_ws, stream))
     # (inside a capture the calls must use the capturing stream: stream=None = current)
     attn_graph = graph_of(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
                                                               buf.workspace, buf.sm_busy_ns))
@@ -342,42 +347,52 @@ def run_ours(args, rank, world, local_rank, wl=None):
                                                         None))
     dense_ms = statistics.median(per_call(dense_graph, min(args.steps, 10)))
 
-    # end to end through the public API with host buffers (pinned), copies timed: each
-    # step copies Q/K/V into the captured input buffers, replays the layer, reads
-    # out and lse back
+    # end to end through the public API with host buffers (pinned), copies timed.
+    # HostPipeline (the e2e figure): the slices in chunks, each chunk's copies in and out
+    # overlapped with the neighbouring chunks' kernels.  For comparison, the serial form:
+    # copy Q/K/V into the captured buffers, replay the layer, read out and lse back.
     pinned = {n: host[n].pin_memory() for n in ("q", "k", "v")}
     out_h = torch.empty(buf.out.shape, dtype=torch.bfloat16).pin_memory()
     lse_h = torch.empty(buf.lse.shape, dtype=torch.float32).pin_memory()
-    e2e_t = []
     n_e2e = min(args.steps, 5)
-    for i in range(2 + n_e2e):
-        a = torch.cuda.Event(enable_timing=True)
-        b = torch.cuda.Event(enable_timing=True)
-        a.record(stream)
+    pipe = fv.HostPipeline(g, wl.p, wl.k_floor, scale, chunks=args.e2e_chunks, device=dev)
+
+    def e2e_time(fn):
+        ts = []
+        for i in range(2 + n_e2e):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            a.record(stream)
+            fn()
+            b.record(stream)
+            torch.cuda.synchronize(dev)
+            if i >= 2:
+                ts.append(a.elapsed_time(b))
+        return max_over_ranks(statistics.mean(ts), world, dev)
+
+    def serial():
         q.copy_(pinned["q"], non_blocking=True)
         k.copy_(pinned["k"], non_blocking=True)
         v.copy_(pinned["v"], non_blocking=True)
         step()
         out_h.copy_(buf.out, non_blocking=True)
         lse_h.copy_(buf.lse, non_blocking=True)
-        b.record(stream)
-        torch.cuda.synchronize(dev)
-        if i >= 2:
-            e2e_t.append(a.elapsed_time(b))
-    e2e_ms = max_over_ranks(statistics.mean(e2e_t), world, dev)
+
+    e2e_ms = e2e_time(lambda: pipe.run(pinned["q"], pinned["k"], pinned["v"], out_h, lse_h))
+    e2e_serial_ms = e2e_time(serial)
     h2d = sum(pinned[n].numel() * 2 for n in ("q", "k", "v"))
     d2h = out_h.numel() * 2 + lse_h.numel() * 4
 
     # the library's kernels one layer step launches: pool; route (logits + select through
     # the route workspace, else the one-kernel route); prep_cost, prep_order, attention
-    launches_per_step = 1 + (2 if buf.route_ws is not None else 1) + 3
+    launches_per_step = (1 if fused else 1 + (2 if buf.route_ws is not None else 1)) + 3
     ms_step = total_ms / args.steps
     value = whole_job_tflops(eff, world, ms_step)
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
     # the roofline divides by the average duration of the same timed calls
     attn_tflops_avg = eff / (attn_ms_mean * 1e-3) / 1e12
     pr_bytes = MX.pool_route_bytes(wl.B, wl.H, wl.N, g.nB, wl.d, g.words)
-    pr_ms = t_pool + t_route
+    pr_ms = t_pool_route if buf.pool_route_ws is not None else t_pool + t_route
     line = {
         "metric": METRIC, "value": round(value, 3), "unit": UNIT, "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(ms_step, 4),
@@ -393,8 +408,11 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "attn_effective_tflops": round(attn_tflops, 2),
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
+        "pool_route_ms": round(t_pool_route, 4),
+        "pool_route_kernel": "fused (one persistent kernel)" if fused else "pool + two-kernel route",
         "route_one_kernel_ms": round(t_route1, 4),
-        "stage_timing": "pool, route (fvattn_route_ws, the layer's route): device time per launch over 20 "
+        "stage_timing": "pool, route (fvattn_route_ws), pool_route (fvattn_pool_route, the layer's): device "
+                        "time per launch over 20 "
                         "back-to-back launches; attention: one captured call after L2 flush + pool + route "
                         "(attn_ms median, attn_ms_mean and roofline mean)",
         "layer_step": "CUDA graph of pool -> route -> attention (LayerGraph)" if args.graph else "direct calls",
@@ -412,8 +430,10 @@ def run_ours(args, rank, world, local_rank, wl=None):
                      "duration": f"mean of {len(attn_ts)} event-timed calls, {attn_ms_mean:.4f} ms",
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
         "e2e": {"value": round(whole_job_tflops(eff, world, e2e_ms), 3), "unit": UNIT,
-                "how": "pinned host Q/K/V -> device, layer step, out/lse -> pinned host, one stream",
-                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h},
+                "how": f"HostPipeline: pinned host Q/K/V -> device -> out/lse -> pinned host in "
+                       f"{len(pipe.ranges)} chunks of slices, copies overlapped with the kernels",
+                "ms_per_step": round(e2e_ms, 3), "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "serial_ms_per_step": round(e2e_serial_ms, 3)},
         "gpu_launches": launches_per_step * args.steps,
         "clocks": clocks,
     }
@@ -554,6 +574,8 @@ def main():
                     help="after the 480p line, one line per other workload (tiny, 720p, 6x horizon)")
     ap.add_argument("--no-graph", dest="graph", action="store_false",
                     help="time the layer as three direct calls instead of a captured CUDA graph")
+    ap.add_argument("--e2e-chunks", type=int, default=4,
+                    help="chunks of (b, h) slices in the end-to-end leg (HostPipeline)")
     ap.add_argument("--layer-only", action="store_true",
                     help="time the layer steps only (no dense, e2e or CPU legs); for profilers")
     args = ap.parse_args()

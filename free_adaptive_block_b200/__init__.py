@@ -26,9 +26,10 @@ from typing import Optional
 __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
-    "fvattn_route_workspace_size", "fvattn_route_ws",
+    "fvattn_route_workspace_size", "fvattn_route_ws", "fvattn_pool_route_workspace_size",
+    "fvattn_pool_route",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
-    "LayerBuffers", "LayerGraph",
+    "LayerBuffers", "LayerGraph", "HostPipeline",
 ]
 
 _HERE = os.path.dirname(os.path.abspath(__file__))
@@ -95,6 +96,11 @@ _SIGS = {
                                        ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
                                        ctypes.c_void_p, ctypes.c_size_t, ctypes.c_void_p]),
     "fvattn_num_sms": (ctypes.c_int, []),
+    "fvattn_pool_route_workspace_size": (ctypes.c_size_t, [ctypes.c_void_p]),
+    "fvattn_pool_route": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                         ctypes.c_int, ctypes.c_float, ctypes.c_void_p, ctypes.c_void_p,
+                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                         ctypes.c_void_p]),
     "fvattn_block_sparse_attn": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -216,6 +222,27 @@ def fvattn_route_ws(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: 
         _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
 
 
+def fvattn_pool_route_workspace_size(g: Geometry) -> int:
+    cg = g.c()
+    return int(lib().fvattn_pool_route_workspace_size(ctypes.byref(cg)))
+
+
+def fvattn_pool_route(g: Geometry, q, k, p: float, k_floor: int, scale: float, q_pool, k_pool, mask,
+                      counts, workspace, stream=None) -> None:
+    """fvattn_block_pool then fvattn_route_ws, in one persistent kernel; same results."""
+    import torch
+    tok = (g.B, g.H, g.N, g.d)
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_pool_route", lib().fvattn_pool_route(
+        ctypes.byref(cg), _ptr(q, torch.bfloat16, tok, "q"), _ptr(k, torch.bfloat16, tok, "k"),
+        float(p), int(k_floor), float(scale), _ptr(q_pool, torch.float32, pooled, "q_pool"),
+        _ptr(k_pool, torch.float32, pooled, "k_pool"),
+        _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"),
+        _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
+
+
 def fvattn_attn_workspace_size(g: Geometry) -> int:
     cg = g.c()
     return int(lib().fvattn_attn_workspace_size(ctypes.byref(cg)))
@@ -292,6 +319,7 @@ class LayerBuffers:
     workspace: "object"
     sm_busy_ns: "object"
     route_ws: "object" = None   # workspace of fvattn_route_ws (None: the one-kernel route)
+    pool_route_ws: "object" = None   # workspace of fvattn_pool_route (used when present)
 
     @classmethod
     def allocate(cls, g: Geometry, device="cuda") -> "LayerBuffers":
@@ -305,7 +333,9 @@ class LayerBuffers:
                    lse=torch.empty(g.B, g.H, g.N, dtype=torch.float32, device=device),
                    workspace=ws,
                    sm_busy_ns=torch.zeros(max(1, fvattn_num_sms()), dtype=torch.int64, device=device),
-                   route_ws=torch.empty(fvattn_route_workspace_size(g), dtype=torch.uint8, device=device))
+                   route_ws=torch.empty(fvattn_route_workspace_size(g), dtype=torch.uint8, device=device),
+                   pool_route_ws=torch.empty(fvattn_pool_route_workspace_size(g), dtype=torch.uint8,
+                                             device=device))
 
 
 def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optional[float] = None,
@@ -315,11 +345,15 @@ def attention_layer(g: Geometry, q, k, v, p: float, k_floor: int, scale: Optiona
     if scale is None:
         scale = 1.0 / math.sqrt(g.d)
     b = buffers if buffers is not None else LayerBuffers.allocate(g, q.device)
-    fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
-    if b.route_ws is not None:
-        fvattn_route_ws(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, b.route_ws, stream)
+    if b.pool_route_ws is not None:
+        fvattn_pool_route(g, q, k, p, k_floor, scale, b.q_pool, b.k_pool, b.mask, b.counts, b.pool_route_ws,
+                          stream)
     else:
-        fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
+        fvattn_block_pool(g, q, k, b.q_pool, b.k_pool, stream)
+        if b.route_ws is not None:
+            fvattn_route_ws(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, b.route_ws, stream)
+        else:
+            fvattn_route(g, b.q_pool, b.k_pool, p, k_floor, scale, b.mask, b.counts, stream)
     fvattn_block_sparse_attn(g, q, k, v, b.mask, scale, b.out, b.lse, b.workspace, b.sm_busy_ns, stream)
     return b
 
@@ -357,3 +391,98 @@ class LayerGraph:
         """Launches the captured layer on the current stream; returns its buffers."""
         self.graph.replay()
         return self.buffers
+
+
+class HostPipeline:
+    """One attention layer on inputs in (pinned) host memory, with the transfers overlapped
+    with the kernels.
+
+    The (b, h) slices run in ``chunks`` groups of consecutive slices.  A copy stream sends
+    every group's Q, K and V to the device in turn; the current stream runs pool, route and
+    attention on group c as soon as its inputs have arrived, while group c + 1 is still in
+    transit; a second copy stream brings group c's out and lse back while group c + 1
+    computes.  Pooling, routing and attention of a slice depend on that slice alone, so
+    the results equal one ``attention_layer`` call on the whole layer, bit for bit.
+
+    ``run`` is asynchronous on the current stream: the host inputs must stay unchanged, and
+    the host outputs are valid, once the current stream has passed the call (for instance
+    after ``torch.cuda.current_stream().synchronize()``)."""
+
+    def __init__(self, g: Geometry, p: float, k_floor: int, scale: Optional[float] = None,
+                 chunks: int = 4, device=None):
+        import torch
+        dev = torch.device("cuda", torch.cuda.current_device()) if device is None else torch.device(device)
+        self.g = g
+        self.p, self.k_floor = float(p), int(k_floor)
+        self.scale = 1.0 / math.sqrt(g.d) if scale is None else float(scale)
+        S = g.B * g.H
+        n = max(1, min(int(chunks), S))
+        edges = [round(i * S / n) for i in range(n + 1)]
+        self.ranges = [(a, b) for a, b in zip(edges[:-1], edges[1:]) if b > a]
+        tok = (g.B, g.H, g.N, g.d)
+        self.q = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        self.k = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        self.v = torch.empty(tok, dtype=torch.bfloat16, device=dev)
+        full = LayerBuffers.allocate(g, dev)
+        self.buffers = full
+        widest = max(b - a for a, b in self.ranges)
+        gw = dataclasses.replace(g, B=1, H=widest)
+        ws = torch.empty(fvattn_attn_workspace_size(gw), dtype=torch.uint8, device=dev)
+        rws = torch.empty(fvattn_route_workspace_size(gw), dtype=torch.uint8, device=dev)
+        prws = torch.empty(fvattn_pool_route_workspace_size(gw), dtype=torch.uint8, device=dev)
+        self.workspace = ws
+        self.pool_route_ws = prws
+
+        def rows(t, a, b):
+            # slices [a, b) of a [B][H][...] tensor as a [1][b - a][...] view
+            flat = t.reshape((S,) + tuple(t.shape[2:]))
+            return flat[a:b].reshape((1, b - a) + tuple(t.shape[2:]))
+
+        self._rows = rows
+        self.sub = []
+        for a, b in self.ranges:
+            gc = dataclasses.replace(g, B=1, H=b - a)
+            bc = LayerBuffers(q_pool=rows(full.q_pool, a, b), k_pool=rows(full.k_pool, a, b),
+                              mask=rows(full.mask, a, b), counts=rows(full.counts, a, b),
+                              out=rows(full.out, a, b), lse=rows(full.lse, a, b), workspace=ws,
+                              sm_busy_ns=full.sm_busy_ns, route_ws=rws, pool_route_ws=prws)
+            self.sub.append((gc, bc, rows(self.q, a, b), rows(self.k, a, b), rows(self.v, a, b)))
+        self.s_in = torch.cuda.Stream(dev)
+        self.s_out = torch.cuda.Stream(dev)
+        self.ev_in = [torch.cuda.Event() for _ in self.ranges]
+        self.ev_done = [torch.cuda.Event() for _ in self.ranges]
+
+    def run(self, q_h, k_h, v_h, out_h, lse_h) -> LayerBuffers:
+        """q_h, k_h, v_h: bf16 [B][H][N][d] host tensors (pinned for overlap); out_h: bf16
+        [B][H][N][d] and lse_h: fp32 [B][H][N] host tensors that receive the results.
+        Returns the device buffers (mask, counts, pooled rows, out, lse)."""
+        import torch
+        g = self.g
+        tok = (g.B, g.H, g.N, g.d)
+        for t, name, dt, shape in ((q_h, "q", torch.bfloat16, tok), (k_h, "k", torch.bfloat16, tok),
+                                   (v_h, "v", torch.bfloat16, tok), (out_h, "out", torch.bfloat16, tok),
+                                   (lse_h, "lse", torch.float32, tok[:3])):
+            if t.is_cuda or t.dtype != dt or tuple(t.shape) != shape or not t.is_contiguous():
+                raise ValueError(f"{name} must be a contiguous host tensor of {dt} and shape {shape}")
+        cur = torch.cuda.current_stream(self.q.device)
+        # the previous run's kernels read q, k, v and wrote out, lse: wait for them
+        self.s_in.wait_stream(cur)
+        self.s_out.wait_stream(cur)
+        with torch.cuda.stream(self.s_in):
+            for (a, b), (gc, bc, qd, kd, vd), ev in zip(self.ranges, self.sub, self.ev_in):
+                qd.copy_(self._rows(q_h, a, b), non_blocking=True)
+                kd.copy_(self._rows(k_h, a, b), non_blocking=True)
+                vd.copy_(self._rows(v_h, a, b), non_blocking=True)
+                ev.record(self.s_in)
+        for (a, b), (gc, bc, qd, kd, vd), e_in, e_done in zip(self.ranges, self.sub, self.ev_in, self.ev_done):
+            cur.wait_event(e_in)
+            attention_layer(gc, qd, kd, vd, self.p, self.k_floor, self.scale, bc, cur)
+            e_done.record(cur)
+            with torch.cuda.stream(self.s_out):
+                self.s_out.wait_event(e_done)
+                self._rows(out_h, a, b).copy_(bc.out, non_blocking=True)
+                self._rows(lse_h, a, b).copy_(bc.lse, non_blocking=True)
+        cur.wait_stream(self.s_out)
+        cur.wait_stream(self.s_in)
+        return self.buffers
+

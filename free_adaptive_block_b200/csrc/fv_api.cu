@@ -223,6 +223,35 @@ fvattn_status_t fvattn_route_ws(const fvattn_geom_t* gi, const float* q_pool, co
                                          reinterpret_cast<cudaStream_t>(stream)));
 }
 
+size_t fvattn_pool_route_workspace_size(const fvattn_geom_t* gi) {
+  Geo g;
+  if (make_geo(gi, &g) != FVATTN_OK) return 0;
+  return fv::pool_route_ws_bytes(g);
+}
+
+fvattn_status_t fvattn_pool_route(const fvattn_geom_t* gi, const void* q, const void* k, float p,
+                                  int k_floor, float scale, float* q_pool, float* k_pool, uint32_t* mask,
+                                  int32_t* counts, void* workspace, size_t ws_bytes,
+                                  fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr(q));
+  FV_CHECK(check_ptr(k));
+  FV_CHECK(check_ptr(q_pool));
+  FV_CHECK(check_ptr(k_pool));
+  FV_CHECK(check_ptr(mask));
+  FV_CHECK(check_ptr(counts));
+  if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
+  if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < fv::pool_route_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FVATTN_ERR_UNSUPPORTED;
+  const int nsm = current_num_sms();
+  if (nsm <= 0) return cuda_status(cudaGetLastError() == cudaSuccess ? cudaErrorNoDevice : cudaGetLastError());
+  return cuda_status(fv::launch_pool_route(g, q, k, q_pool, k_pool, p, k_floor, scale, mask, counts, workspace,
+                                           nsm, reinterpret_cast<cudaStream_t>(stream)));
+}
+
 size_t fvattn_attn_workspace_size(const fvattn_geom_t* gi) {
   Geo g;
   if (make_geo(gi, &g) != FVATTN_OK) return 0;

@@ -318,6 +318,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         // blocks; the members' own mask rows go to gmask for the softmax warps
         const int gcnt = q_group_cnt(g, tile - (tile / g.nB) * g.nB, prm.qg);
         const int tail = g.nB & 31;
+        // bits of the last word at or past nB: cleared, so that no id past the last block
+        // reaches the list (fvattn_route never sets them; a caller's mask might)
+        const uint32_t last = tail ? (1u << tail) - 1u : 0xffffffffu;
         uint32_t w0 = 0u, w1 = 0u;
 #pragma unroll 1
         for (int s4 = 0; s4 < 4; ++s4) {
@@ -326,9 +329,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             const int w = lane + 32 * h;
             uint32_t m = 0u;
             if (s4 < gcnt && w < g.words) {
-              m = prm.mask != nullptr
-                      ? __ldg(prm.mask + static_cast<size_t>(tile + s4 * g.nBx) * g.words + w)
-                      : (w < g.words - 1 ? 0xffffffffu : (tail ? (1u << tail) - 1u : 0xffffffffu));
+              m = (prm.mask != nullptr ? __ldg(prm.mask + static_cast<size_t>(tile + s4 * g.nBx) * g.words + w)
+                                       : 0xffffffffu) &
+                  (w < g.words - 1 ? 0xffffffffu : last);
             }
             bars.gmask[slot][s4][w] = m;
             if (h == 0) w0 |= m; else w1 |= m;
@@ -797,6 +800,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.xread[quarter]);
       ++xn;
+      // a row whose kept set is empty (possible only with a caller's mask that keeps no
+      // block for it) has lt = 0: its out is written as zeros and its lse is -inf
+      const bool empty = !(lt > 0.f);
       const float inv = 1.f / lt;
       tc_fence_after();
       uint4* dst = reinterpret_cast<uint4*>(prm.out + (static_cast<size_t>(bhi) * g.N + (token >= 0 ? token : 0)) * D +
@@ -814,6 +820,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
             wv.y = pack_bf16x2(__uint_as_float(o[8 * q8 + 2]) * inv, __uint_as_float(o[8 * q8 + 3]) * inv);
             wv.z = pack_bf16x2(__uint_as_float(o[8 * q8 + 4]) * inv, __uint_as_float(o[8 * q8 + 5]) * inv);
             wv.w = pack_bf16x2(__uint_as_float(o[8 * q8 + 6]) * inv, __uint_as_float(o[8 * q8 + 7]) * inv);
+            if (empty) wv = make_uint4(0u, 0u, 0u, 0u);   // the tensor memory may hold stale values
             dst[4 * q + q8] = wv;
           }
         }
@@ -920,10 +927,12 @@ __global__ void __launch_bounds__(32 * kCostWarps) prep_cost_kernel(Geo g, const
     }
     const int gcnt = q_group_cnt(g, qb, qg);
     const uint32_t* row = mask + static_cast<size_t>(tile) * g.words;
+    const int tail = g.nB & 31;
     int cost = 0;
     for (int w = lane; w < g.words; w += 32) {
       uint32_t m = 0u;
       for (int s4 = 0; s4 < gcnt; ++s4) m |= __ldg(row + static_cast<size_t>(s4) * g.nBx * g.words + w);
+      if (w == g.words - 1 && tail) m &= (1u << tail) - 1u;   // no block at or past nB
       const uint32_t ex = edge[0][w], ey = edge[1][w], et = edge[2][w];
 #pragma unroll
       for (int k = 0; k < 8; ++k) {

@@ -26,6 +26,13 @@ size_t route_ws_bytes(const Geo& g);
 cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
                             float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st);
 
+// Pool and route in one persistent kernel; ws holds pool_route_ws_bytes(g) bytes (a
+// header with the item queue, the error word and per-slice counters, then the logits).
+size_t pool_route_ws_bytes(const Geo& g);
+cudaError_t launch_pool_route(const Geo& g, const void* q, const void* k, float* qp, float* kp, float p,
+                              int k_floor, float scale, uint32_t* mask, int32_t* counts, void* ws, int nsm,
+                              cudaStream_t st);
+
 struct AttnMaps {
   CUtensorMap q, qe, k, ke, v, ve;   // full-width and x-edge boxes of Q, K, V
 };

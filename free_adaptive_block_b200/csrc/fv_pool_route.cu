@@ -11,6 +11,7 @@
 
 #include "fv_common.cuh"
 #include "fv_launch.h"
+#include "fv_plan.h"
 
 namespace fv {
 
@@ -24,21 +25,17 @@ namespace fv {
 // ----------------------------------------------------------------------------
 constexpr int kPoolThreads = 256;
 
+// One pooling item: block j of slice bhi of one tensor (src -> dst).  `red` is the
+// CTA's [8][D] reduction buffer; the caller separates items with a block barrier.
 template <int D>
-__global__ void __launch_bounds__(kPoolThreads, 4) pool_kernel(Geo g, const uint4* __restrict__ q,
-                                                               const uint4* __restrict__ k,
-                                                               float* __restrict__ qp,
-                                                               float* __restrict__ kp) {
+__device__ __forceinline__ void pool_item(const Geo& g, const uint4* __restrict__ src,
+                                          float* __restrict__ dst, int j, int bhi,
+                                          float (*red)[D]) {
   constexpr int CH = D / 8;                // 16-byte chunks per token
   constexpr int TPI = 32 / CH;             // tokens a warp covers per load instruction
   constexpr int NW = kPoolThreads / 32;
   constexpr int BATCH = 8;                 // loads in flight per lane
-  __shared__ float red[NW][D];
 
-  const int j = blockIdx.x;
-  const int bhi = blockIdx.y;
-  const uint4* __restrict__ src = blockIdx.z ? k : q;
-  float* __restrict__ dst = blockIdx.z ? kp : qp;
   const BlockInfo bi = block_info(g, j);
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int ch = lane % CH, tsub = lane / CH;
@@ -88,6 +85,15 @@ __global__ void __launch_bounds__(kPoolThreads, 4) pool_kernel(Geo g, const uint
     for (int w = 0; w < NW; ++w) sum += red[w][t];
     dst[(static_cast<size_t>(bhi) * g.nB + j) * D + t] = sum * inv;
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(kPoolThreads, 4) pool_kernel(Geo g, const uint4* __restrict__ q,
+                                                               const uint4* __restrict__ k,
+                                                               float* __restrict__ qp,
+                                                               float* __restrict__ kp) {
+  __shared__ float red[kPoolThreads / 32][D];
+  pool_item<D>(g, blockIdx.z ? k : q, blockIdx.z ? kp : qp, blockIdx.x, blockIdx.y, red);
 }
 
 cudaError_t launch_pool(const Geo& g, const void* q, const void* k, float* qp, float* kp,
@@ -428,28 +434,31 @@ cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p
 // kernel's (two partial sums over the even and odd components of each float4 of d, in
 // ascending d, added at the end, times scale), so both paths give the same mask.
 // ----------------------------------------------------------------------------
-constexpr int kLogitTile = 64;         // query x key blocks per CTA
 
-template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restrict__ qp,
-                                                     const float* __restrict__ kp, float scale,
-                                                     float* __restrict__ logits) {
+// One 64 x 64 tile of logits: query blocks [64 qt, +64) against key blocks [64 kt, +64)
+// of slice bhi.  sQ and sK are [64][D + 4] floats of shared memory each.  kL2 reads the
+// pooled rows from L2 only (ld.global.cg): set when they were written earlier in the
+// same kernel, by other CTAs.
+// kSplit loads each float4 step's (x, y) operands, runs their 16 products, then the
+// (z, w) ones: every accumulator sees the same operations in the same order as without
+// it, with half the operand registers live (for the fused kernel's register budget).
+template <int D, bool kL2, bool kSplit>
+__device__ __forceinline__ void logits_tile(const Geo& g, const float* __restrict__ qp,
+                                            const float* __restrict__ kp, float scale,
+                                            float* __restrict__ logits, int qt, int kt, int bhi,
+                                            float* sQ, float* sK) {
   constexpr int RS = D + 4;            // padded row (floats)
-  extern __shared__ __align__(16) unsigned char lg_smem[];
-  float* sQ = reinterpret_cast<float*>(lg_smem);   // [64][D + 4]
-  float* sK = sQ + kLogitTile * RS;                // [64][D + 4]
   const int nB = g.nB, nBpad = g.words * 32;
-  const int bhi = blockIdx.z;
-  const int q0 = blockIdx.x * kLogitTile, k0 = blockIdx.y * kLogitTile;
+  const int q0 = qt * kLogitTile, k0 = kt * kLogitTile;
   const float* qh = qp + static_cast<size_t>(bhi) * nB * D;
   const float* kh = kp + static_cast<size_t>(bhi) * nB * D;
   for (int e = threadIdx.x; e < kLogitTile * D / 4; e += 256) {
     const int r = e / (D / 4), d4 = e - r * (D / 4);
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    reinterpret_cast<float4*>(sQ + r * RS)[d4] =
-        q0 + r < nB ? reinterpret_cast<const float4*>(qh + static_cast<size_t>(q0 + r) * D)[d4] : z;
-    reinterpret_cast<float4*>(sK + r * RS)[d4] =
-        k0 + r < nB ? reinterpret_cast<const float4*>(kh + static_cast<size_t>(k0 + r) * D)[d4] : z;
+    const float4* qs = reinterpret_cast<const float4*>(qh + static_cast<size_t>(q0 + r) * D) + d4;
+    const float4* ks = reinterpret_cast<const float4*>(kh + static_cast<size_t>(k0 + r) * D) + d4;
+    reinterpret_cast<float4*>(sQ + r * RS)[d4] = q0 + r < nB ? (kL2 ? __ldcg(qs) : *qs) : z;
+    reinterpret_cast<float4*>(sK + r * RS)[d4] = k0 + r < nB ? (kL2 ? __ldcg(ks) : *ks) : z;
   }
   __syncthreads();
   // thread (ty, tx) takes query rows ty + 16 i and key blocks tx + 16 j, i, j < 4
@@ -459,25 +468,46 @@ __global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restr
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
-#pragma unroll 4
-  for (int d4 = 0; d4 < D / 4; ++d4) {
-    uint64_t qxy[4], qzw[4], kxy[4], kzw[4];
+  if constexpr (kSplit) {
+#pragma unroll 2
+    for (int d4 = 0; d4 < D / 4; ++d4) {
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float4 x = reinterpret_cast<const float4*>(sQ + (ty + 16 * i) * RS)[d4];
-      qxy[i] = f32x2(x.x, x.y);
-      qzw[i] = f32x2(x.z, x.w);
-      const float4 k4 = reinterpret_cast<const float4*>(sK + (tx + 16 * i) * RS)[d4];
-      kxy[i] = f32x2(k4.x, k4.y);
-      kzw[i] = f32x2(k4.z, k4.w);
-    }
+      for (int h = 0; h < 2; ++h) {    // h = 0: (x, y) components, h = 1: (z, w)
+        uint64_t qv[4], kv[4];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+        for (int i = 0; i < 4; ++i) {
+          const float2 x = reinterpret_cast<const float2*>(sQ + (ty + 16 * i) * RS)[2 * d4 + h];
+          qv[i] = f32x2(x.x, x.y);
+          const float2 k2 = reinterpret_cast<const float2*>(sK + (tx + 16 * i) * RS)[2 * d4 + h];
+          kv[i] = f32x2(k2.x, k2.y);
+        }
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        acc[i][j] = ffma2(qxy[i], kxy[j], acc[i][j]);   // a0 += x.x k.x, a1 += x.y k.y
-        acc[i][j] = ffma2(qzw[i], kzw[j], acc[i][j]);   // a0 += x.z k.z, a1 += x.w k.w
+        for (int i = 0; i < 4; ++i)
+#pragma unroll
+          for (int j = 0; j < 4; ++j) acc[i][j] = ffma2(qv[i], kv[j], acc[i][j]);
       }
+    }
+  } else {
+#pragma unroll 4
+    for (int d4 = 0; d4 < D / 4; ++d4) {
+      uint64_t qxy[4], qzw[4], kxy[4], kzw[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float4 x = reinterpret_cast<const float4*>(sQ + (ty + 16 * i) * RS)[d4];
+        qxy[i] = f32x2(x.x, x.y);
+        qzw[i] = f32x2(x.z, x.w);
+        const float4 k4 = reinterpret_cast<const float4*>(sK + (tx + 16 * i) * RS)[d4];
+        kxy[i] = f32x2(k4.x, k4.y);
+        kzw[i] = f32x2(k4.z, k4.w);
+      }
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          acc[i][j] = ffma2(qxy[i], kxy[j], acc[i][j]);   // a0 += x.x k.x, a1 += x.y k.y
+          acc[i][j] = ffma2(qzw[i], kzw[j], acc[i][j]);   // a0 += x.z k.z, a1 += x.w k.w
+        }
+    }
   }
   float* out = logits + static_cast<size_t>(bhi) * nB * nBpad;
 #pragma unroll
@@ -493,6 +523,16 @@ __global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restr
       out[static_cast<size_t>(qr) * nBpad + kc] = (a0 + a1) * scale;
     }
   }
+}
+
+template <int D>
+__global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restrict__ qp,
+                                                     const float* __restrict__ kp, float scale,
+                                                     float* __restrict__ logits) {
+  extern __shared__ __align__(16) unsigned char lg_smem[];
+  float* sQ = reinterpret_cast<float*>(lg_smem);   // [64][D + 4]
+  float* sK = sQ + kLogitTile * (D + 4);           // [64][D + 4]
+  logits_tile<D, false, false>(g, qp, kp, scale, logits, blockIdx.x, blockIdx.y, blockIdx.z, sQ, sK);
 }
 
 template <int MAXW>
@@ -548,6 +588,188 @@ cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, floa
   float* logits = static_cast<float*>(ws);
   return g.d == 128 ? launch_route2_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st)
                     : launch_route2_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+}
+
+// ----------------------------------------------------------------------------
+// Pool and route in one persistent kernel (fvattn_pool_route).  Pooling streams Q and K
+// from HBM and leaves most instruction-issue slots idle; the route is bound by issue and
+// reads only the pooled rows and logits, which stay in L2.  So the route of one (b, h)
+// slice runs while later slices are still being pooled.  One queue holds three kinds of
+// item, one CTA per item at a time:
+//   pool      block j of slice s of Q or K                 (2 nB per slice)
+//   logits    a 64 x 64 tile of slice s's logits           (tiles^2 per slice)
+//   select    8 query blocks of slice s: Top-p / Top-k     (ceil(nB / 8) per slice)
+// in steps: step i holds pool(i), then logits(i - 1), then select(i - 2), for the
+// slices that exist.  A logits item waits for all pool items of its slice, a select item
+// for all logits items of its slice (counters in the workspace header).  Every item
+// waited on comes earlier in the queue, where a running CTA took it, so every wait ends;
+// waits are bounded all the same, and on a timeout the select items write a mask that
+// keeps every block.
+// ----------------------------------------------------------------------------
+constexpr int kFusedThreads = 256;
+constexpr int kFusedMaxWords = 24;     // larger rows run the separate pool and route kernels
+constexpr size_t kPrHeader = 256;      // queue counter, error bits; then 2 counters per slice
+
+size_t pool_route_ws_bytes(const Geo& g) {
+  const size_t S = static_cast<size_t>(g.B) * g.H;
+  const size_t head = ((kPrHeader + 8 * S) + 255) / 256 * 256;
+  return head + route_ws_bytes(g);
+}
+
+// Thread 0 waits until *cnt >= need: acquire loads, bounded by a clock64 deadline (2 s at
+// up to 2 GHz) and by the error word (another item already gave up).  False on either.
+__device__ __forceinline__ bool pr_wait(const uint32_t* cnt, uint32_t need, uint32_t* err) {
+  long long t0 = clock64();
+  for (uint32_t i = 0;; ++i) {
+    uint32_t v;
+    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
+    if (v >= need) return true;
+    if ((i & 15u) == 15u) {
+      if (*reinterpret_cast<volatile uint32_t*>(err) & kErrTimeout) return false;
+      if (static_cast<uint64_t>(clock64() - t0) > 4000000000ull) {
+        atomicOr(err, kErrTimeout);
+        return false;
+      }
+    }
+    __nanosleep(128);
+  }
+}
+
+// Every thread's writes of the item, then one count for the slice.
+__device__ __forceinline__ void pr_done(uint32_t* cnt) {
+  __threadfence();
+  __syncthreads();
+  if (threadIdx.x == 0) atomicAdd(cnt, 1u);
+}
+
+template <int D, int MAXW>
+__global__ void __launch_bounds__(kFusedThreads, 3) pool_route_kernel(
+    Geo g, const uint4* __restrict__ q, const uint4* __restrict__ k, float* qp, float* kp, float p,
+    int k_floor, float scale, uint32_t* __restrict__ mask, int32_t* __restrict__ counts,
+    uint32_t* hdr, float* logits) {
+  extern __shared__ __align__(16) unsigned char pr_smem[];
+  float* sQ = reinterpret_cast<float*>(pr_smem);    // [64][D + 4]; select rows reuse it
+  float* sK = sQ + kLogitTile * (D + 4);            // [64][D + 4]
+  __shared__ float red[kPoolThreads / 32][D];
+  __shared__ long long s_item;
+  __shared__ int s_ok;
+  uint32_t* err = hdr + 1;
+  const int nB = g.nB, nBpad = g.words * 32;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  for (;;) {
+    if (threadIdx.x == 0) s_item = static_cast<long long>(atomicAdd(reinterpret_cast<unsigned long long*>(hdr + 2), 1ull));
+    __syncthreads();
+    const long long t = s_item;
+    __syncthreads();   // s_item is rewritten by the next iteration
+    // the plan is recomputed per item (a few integer operations) rather than held in
+    // registers across the loop
+    const PrPlan pl = pr_plan(g.B * g.H, nB);
+    if (t >= pl.total) break;
+    uint32_t* cnt_pool = hdr + kPrHeader / 4;
+    uint32_t* cnt_logit = cnt_pool + pl.S;
+    int kind, slice, idx;
+    pr_decode(pl, t, kind, slice, idx);
+    if (kind == 0) {
+      const int tensor = idx >= nB ? 1 : 0;
+      const int j = idx - tensor * nB;
+      pool_item<D>(g, tensor ? k : q, tensor ? kp : qp, j, slice, red);
+      pr_done(cnt_pool + slice);
+    } else if (kind == 1) {
+      if (threadIdx.x == 0) s_ok = pr_wait(cnt_pool + slice, static_cast<uint32_t>(pl.nP), err) ? 1 : 0;
+      __syncthreads();
+      if (s_ok) {
+        logits_tile<D, true, true>(g, qp, kp, scale, logits, idx / pl.tiles, idx - (idx / pl.tiles) * pl.tiles,
+                             slice, sQ, sK);
+        pr_done(cnt_logit + slice);
+      }
+    } else {
+      if (threadIdx.x == 0) s_ok = pr_wait(cnt_logit + slice, static_cast<uint32_t>(pl.nL), err) ? 1 : 0;
+      __syncthreads();
+      const int qb = idx * 8 + warp;
+      const size_t row = static_cast<size_t>(slice) * nB + qb;
+      if (qb < nB) {
+        uint32_t* mrow = mask + row * g.words;
+        if (s_ok) {
+          float* sL = sQ + warp * nBpad;
+          const float* lrow = logits + row * nBpad;
+          for (int c = lane; c < nBpad; c += 32) sL[c] = c < nB ? __ldcg(lrow + c) : 0.f;
+          __syncwarp();
+          select_row<MAXW>(sL, nB, g.words, qb, p, k_floor, mrow, counts + row, lane);
+        } else {
+          // the logits never arrived: keep every block, a mask the attention accepts
+          const int tail = nB & 31;
+          for (int w = lane; w < g.words; w += 32)
+            mrow[w] = (w < g.words - 1 || tail == 0) ? 0xffffffffu : (1u << tail) - 1u;
+          if (lane == 0) counts[row] = nB;
+        }
+      }
+    }
+  }
+}
+
+template <int D, int MAXW>
+static cudaError_t launch_pool_route_t(const Geo& g, const void* q, const void* k, float* qp, float* kp,
+                                       float p, int k_floor, float scale, uint32_t* mask, int32_t* counts,
+                                       void* ws, int nsm, cudaStream_t st) {
+  const PrPlan pl = pr_plan(g.B * g.H, g.nB);
+  const size_t head = pool_route_ws_bytes(g) - route_ws_bytes(g);
+  cudaError_t e = cudaMemsetAsync(ws, 0, head, st);
+  if (e != cudaSuccess) return e;
+  const int smem = 2 * kLogitTile * (D + 4) * 4;
+  e = cudaFuncSetAttribute(pool_route_kernel<D, MAXW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  if (e != cudaSuccess) return e;
+  // resident CTAs per SM, queried once per device (the first call, normally outside any
+  // stream capture) and reused
+  static int per_sm_of[64] = {};
+  int dev = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  int per_sm = dev >= 0 && dev < 64 ? per_sm_of[dev] : 0;
+  if (per_sm == 0) {
+    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_route_kernel<D, MAXW>, kFusedThreads, smem);
+    if (e != cudaSuccess) return e;
+    if (per_sm < 1) return cudaErrorInvalidConfiguration;
+    if (dev >= 0 && dev < 64) per_sm_of[dev] = per_sm;
+  }
+  const long long want = static_cast<long long>(nsm) * per_sm;
+  const int grid = static_cast<int>(pl.total < want ? pl.total : want);
+  uint32_t* hdr = static_cast<uint32_t*>(ws);
+  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + head);
+  pool_route_kernel<D, MAXW><<<grid, kFusedThreads, smem, st>>>(
+      g, static_cast<const uint4*>(q), static_cast<const uint4*>(k), qp, kp, p, k_floor, scale, mask, counts,
+      hdr, logits);
+  return cudaGetLastError();
+}
+
+template <int D>
+static cudaError_t launch_pool_route_d(const Geo& g, const void* q, const void* k, float* qp, float* kp,
+                                       float p, int k_floor, float scale, uint32_t* mask, int32_t* counts,
+                                       void* ws, int nsm, cudaStream_t st) {
+  // MAXW sizes without register spills at three CTAs per SM (20 and, at d = 64, 4 spill);
+  // empty slots of a row hold zero keys and add exact zeros, so the mask does not depend
+  // on MAXW
+  if (g.words <= 8) return launch_pool_route_t<D, 8>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
+  if (g.words <= 12) return launch_pool_route_t<D, 12>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
+  if (g.words <= 16) return launch_pool_route_t<D, 16>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
+  return launch_pool_route_t<D, 24>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
+}
+
+cudaError_t launch_pool_route(const Geo& g, const void* q, const void* k, float* qp, float* kp, float p,
+                              int k_floor, float scale, uint32_t* mask, int32_t* counts, void* ws, int nsm,
+                              cudaStream_t st) {
+  if (g.words > kFusedMaxWords) {
+    // rows of more than 768 blocks: the separate kernels (the fused one would need more
+    // registers per thread than three CTAs per SM leave)
+    const size_t head = pool_route_ws_bytes(g) - route_ws_bytes(g);
+    cudaError_t e = cudaMemsetAsync(ws, 0, head, st);   // clean error word for device_status
+    if (e != cudaSuccess) return e;
+    e = launch_pool(g, q, k, qp, kp, st);
+    if (e != cudaSuccess) return e;
+    return launch_route_ws(g, qp, kp, p, k_floor, scale, mask, counts,
+                           static_cast<unsigned char*>(ws) + head, st);
+  }
+  return g.d == 128 ? launch_pool_route_d<128>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st)
+                    : launch_pool_route_d<64>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
 }
 
 }  // namespace fv

@@ -127,6 +127,33 @@ FVATTN_API fvattn_status_t fvattn_route_ws(const fvattn_geom_t* g, const float* 
                                            int32_t* counts, void* workspace, size_t ws_bytes,
                                            fvattn_stream_t stream);
 
+/* Bytes of device workspace fvattn_pool_route needs: a header (an item queue, an error
+ * word and two counters per (b, h) slice, B * H * 8 bytes plus 256, rounded up to 256)
+ * followed by the logits of fvattn_route_ws (fvattn_route_workspace_size bytes).  0 for
+ * an invalid geometry. */
+FVATTN_API size_t fvattn_pool_route_workspace_size(const fvattn_geom_t* g);
+
+/* fvattn_block_pool followed by fvattn_route_ws, in one persistent kernel (FVAttn
+ * explainer 核心方法 §1: pooled 3D blocks, then Top-p with a Top-k floor and the own
+ * block).  Same definitions, outputs and argument domains as those two calls, and the
+ * same results bit for bit: q_pool, k_pool, mask and counts equal what the two calls
+ * write.  Pooling streams Q and K from HBM; the route of a (b, h) slice runs on the
+ * same SMs while later slices are still being pooled.  When a mask row has more than
+ * 24 words (nB > 768) the call runs the two separate calls' kernels instead.
+ *   q, k              : bf16 [B][H][N][d]           (read)
+ *   q_pool, k_pool    : fp32 [B][H][nB][d]          (written)
+ *   mask, counts      : as fvattn_route             (written)
+ *   workspace, ws_bytes : >= fvattn_pool_route_workspace_size(g) bytes, 16-byte aligned,
+ *                       owned by the caller, contents on entry do not matter; not to be
+ *                       shared by calls that run concurrently.
+ * Its kernel waits, bounded, for its own earlier work items; if a wait gives up, the
+ * rows it could not route keep every block and fvattn_device_status(workspace) reports
+ * FVATTN_ERR_DEVICE_TIMEOUT. */
+FVATTN_API fvattn_status_t fvattn_pool_route(const fvattn_geom_t* g, const void* q, const void* k, float p,
+                                             int k_floor, float scale, float* q_pool, float* k_pool,
+                                             uint32_t* mask, int32_t* counts, void* workspace,
+                                             size_t ws_bytes, fvattn_stream_t stream);
+
 /* Bytes of device workspace fvattn_block_sparse_attn / fvattn_dense_attn need
  * for geometry g (a tile queue and a status word).  0 for a malformed geometry. */
 FVATTN_API size_t fvattn_attn_workspace_size(const fvattn_geom_t* g);
@@ -142,11 +169,10 @@ FVATTN_API int fvattn_num_sms(void);
  *   out[n] = sum_{m in kept(i)} exp((q_n . k_m) * scale - lse[n]) v_m,
  * where m runs over the real tokens of the key blocks whose mask bit is set.
  *   q, k, v : bf16 [B][H][N][d]      (read)
- *   mask    : uint32 [B][H][nB][words], as written by fvattn_route: every row has
- *             at least one bit set (fvattn_route always sets bit i) and no bit at
- *             j >= nB (fvattn_route clears them).  The kernel checks neither on the
- *             device: a row with no bit set gives lse = -inf and unspecified out for
- *             its tokens, and a set bit at j >= nB is undefined behaviour.
+ *   mask    : uint32 [B][H][nB][words], as written by fvattn_route (bit j of a row:
+ *             key block j kept).  Bits at j >= nB are ignored.  A row with no bit set
+ *             (fvattn_route always sets bit i) gives out = 0 and lse = -inf for its
+ *             tokens.
  *   out     : bf16 [B][H][N][d]      (written, every token)
  *   lse     : fp32 [B][H][N]         (written, every token)
  *   workspace, ws_bytes : >= fvattn_attn_workspace_size(g) bytes, 16-byte aligned,
@@ -197,8 +223,8 @@ FVATTN_API fvattn_status_t fvattn_dense_attn(const fvattn_geom_t* g, const void*
                                   void* workspace, size_t ws_bytes,
                                   unsigned long long* sm_busy_ns, fvattn_stream_t stream);
 
-/* Synchronises `stream` and reports whether the last attention call that used
- * `workspace` ran cleanly: FVATTN_OK, FVATTN_ERR_DEVICE_TIMEOUT (a kernel gave up a
+/* Synchronises `stream` and reports whether the last attention or fvattn_pool_route
+ * call that used `workspace` ran cleanly: FVATTN_OK, FVATTN_ERR_DEVICE_TIMEOUT (a kernel gave up a
  * bounded wait), FVATTN_ERR_DEVICE (a kernel found its shared memory misaligned and
  * did no work), or FVATTN_ERR_CUDA if the synchronisation failed. */
 FVATTN_API fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream);

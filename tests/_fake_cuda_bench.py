@@ -37,6 +37,9 @@ class FakeStream:
     def wait_stream(self, other):
         pass
 
+    def wait_event(self, event):
+        pass
+
 
 class FakeGraph:
     def replay(self):
@@ -53,6 +56,7 @@ def fake_device(*a, **k):
 
 
 torch.cuda.set_device = lambda d: None
+torch.cuda.current_device = lambda: 0
 torch.cuda.synchronize = lambda d=None: None
 torch.cuda.Event = FakeEvent
 torch.cuda.current_stream = lambda d=None: FakeStream()
@@ -79,6 +83,8 @@ fv.fvattn_route_ws = keep_all
 fv.fvattn_block_sparse_attn = lambda *a, **k: None
 fv.fvattn_dense_attn = lambda *a, **k: None
 fv.fvattn_device_status = lambda *a, **k: 0
+fv.fvattn_pool_route_workspace_size = lambda g: 1024
+fv.fvattn_pool_route = lambda g, q, k, p, kf, sc, qp, kp, mask, counts, ws, stream=None: mask.fill_(-1)
 
 
 class FakeLayerGraph:

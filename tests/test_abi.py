@@ -92,6 +92,18 @@ def test_host_side_argument_checks(L):
     assert L.fvattn_route_ws(*args, 0x10008, need, None) == E["FVATTN_ERR_UNSUPPORTED"]
     assert L.fvattn_route_ws(ctypes.byref(cg), 0x1000, 0x2000, -1.0, 4, 0.088, 0x3000, 0x4000,
                              0x10000, need, None) == E["FVATTN_ERR_INVALID_ARG"]
+    # pool and route in one call: a header of queue, error word and two counters per
+    # slice, then the same logits
+    need_pr = fv.fvattn_pool_route_workspace_size(G480)
+    assert need_pr == -(-(256 + 8 * 12) // 256) * 256 + need
+    pr = lambda p=0.9, kf=4, qp=0x5000, ws=0x10000, n=need_pr: L.fvattn_pool_route(
+        ctypes.byref(cg), 0x1000, 0x2000, p, kf, 0.088, qp, 0x6000, 0x3000, 0x4000, ws, n, None)
+    assert pr(qp=None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert pr(p=float("nan")) == E["FVATTN_ERR_INVALID_ARG"]
+    assert pr(kf=-2) == E["FVATTN_ERR_INVALID_ARG"]
+    assert pr(ws=None) == E["FVATTN_ERR_WORKSPACE"]
+    assert pr(n=need_pr - 1) == E["FVATTN_ERR_WORKSPACE"]
+    assert pr(ws=0x10008) == E["FVATTN_ERR_UNSUPPORTED"]
 
 
 def test_status_strings(L):
