@@ -155,35 +155,76 @@ def unpack_mask(words: np.ndarray, nB: int) -> np.ndarray:
     return bits.reshape(words.shape[:-1] + (words.shape[-1] * 32,))[..., :nB].astype(bool)
 
 
+def keep_for_cut(r: RouteResult, m: np.ndarray) -> np.ndarray:
+    """The keep matrix for prefix lengths m [B,H,nB] (instead of r.m_keep): the first m
+    key blocks of each row's order, plus the query's own block."""
+    nB = r.order.shape[-1]
+    rank = np.empty_like(r.order)
+    np.put_along_axis(rank, r.order, np.broadcast_to(np.arange(nB), r.order.shape), axis=-1)
+    keep = rank < m[..., None]
+    own = np.arange(nB)
+    keep[..., own, own] = True
+    return keep
+
+
+def band_for_cut(r: RouteResult, m: np.ndarray, band: float = 1e-5) -> np.ndarray:
+    """Key blocks whose kept/dropped state rounding may flip when the prefix has length m.
+
+    The cutoff is the score c of the m-th block in the order.  Blocks whose score lies
+    within `band` of c can change places in an fp32 order, but that changes the kept set
+    only when they sit on both sides of the cut; so a row's near-cutoff blocks are
+    excluded when some of them are inside the prefix and some outside, and none are
+    excluded otherwise.  The own block is kept either way and is never excluded."""
+    nB = r.order.shape[-1]
+    s_sorted = np.take_along_axis(r.scores, r.order, axis=-1)
+    cutoff = np.take_along_axis(s_sorted, (np.maximum(m, 1) - 1)[..., None], axis=-1)
+    near = np.abs(r.scores - cutoff) < band
+    rank = np.empty_like(r.order)
+    np.put_along_axis(rank, r.order, np.broadcast_to(np.arange(nB), r.order.shape), axis=-1)
+    inside = rank < m[..., None]
+    straddles = (near & inside).any(-1) & (near & ~inside).any(-1)
+    excluded = near & straddles[..., None]
+    own = np.arange(nB)
+    excluded[..., own, own] = False
+    return excluded
+
+
+def candidate_cuts(r: RouteResult, p: float, k_floor: int, band: float = 1e-5) -> np.ndarray:
+    """Prefix lengths an fp32 implementation may legitimately reach, per row: int
+    [B,H,nB,3] holding m_keep and, where a cumulative sum next to the Top-p cut lies
+    within `band` of p, the prefix length after the floor with the cut moved one block
+    later (the sum at m_p may round below p) or one block earlier (the sum at m_p - 1
+    may round up to p); m_keep again where no such sum is near p."""
+    B, H, nB, _ = r.scores.shape
+    out = np.repeat(r.m_keep[..., None], 3, axis=-1)
+    if p < 1.0:
+        floor = min(int(k_floor), nB)
+        cs, m_p = r.csum, r.m_p
+        near_at = np.abs(np.take_along_axis(cs, (m_p - 1)[..., None], -1)[..., 0] - p) < band
+        prev = np.take_along_axis(cs, np.maximum(m_p - 2, 0)[..., None], -1)[..., 0]
+        near_prev = (m_p >= 2) & (np.abs(prev - p) < band)
+        alt_up = np.maximum(np.minimum(m_p + 1, nB), floor)
+        alt_dn = np.maximum(np.maximum(m_p - 1, 1), floor)
+        out[..., 1] = np.where(near_at, alt_up, r.m_keep)
+        out[..., 2] = np.where(near_prev, alt_dn, r.m_keep)
+    return out
+
+
 def comparison_band(r: RouteResult, p: float, k_floor: int, band: float = 1e-5
                     ) -> Tuple[np.ndarray, np.ndarray]:
     """Where a GPU mask computed in fp32 may legitimately differ from this fp64 one.
 
     Returns (excluded [B,H,nB,nB] bool, ambiguous [B,H,nB] bool):
     * excluded: key blocks whose score lies within `band` of the cutoff score (the
-      score of the last block of the kept prefix); the own block is never excluded;
+      score of the last block of the kept prefix, after the floor), in rows where such
+      blocks lie on both sides of the cut (:func:`band_for_cut`); the own block is
+      never excluded;
     * ambiguous: rows where a cumulative sum next to the Top-p cut lies within `band`
       of p, so that rounding can move the cut by one block and change the prefix
-      length after the floor.  Such rows are checked only for the invariants."""
-    B, H, nB, _ = r.scores.shape
-    s_sorted = np.take_along_axis(r.scores, r.order, axis=-1)
-    idx = (r.m_keep - 1)[..., None]
-    cutoff = np.take_along_axis(s_sorted, idx, axis=-1)
-    excluded = np.abs(r.scores - cutoff) < band
-    own = np.arange(nB)
-    excluded[..., own, own] = False
-    amb = np.zeros((B, H, nB), dtype=bool)
-    if p < 1.0:
-        floor = min(int(k_floor), nB)
-        cs = r.csum
-        m_p = r.m_p
-        near_at = np.abs(np.take_along_axis(cs, (m_p - 1)[..., None], -1)[..., 0] - p) < band
-        prev = np.take_along_axis(cs, np.maximum(m_p - 2, 0)[..., None], -1)[..., 0]
-        near_prev = (m_p >= 2) & (np.abs(prev - p) < band)
-        # with rounding the cut may move to m_p + 1 (near_at) or m_p - 1 (near_prev)
-        alt_up = np.maximum(np.minimum(m_p + 1, nB), floor)
-        alt_dn = np.maximum(np.maximum(m_p - 1, 1), floor)
-        amb = (near_at & (alt_up != r.m_keep)) | (near_prev & (alt_dn != r.m_keep))
+      length after the floor (:func:`candidate_cuts`).  Such rows are compared with
+      the keep set of each candidate cut."""
+    excluded = band_for_cut(r, r.m_keep, band)
+    amb = (candidate_cuts(r, p, k_floor, band) != r.m_keep[..., None]).any(-1)
     return excluded, amb
 
 

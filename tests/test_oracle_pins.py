@@ -266,3 +266,86 @@ def test_comparison_band_flags_rows_near_p():
     r2 = O.route(Qp, np.eye(3)[None, None], 0.6, 1, 1.0)
     ex2, amb2 = O.comparison_band(r2, 0.6, 1)
     assert not amb2.any()
+
+
+def _route_one(scores, p, k):
+    """Every row of a hand-made routing problem has the given scores (Kp = identity, Qp
+    rows = ln(scores)); row i differs only in its own block, i."""
+    s = np.asarray(scores, dtype=np.float64)
+    nB = s.size
+    Qp = np.tile(np.log(s), (nB, 1))[None, None]
+    r = O.route(Qp, np.eye(nB)[None, None], p, k, 1.0)
+    np.testing.assert_allclose(r.scores[0, 0, 0], s / s.sum(), rtol=1e-12)
+    return r
+
+
+# Scores (hand-made, summing to 1):  block 2 is the Top-p cutoff at p = 0.75 (prefix
+# 0.5 + 0.2 + 0.1 = 0.8 >= 0.75, two blocks give 0.7); block 3 lies 0.5e-5 below the
+# cutoff, block 4 lies 2e-5 below it.
+_BAND_ROW = [0.5, 0.2, 0.1, 0.099995, 0.09998, 0.000025]
+
+
+def test_comparison_band_excludes_only_near_cutoff_blocks_across_the_cut():
+    r = _route_one(_BAND_ROW, 0.75, 1)
+    assert r.m_keep[0, 0].tolist() == [3] * 6
+    ex, amb = O.comparison_band(r, 0.75, 1)
+    assert not amb.any()
+    # own block 5 (outside the prefix): blocks 2 and 3 may swap places; 4 (2e-5 away) may not
+    assert np.nonzero(ex[0, 0, 5])[0].tolist() == [2, 3]
+    # own block 3: it is kept either way, so it is not excluded; block 2 still is
+    assert np.nonzero(ex[0, 0, 3])[0].tolist() == [2]
+    # own block 2 (the cutoff block itself): only block 3 can flip
+    assert np.nonzero(ex[0, 0, 2])[0].tolist() == [3]
+    # a plain row with no near-cutoff block on the far side excludes nothing
+    r2 = _route_one([0.5, 0.2, 0.1, 0.09, 0.08, 0.03], 0.75, 1)
+    assert not O.comparison_band(r2, 0.75, 1)[0].any()
+
+
+def test_comparison_band_cutoff_is_taken_after_the_floor():
+    # p = 0.5 keeps one block (0.6); the floor k = 4 lengthens the prefix to block 3
+    # (0.05), and block 4 lies 4e-6 below it: the band sits at block 3, not at block 0.
+    row = [0.6, 0.2, 0.1, 0.05, 0.049996, 0.000004]
+    r = _route_one(row, 0.5, 4)
+    assert r.m_p[0, 0, 0] == 1 and r.m_keep[0, 0, 0] == 4
+    ex, amb = O.comparison_band(r, 0.5, 4)
+    assert np.nonzero(ex[0, 0, 5])[0].tolist() == [3, 4]
+    assert not ex[0, 0, 5, :3].any()
+    # with the floor at 5 the cut moves past block 4: nothing near it lies outside
+    r5 = _route_one(row, 0.5, 5)
+    assert not O.comparison_band(r5, 0.5, 5)[0].any()
+    # when the floor keeps every block no bit can flip
+    r6 = _route_one(row, 0.5, 6)
+    assert r6.keep.all() and not O.comparison_band(r6, 0.5, 6)[0].any()
+
+
+def test_candidate_cuts_and_keep_for_cut():
+    # cumulative masses 0.5, 0.8, 1.0: at p = 0.8 the second sum sits on p, so an fp32
+    # sum may need one more block (cut 3) -- and the floor takes precedence over both
+    s = [0.5, 0.3, 0.2]
+    r = _route_one(s, 0.8, 1)
+    m_p = int(r.m_p[0, 0, 0])
+    cands = O.candidate_cuts(r, 0.8, 1)
+    assert sorted(set(cands[0, 0, 0].tolist())) in ([1, 2], [2, 3])
+    assert m_p in cands[0, 0, 0]
+    assert O.comparison_band(r, 0.8, 1)[1].all()
+    r_fl = _route_one(s, 0.8, 3)
+    assert (O.candidate_cuts(r_fl, 0.8, 3) == 3).all()
+    assert not O.comparison_band(r_fl, 0.8, 3)[1].any()
+    # a floor two blocks past m_p: moving the Top-p cut by one changes nothing
+    s4 = [0.5, 0.3, 0.1, 0.1]
+    for pp in (0.8 - 1e-7, 0.8 + 1e-7):      # the sum at the cut just above / below p
+        r4 = _route_one(s4, pp, 4)
+        assert (O.candidate_cuts(r4, pp, 4) == 4).all()
+        assert not O.comparison_band(r4, pp, 4)[1].any()
+        # without the floor the other side of the cut is a candidate: cut 2 moves up to
+        # 3 (sum at the cut just above p), or cut 3 down to 2 (just below)
+        r1 = _route_one(s4, pp, 1)
+        assert r1.m_p[0, 0, 0] == (2 if pp < 0.8 else 3)
+        assert sorted(set(O.candidate_cuts(r1, pp, 1)[0, 0, 0].tolist())) == [2, 3]
+    # far from p: every candidate is m_keep
+    r2 = _route_one(s, 0.6, 1)
+    assert (O.candidate_cuts(r2, 0.6, 1) == r2.m_keep[..., None]).all()
+    # keep_for_cut: prefix of the order plus the own block
+    keep = O.keep_for_cut(r2, np.full((1, 1, 3), 1))
+    assert keep[0, 0].astype(int).tolist() == [[1, 0, 0], [1, 1, 0], [1, 0, 1]]
+    assert (O.keep_for_cut(r2, r2.m_keep) == r2.keep).all()
