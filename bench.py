@@ -313,8 +313,8 @@ def run_ours(args, rank, world, local_rank, wl=None):
                                                       buf.mask, buf.counts, buf.route_ws, stream))
     t_route1 = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
                                                     buf.mask, buf.counts, stream))
-    # the layer's pool and route: one persistent kernel when the mask row has <= 24 words
-    fused = buf.pool_route_ws is not None and g.words <= 24
+    # the layer's pool and route (fvattn_pool_route: pool, tensor-core logits, selection)
+    fused = buf.pool_route_ws is not None
     t_pool_route = back_to_back(lambda: fv.fvattn_pool_route(g, q, k, wl.p, wl.k_floor, scale, buf.q_pool,
                                                              buf.k_pool, buf.mask, buf.counts,
                                                              buf.pool_route_ws, stream))
@@ -385,7 +385,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
 
     # the library's kernels one layer step launches: pool; route (logits + select through
     # the route workspace, else the one-kernel route); prep_cost, prep_order, attention
-    launches_per_step = (1 if fused else 1 + (2 if buf.route_ws is not None else 1)) + 3
+    launches_per_step = 1 + (2 if (fused or buf.route_ws is not None) else 1) + 3
     ms_step = total_ms / args.steps
     value = whole_job_tflops(eff, world, ms_step)
     attn_tflops = eff / (attn_ms * 1e-3) / 1e12
@@ -409,7 +409,8 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
         "pool_route_ms": round(t_pool_route, 4),
-        "pool_route_kernel": "fused (one persistent kernel)" if fused else "pool + two-kernel route",
+        "pool_route_kernel": ("fvattn_pool_route: pool, tensor-core logits, histogram selection" if fused
+                              else "pool + two-kernel route"),
         "route_one_kernel_ms": round(t_route1, 4),
         "stage_timing": "pool, route (fvattn_route_ws), pool_route (fvattn_pool_route, the layer's): device "
                         "time per launch over 20 "

@@ -27,8 +27,8 @@ __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
     "fvattn_route_workspace_size", "fvattn_route_ws", "fvattn_pool_route_workspace_size",
-    "fvattn_pool_route",
-    "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_device_status", "fvattn_status_string", "attention_layer",
+    "fvattn_pool_route", "RouteOpts", "fvattn_route_ex", "fvattn_mask_repair",
+    "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_noalloc_device_status", "fvattn_device_status", "fvattn_status_string", "attention_layer",
     "LayerBuffers", "LayerGraph", "HostPipeline",
 ]
 
@@ -52,6 +52,14 @@ class FvattnError(RuntimeError):
 
 class _CGeom(ctypes.Structure):
     _fields_ = [(n, ctypes.c_int) for n in ("B", "H", "T", "Hs", "Ws", "d", "bt", "bh", "bw")]
+
+
+class RouteOpts(ctypes.Structure):
+    """fvattn_route_opts_t: Top-p mass, floor and scale, plus the optional frontend steps
+    (token-level Top-p masses, keyframe blocks, runtime mask repair)."""
+    _fields_ = [("p", ctypes.c_float), ("k_floor", ctypes.c_int), ("scale", ctypes.c_float),
+                ("token_mass", ctypes.c_int), ("kf_stride", ctypes.c_int), ("kf_phase", ctypes.c_int),
+                ("repair", ctypes.c_int)]
 
 
 @dataclasses.dataclass(frozen=True)
@@ -114,6 +122,16 @@ _SIGS = {
                                                         ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                         ctypes.c_void_p]),
     "fvattn_device_status": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p]),
+    "fvattn_noalloc_device_status": (ctypes.c_int, [ctypes.c_void_p]),
+    "fvattn_route_ex": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                       ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t,
+                                       ctypes.c_void_p]),
+    "fvattn_mask_repair": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                          ctypes.c_void_p]),
+    "fvattn_testing_attn_stall": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
+                                                 ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                                 ctypes.c_size_t, ctypes.c_ulonglong, ctypes.c_void_p]),
     "fvattn_status_string": (ctypes.c_char_p, [ctypes.c_int]),
     "fvattn_last_cuda_error": (ctypes.c_char_p, []),
 }
@@ -222,6 +240,31 @@ def fvattn_route_ws(g: Geometry, q_pool, k_pool, p: float, k_floor: int, scale: 
         _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
 
 
+def fvattn_route_ex(g: Geometry, q_pool, k_pool, opts: RouteOpts, mask, counts, workspace,
+                    stream=None) -> None:
+    """fvattn_route_ws with the options of ``RouteOpts`` (token-level Top-p, keyframes,
+    mask repair)."""
+    import torch
+    pooled = (g.B, g.H, g.nB, g.d)
+    cg = g.c()
+    _ok("fvattn_route_ex", lib().fvattn_route_ex(
+        ctypes.byref(cg), _ptr(q_pool, torch.float32, pooled, "q_pool"),
+        _ptr(k_pool, torch.float32, pooled, "k_pool"), ctypes.byref(opts),
+        _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"),
+        _ptr(workspace, torch.uint8, None, "workspace"), workspace.numel(), _stream(stream)))
+
+
+def fvattn_mask_repair(g: Geometry, mask_in, mask_out, counts, stream=None) -> None:
+    """Runtime mask repair: one-block holes of every row filled (mask_out may be mask_in)."""
+    import torch
+    shape = (g.B, g.H, g.nB, g.words)
+    cg = g.c()
+    _ok("fvattn_mask_repair", lib().fvattn_mask_repair(
+        ctypes.byref(cg), _ptr(mask_in, torch.int32, shape, "mask_in"), _ptr(mask_out, torch.int32, shape, "mask_out"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"), _stream(stream)))
+
+
 def fvattn_pool_route_workspace_size(g: Geometry) -> int:
     cg = g.c()
     return int(lib().fvattn_pool_route_workspace_size(ctypes.byref(cg)))
@@ -229,7 +272,7 @@ def fvattn_pool_route_workspace_size(g: Geometry) -> int:
 
 def fvattn_pool_route(g: Geometry, q, k, p: float, k_floor: int, scale: float, q_pool, k_pool, mask,
                       counts, workspace, stream=None) -> None:
-    """fvattn_block_pool then fvattn_route_ws, in one persistent kernel; same results."""
+    """fvattn_block_pool then fvattn_route_ws in one call (the same kernels); same results."""
     import torch
     tok = (g.B, g.H, g.N, g.d)
     pooled = (g.B, g.H, g.nB, g.d)
@@ -299,6 +342,11 @@ def fvattn_block_sparse_attn_noalloc(g: Geometry, q, k, v, mask, scale: float, o
         _ptr(v, torch.bfloat16, tok, "v"), _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
         float(scale), _ptr(out, torch.bfloat16, tok, "out"), _ptr(lse, torch.float32, tok[:3], "lse"),
         _ptr(sm_busy_ns, torch.int64, None, "sm_busy_ns"), _stream(stream)))
+
+
+def fvattn_noalloc_device_status(stream=None) -> int:
+    """Status of the last fvattn_block_sparse_attn_noalloc call on the current device."""
+    return int(lib().fvattn_noalloc_device_status(_stream(stream)))
 
 
 def fvattn_device_status(workspace, stream=None) -> int:

@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfvattn.so")
-SOURCES = ["fv_api.cu", "fv_pool_route.cu", "fv_attn.cu"]
+SOURCES = ["fv_api.cu", "fv_pool_route.cu", "fv_route_tc.cu", "fv_attn.cu"]
 
 
 def nvcc() -> str:
@@ -20,7 +20,7 @@ def nvcc() -> str:
 def build(verbose: bool = False, extra: list | None = None) -> str:
     srcs = [os.path.join(CSRC, s) for s in SOURCES]
     deps = srcs + [os.path.join(CSRC, h) for h in os.listdir(CSRC) if h.endswith((".cuh", ".h"))]
-    deps.append(os.path.join(ROOT, "include", "fvattn.h"))
+    deps += [os.path.join(ROOT, "include", h) for h in os.listdir(os.path.join(ROOT, "include"))]
     if os.path.exists(LIB) and not extra and all(os.path.getmtime(LIB) >= os.path.getmtime(d) for d in deps):
         return LIB
     cmd = [nvcc(), "-gencode", "arch=compute_100a,code=sm_100a", "-O3", "-lineinfo", "-std=c++17",

@@ -8,6 +8,7 @@
 
 #include "fv_launch.h"
 #include "fvattn.h"
+#include "fvattn_testing.h"
 
 namespace {
 
@@ -55,6 +56,13 @@ fvattn_status_t make_geo(const fvattn_geom_t* gi, Geo* g) {
 fvattn_status_t check_ptr(const void* p) {
   if (p == nullptr) return FVATTN_ERR_INVALID_ARG;
   if (reinterpret_cast<uintptr_t>(p) & 15u) return FVATTN_ERR_UNSUPPORTED;
+  return FVATTN_OK;
+}
+
+// mask, counts and lse are read and written one 32-bit word at a time
+fvattn_status_t check_ptr4(const void* p) {
+  if (p == nullptr) return FVATTN_ERR_INVALID_ARG;
+  if (reinterpret_cast<uintptr_t>(p) & 3u) return FVATTN_ERR_UNSUPPORTED;
   return FVATTN_OK;
 }
 
@@ -107,15 +115,16 @@ int current_num_sms() {
 
 fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, const void* v,
                          const uint32_t* mask, float scale, void* out, float* lse, void* ws,
-                         size_t ws_bytes, unsigned long long* busy, fvattn_stream_t stream) {
+                         size_t ws_bytes, unsigned long long* busy, fvattn_stream_t stream,
+                         unsigned long long stall_ns = 0) {
   Geo g;
   FV_CHECK(make_geo(gi, &g));
   FV_CHECK(check_ptr(q));
   FV_CHECK(check_ptr(k));
   FV_CHECK(check_ptr(v));
   FV_CHECK(check_ptr(out));
-  FV_CHECK(check_ptr(lse));
-  if (mask != nullptr) FV_CHECK(check_ptr(mask));
+  FV_CHECK(check_ptr4(lse));
+  if (mask != nullptr) FV_CHECK(check_ptr4(mask));
   if (busy != nullptr && (reinterpret_cast<uintptr_t>(busy) & 7u)) return FVATTN_ERR_UNSUPPORTED;
   if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
   if (ws == nullptr || ws_bytes < fv::attn_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
@@ -129,7 +138,7 @@ fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, 
       !encode_map(&maps.v, v, g, g.bw) || !encode_map(&maps.ve, v, g, rx_edge))
     return FVATTN_ERR_CUDA;
   return cuda_status(fv::launch_attn(g, maps, mask, scale, out, lse, ws, busy, nsm,
-                                     reinterpret_cast<cudaStream_t>(stream)));
+                                     reinterpret_cast<cudaStream_t>(stream), stall_ns));
 }
 
 // Scratch for fvattn_block_sparse_attn_noalloc: the tile queue, the error word and the
@@ -140,23 +149,58 @@ static __device__ __align__(256) unsigned char g_noalloc_scratch[kNoAllocScratch
 
 constexpr int kMaxDevices = 64;
 std::mutex g_noalloc_mu;
-void* g_noalloc_addr[kMaxDevices] = {};
+struct NoAllocSlot {
+  unsigned long long ctx_id;   // driver context the address belongs to (0: none yet)
+  void* addr;
+};
+NoAllocSlot g_noalloc_slot[kMaxDevices] = {};
 
-// Device address of g_noalloc_scratch on the current device, resolved once per device
-// (host code only holds a host-side stand-in for the symbol).
+// Identifier of the calling thread's current driver context (0 when there is none).  A
+// device reset or a new context loads the library's module again, and the static array
+// may then sit at another address, so the cached address is keyed on this identifier.
+unsigned long long current_ctx_id() {
+  static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
+  static PFN_cuCtxGetId_v12000 get_id = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_cur = reinterpret_cast<PFN_cuCtxGetCurrent_v4000>(p);
+    p = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      get_id = reinterpret_cast<PFN_cuCtxGetId_v12000>(p);
+  });
+  if (get_cur == nullptr || get_id == nullptr) return 0;
+  CUcontext ctx = nullptr;
+  if (get_cur(&ctx) != CUDA_SUCCESS || ctx == nullptr) return 0;
+  unsigned long long id = 0;
+  if (get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+  return id;
+}
+
+// Device address of g_noalloc_scratch in the current context.  Host code only holds a
+// host-side stand-in for the symbol, so the address is asked of the runtime
+// (cudaGetSymbolAddress) the first time a device's context is seen, and again whenever
+// that device's current context has changed since (for instance after cudaDeviceReset).
 fvattn_status_t noalloc_scratch(void** out) {
   int dev = 0;
   fvattn_status_t st = cuda_status(cudaGetDevice(&dev));
   if (st != FVATTN_OK) return st;
   if (dev < 0 || dev >= kMaxDevices) return FVATTN_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
-  if (g_noalloc_addr[dev] == nullptr) {
+  NoAllocSlot& slot = g_noalloc_slot[dev];
+  const unsigned long long id = current_ctx_id();
+  if (slot.addr == nullptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     st = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
     if (st != FVATTN_OK) return st;
-    g_noalloc_addr[dev] = p;
+    slot.addr = p;
+    slot.ctx_id = current_ctx_id();   // the runtime call made the primary context current
   }
-  *out = g_noalloc_addr[dev];
+  *out = slot.addr;
   return FVATTN_OK;
 }
 
@@ -190,8 +234,8 @@ fvattn_status_t fvattn_route(const fvattn_geom_t* gi, const float* q_pool, const
   FV_CHECK(make_geo(gi, &g));
   FV_CHECK(check_ptr(q_pool));
   FV_CHECK(check_ptr(k_pool));
-  FV_CHECK(check_ptr(mask));
-  FV_CHECK(check_ptr(counts));
+  FV_CHECK(check_ptr4(mask));
+  FV_CHECK(check_ptr4(counts));
   if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
   if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
@@ -212,8 +256,8 @@ fvattn_status_t fvattn_route_ws(const fvattn_geom_t* gi, const float* q_pool, co
   FV_CHECK(make_geo(gi, &g));
   FV_CHECK(check_ptr(q_pool));
   FV_CHECK(check_ptr(k_pool));
-  FV_CHECK(check_ptr(mask));
-  FV_CHECK(check_ptr(counts));
+  FV_CHECK(check_ptr4(mask));
+  FV_CHECK(check_ptr4(counts));
   if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
   if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
@@ -221,6 +265,46 @@ fvattn_status_t fvattn_route_ws(const fvattn_geom_t* gi, const float* q_pool, co
   if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FVATTN_ERR_UNSUPPORTED;
   return cuda_status(fv::launch_route_ws(g, q_pool, k_pool, p, k_floor, scale, mask, counts, workspace,
                                          reinterpret_cast<cudaStream_t>(stream)));
+}
+
+fvattn_status_t fvattn_route_ex(const fvattn_geom_t* gi, const float* q_pool, const float* k_pool,
+                                const fvattn_route_opts_t* opts, uint32_t* mask, int32_t* counts,
+                                void* workspace, size_t ws_bytes, fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr(q_pool));
+  FV_CHECK(check_ptr(k_pool));
+  FV_CHECK(check_ptr4(mask));
+  FV_CHECK(check_ptr4(counts));
+  if (opts == nullptr) return FVATTN_ERR_INVALID_ARG;
+  const float p = opts->p, scale = opts->scale;
+  if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
+  if (opts->k_floor < 0) return FVATTN_ERR_INVALID_ARG;
+  if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
+  if (opts->token_mass != 0 && opts->token_mass != 1) return FVATTN_ERR_INVALID_ARG;
+  if (opts->repair != 0 && opts->repair != 1) return FVATTN_ERR_INVALID_ARG;
+  if (opts->kf_stride < 0) return FVATTN_ERR_INVALID_ARG;
+  if (workspace == nullptr || ws_bytes < fv::route_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
+  if (reinterpret_cast<uintptr_t>(workspace) & 15u) return FVATTN_ERR_UNSUPPORTED;
+  fv::RouteOpts o;
+  o.token_mass = opts->token_mass;
+  o.kf_stride = opts->kf_stride;
+  o.kf_phase = opts->kf_stride > 0 ? opts->kf_phase % opts->kf_stride : 0;
+  cudaStream_t st = reinterpret_cast<cudaStream_t>(stream);
+  fvattn_status_t s = cuda_status(fv::launch_route_ws(g, q_pool, k_pool, p, opts->k_floor, scale, mask, counts,
+                                                      workspace, st, o));
+  if (s != FVATTN_OK || !opts->repair) return s;
+  return cuda_status(fv::launch_mask_repair(g, mask, mask, counts, st));
+}
+
+fvattn_status_t fvattn_mask_repair(const fvattn_geom_t* gi, const uint32_t* mask_in, uint32_t* mask_out,
+                                   int32_t* counts, fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr4(mask_in));
+  FV_CHECK(check_ptr4(mask_out));
+  FV_CHECK(check_ptr4(counts));
+  return cuda_status(fv::launch_mask_repair(g, mask_in, mask_out, counts, reinterpret_cast<cudaStream_t>(stream)));
 }
 
 size_t fvattn_pool_route_workspace_size(const fvattn_geom_t* gi) {
@@ -239,8 +323,8 @@ fvattn_status_t fvattn_pool_route(const fvattn_geom_t* gi, const void* q, const 
   FV_CHECK(check_ptr(k));
   FV_CHECK(check_ptr(q_pool));
   FV_CHECK(check_ptr(k_pool));
-  FV_CHECK(check_ptr(mask));
-  FV_CHECK(check_ptr(counts));
+  FV_CHECK(check_ptr4(mask));
+  FV_CHECK(check_ptr4(counts));
   if (!(p >= 0.f) || !isfinite(p)) return FVATTN_ERR_INVALID_ARG;
   if (k_floor < 0) return FVATTN_ERR_INVALID_ARG;
   if (!(scale > 0.f) || !isfinite(scale)) return FVATTN_ERR_INVALID_ARG;
@@ -286,6 +370,21 @@ fvattn_status_t fvattn_block_sparse_attn_noalloc(const fvattn_geom_t* gi, const 
   void* scratch = nullptr;
   FV_CHECK(noalloc_scratch(&scratch));
   return run_attn(gi, q, k, v, mask, scale, out, lse, scratch, kNoAllocScratchBytes, sm_busy_ns, stream);
+}
+
+fvattn_status_t fvattn_testing_attn_stall(const fvattn_geom_t* g, const void* q, const void* k,
+                                          const void* v, const uint32_t* mask, float scale, void* out,
+                                          float* lse, void* workspace, size_t ws_bytes,
+                                          unsigned long long stall_ns, fvattn_stream_t stream) {
+  if (mask == nullptr) return FVATTN_ERR_INVALID_ARG;
+  if (stall_ns == 0ull || stall_ns > 100000000ull) return FVATTN_ERR_INVALID_ARG;
+  return run_attn(g, q, k, v, mask, scale, out, lse, workspace, ws_bytes, nullptr, stream, stall_ns);
+}
+
+fvattn_status_t fvattn_noalloc_device_status(fvattn_stream_t stream) {
+  void* scratch = nullptr;
+  FV_CHECK(noalloc_scratch(&scratch));
+  return fvattn_device_status(scratch, stream);
 }
 
 fvattn_status_t fvattn_device_status(const void* workspace, fvattn_stream_t stream) {

@@ -62,14 +62,6 @@ constexpr uint32_t kColO = 128 * kNS;  // O: columns [256, 256 + d)
 template <int D> __host__ __device__ constexpr uint32_t col_p() { return kColO + D; }   // P slot r: +64r
 static_assert(col_p<128>() + 64 * kNP <= 512, "tensor memory layout exceeds 512 columns");
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
-// True in exactly one lane of the (converged) warp.
-__device__ __forceinline__ bool elect_one() {
-  uint32_t pred;
-  asm volatile(
-      "{\n\t.reg .pred P;\n\telect.sync _|P, 0xffffffff;\n\tselp.u32 %0, 1, 0, P;\n\t}"
-      : "=r"(pred));
-  return pred != 0;
-}
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
   float r;
@@ -91,6 +83,8 @@ struct AttnParams {
   int rows_e;             // box rows of a W-edge block (bt * bh * (Ws mod bw))
   int qg;                 // narrow query blocks grouped per 128-row tile (1: none)
   int qps;                // lane quarters per grouped query block (rows_e / 32)
+  unsigned long long stall_ns;  // test hook: > 0 makes the S issuer wait this long on a
+                                // barrier nothing arrives at, at its first tile (0: off)
 };
 
 struct __align__(8) AttnBars {
@@ -108,6 +102,7 @@ struct __align__(8) AttnBars {
   uint64_t xread[4];      //   ... and read by both warps of the quarter pair
   uint64_t t_full[kTR], t_empty[kTR];
   uint64_t fin[2];        // drain after an abort: S issuer, P.V issuer
+  uint64_t never;         // no thread arrives here (the stall test hook waits on it)
   int tile[kTR];
   int bcount[kTR];        // kept wide blocks of the tile
   int ncount[kTR];        // kept narrow (packed) blocks of the tile
@@ -249,6 +244,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kTR; ++i) { mbar_init(&bars.t_full[i], 1); mbar_init(&bars.t_empty[i], 3 + kSoftWarps); }
     mbar_init(&bars.fin[0], 1);
     mbar_init(&bars.fin[1], 1);
+    mbar_init(&bars.never, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
@@ -475,6 +471,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       const int nitems = num_items(nw, nn, prm.pack);
       if (!wwait(&bars.q_full, mqc & 1)) break;
       ++mqc;
+      if (prm.stall_ns != 0ull && tcount == 1 &&
+          !__all_sync(0xffffffffu, mbar_wait(&bars.never, 0, abort, err, prm.stall_ns)))
+        break;   // the wait gives up (it always does): the CTA aborts and drains
       int n = 0;
       for (; n < nitems; ++n) {
         const uint32_t c = gc + n;
@@ -1095,7 +1094,7 @@ static cudaError_t launch_attn_d(const Geo& g, const AttnMaps& maps, const AttnP
 
 cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask, float scale,
                         void* out, float* lse, void* ws, unsigned long long* busy, int nsm,
-                        cudaStream_t st) {
+                        cudaStream_t st, unsigned long long stall_ns) {
   const int ntiles = g.B * g.H * g.nB;
   uint32_t* hdr = static_cast<uint32_t*>(ws);
   int* order = reinterpret_cast<int*>(static_cast<unsigned char*>(ws) + kWsHeader);
@@ -1134,6 +1133,7 @@ cudaError_t launch_attn(const Geo& g, const AttnMaps& maps, const uint32_t* mask
   prm.order = order;
   prm.ntiles = ntiles;
   prm.busy = busy;
+  prm.stall_ns = stall_ns;
   const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
   prm.rows_e = g.bt * g.bh * rx_edge;
   const bool narrow_ok = rx_edge < g.bw && (prm.rows_e == 16 || prm.rows_e == 32 || prm.rows_e == 64) &&

@@ -11,7 +11,6 @@
 
 #include "fv_common.cuh"
 #include "fv_launch.h"
-#include "fv_plan.h"
 
 namespace fv {
 
@@ -162,10 +161,25 @@ __device__ __forceinline__ bool unique_prefix(const uint32_t* key, uint32_t& u) 
   return true;
 }
 
+// Whether key block j holds a keyframe: latent frame t is one when (t - phase) mod
+// stride == 0 (LVSA README, rotating keyframes); stride 0: no keyframes.
+__device__ __forceinline__ bool keyframe_block(const Geo& g, const RouteOpts& o, int j) {
+  if (o.kf_stride <= 0) return false;
+  const int tb = div_r(j, g.nBy * g.nBx, g.r_plane);
+  const int t0 = tb * g.bt, t1 = min(g.T, t0 + g.bt);
+  int off = (o.kf_phase - t0) % o.kf_stride;
+  if (off < 0) off += o.kf_stride;
+  return t0 + off < t1;
+}
+
 // Selection for one query block; the row's logits are in sL[i], i = c*32 + lane.
+// With o.token_mass the Top-p runs over tokens: the blocks keep the logits' order and a
+// block's mass is its real token count times exp(logit - max), normalised over the row.
+// Keyframe blocks (o.kf_stride > 0) are kept in every row, after the prefix rule.
 template <int MAXW>
-__device__ __forceinline__ void select_row(const float* sL, int nB, int words, int qb, float p,
-                                           int k_floor, uint32_t* mrow, int32_t* cnt_out, int lane) {
+__device__ __forceinline__ void select_row(const Geo& g, const RouteOpts& o, const float* sL, int nB,
+                                           int words, int qb, float p, int k_floor, uint32_t* mrow,
+                                           int32_t* cnt_out, int lane) {
   uint32_t key[MAXW];
   float sc[MAXW];
   float mx = -INFINITY;
@@ -182,7 +196,8 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
   float z = 0.f;
 #pragma unroll
   for (int c = 0; c < MAXW; ++c) {
-    const float e = key[c] ? expf(sc[c] - mx) : 0.f;
+    float e = key[c] ? expf(sc[c] - mx) : 0.f;
+    if (o.token_mass && key[c]) e *= static_cast<float>(block_info(g, c * 32 + lane).nvalid);
     sc[c] = e;
     z += e;
   }
@@ -220,22 +235,27 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
     if (!unique_prefix<MAXW>(key, u)) {
       for (int bit = 15; bit >= 0; --bit) mass_step(bit);
     }
-    int gt = 0, eq = 0;
-    float gm = 0.f, es = 0.f;
+    int gt = 0;
+    float gm = 0.f;
 #pragma unroll
     for (int c = 0; c < MAXW; ++c) {
       if (key[c] > u) { ++gt; gm += sc[c]; }
-      if (key[c] == u && key[c] != 0u) { ++eq; es = sc[c]; }
     }
     gt = warp_sum_i(gt);
-    eq = warp_sum_i(eq);
     gm = warp_sum(gm);
-    es = warp_max(es);
+    // blocks with key u (ties) join in ascending block index, each with its own mass,
+    // until the prefix reaches p
     float acc = gm;
     int r = 0;
-    while (acc < p && r < eq) {
-      acc += es;
-      ++r;
+#pragma unroll
+    for (int c = 0; c < MAXW; ++c) {
+      uint32_t tb = __ballot_sync(0xffffffffu, key[c] != 0u && key[c] == u);
+      while (tb != 0u && acc < p) {
+        const int l = __ffs(tb) - 1;
+        tb &= tb - 1u;
+        acc += __shfl_sync(0xffffffffu, sc[c], l);
+        ++r;
+      }
     }
     m_p = gt + r;
     ties_needed = r;
@@ -274,7 +294,246 @@ __device__ __forceinline__ void select_row(const float* sL, int nB, int words, i
       const uint32_t tb = __ballot_sync(0xffffffffu, tie);
       const int rank = tie_base + __popc(tb & ((1u << lane) - 1u));
       tie_base += __popc(tb);
-      const bool kept = valid && (key[c] > u || (tie && rank < ties_needed) || i == qb);
+      const bool kept = valid && (key[c] > u || (tie && rank < ties_needed) || i == qb ||
+                                  keyframe_block(g, o, i));
+      const uint32_t word = __ballot_sync(0xffffffffu, kept);
+      cnt += __popc(word);
+      if (lane == 0) mrow[c] = word;
+    }
+  }
+  if (lane == 0) *cnt_out = cnt;
+}
+
+// ----------------------------------------------------------------------------
+// Selection by mass histogram (the form fvattn_route_ws, fvattn_route_ex and
+// fvattn_pool_route use).  Same rule as select_row, with the masses summed exactly: every
+// block's mass exp(l - max) (times its real token count for the Top-p over tokens) is
+// rounded once to a fixed-point integer of 2^-32 units, and all sums are integer sums, so
+// they do not depend on summation order and the prefix test "mass >= p" reads
+// sum >= ceil(p * Z) in integers.  Per row (one warp):
+//   1. logits into registers (lane l holds blocks c * 32 + l), row maximum;
+//   2. a 256-bucket histogram of mass and count in shared memory, bucket
+//      b = min(255, floor((max - l) * 16)): buckets are contiguous ranges of the logit
+//      order, 1/16 logit wide, the last one holding everything 16 or more below the max
+//      (at most e^-16 of the row's mass per block);
+//   3. a warp scan over the buckets finds the bucket where the prefix mass reaches p;
+//   4. that bucket's blocks (a few at these shapes) are gathered and ranked exactly by
+//      (logit desc, index asc); the cut is the first rank at which the prefix reaches p;
+//   5. the Top-k floor, when it lengthens the prefix, repeats 3-4 on counts;
+//   6. the mask: blocks above the cut's key, tied blocks up to the cut's index, the own
+//      block and keyframe blocks.
+// A bucket with more than kSelCap blocks (a cut far down a nearly flat tail) runs
+// select_row on the row instead.
+// ----------------------------------------------------------------------------
+constexpr int kSelBuckets = 256;
+constexpr float kSelPerLogit = 16.f;
+constexpr int kSelCap = 64;
+
+struct SelScratch {                      // one per warp
+  unsigned long long hm[kSelBuckets];    // mass per bucket (2^-32 units)
+  uint32_t hc[kSelBuckets];              // blocks per bucket
+  unsigned long long lw[kSelCap];        // gathered bucket: mass,
+  uint32_t lkey[kSelCap];                //   order key,
+  uint32_t lidx[kSelCap];                //   block index
+};
+
+__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+__device__ __forceinline__ int sel_bucket(float mx, float x) {
+  return min(kSelBuckets - 1, __float2int_rz((mx - x) * kSelPerLogit));
+}
+
+__device__ __forceinline__ unsigned long long sel_fixed(float w) {
+  return __float2ull_rn(w * 4294967296.0f);
+}
+
+// Finds the bucket where the running sum (mass when `by_mass`, else count) first reaches
+// `target`, scanning buckets from the top of the order.  Returns the bucket and, through
+// `above`, the sum over the buckets before it (and `cnt_above`, their block count).
+__device__ __forceinline__ int sel_find_bucket(const SelScratch& sh, bool by_mass, unsigned long long target,
+                                               unsigned long long& above, int& cnt_above, int lane) {
+  unsigned long long loc[8];
+  int cl[8];
+  unsigned long long run = 0;
+  int crun = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    const int b = lane * 8 + e;
+    cl[e] = static_cast<int>(sh.hc[b]);
+    loc[e] = by_mass ? sh.hm[b] : static_cast<unsigned long long>(cl[e]);
+    run += loc[e];
+    crun += cl[e];
+  }
+  unsigned long long incl = run;
+  int cincl = crun;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    const int cv = __shfl_up_sync(0xffffffffu, cincl, off);
+    if (lane >= off) { incl += v; cincl += cv; }
+  }
+  unsigned long long excl = incl - run;
+  int cexcl = cincl - crun;
+  int found = kSelBuckets;
+  unsigned long long f_above = 0;
+  int f_cnt = 0;
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    if (found == kSelBuckets && excl + loc[e] >= target) {
+      found = lane * 8 + e;
+      f_above = excl;
+      f_cnt = cexcl;
+    }
+    excl += loc[e];
+    cexcl += cl[e];
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, found < kSelBuckets);
+  const int src = hit ? __ffs(hit) - 1 : 31;
+  above = __shfl_sync(0xffffffffu, f_above, src);
+  cnt_above = __shfl_sync(0xffffffffu, f_cnt, src);
+  return hit ? __shfl_sync(0xffffffffu, found, src) : kSelBuckets - 1;
+}
+
+template <int MAXW>
+__device__ __forceinline__ void select_row_hist(const Geo& g, const RouteOpts& o, const float* lrow, int nB,
+                                                int words, int qb, float p, int k_floor, uint32_t* mrow,
+                                                int32_t* cnt_out, int lane, SelScratch& sh) {
+  uint32_t key[MAXW];
+  float x[MAXW];
+  float mx = -INFINITY;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    const int i = c * 32 + lane;
+    const bool v = c < words && i < nB;
+    x[c] = v ? __ldcg(lrow + i) : -INFINITY;
+    key[c] = v ? order_key(x[c]) : 0u;
+    mx = fmaxf(mx, x[c]);
+  }
+  mx = warp_max(mx);
+#pragma unroll
+  for (int e = 0; e < 8; ++e) {
+    sh.hm[lane * 8 + e] = 0ull;
+    sh.hc[lane * 8 + e] = 0u;
+  }
+  __syncwarp();
+  auto mass_of = [&](int c) -> float {
+    float w = expf(x[c] - mx);
+    if (o.token_mass) w *= static_cast<float>(block_info(g, c * 32 + lane).nvalid);
+    return w;
+  };
+  unsigned long long z = 0;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    if (key[c] != 0u) {
+      const unsigned long long w = sel_fixed(mass_of(c));
+      const int b = sel_bucket(mx, x[c]);
+      atomicAdd(&sh.hm[b], w);
+      atomicAdd(&sh.hc[b], 1u);
+      z += w;
+    }
+  }
+  z = warp_sum_u64(z);
+  __syncwarp();
+
+  // Gathers bucket b's blocks into the list; false when they do not fit.
+  auto gather = [&](int b, int n) -> bool {
+    if (n > kSelCap) return false;
+    int base = 0;
+#pragma unroll
+    for (int c = 0; c < MAXW; ++c) {
+      const bool in = key[c] != 0u && sel_bucket(mx, x[c]) == b;
+      const uint32_t bal = __ballot_sync(0xffffffffu, in);
+      if (in) {
+        const int pos = base + __popc(bal & ((1u << lane) - 1u));
+        sh.lkey[pos] = key[c];
+        sh.lidx[pos] = static_cast<uint32_t>(c * 32 + lane);
+        sh.lw[pos] = sel_fixed(mass_of(c));
+      }
+      base += __popc(bal);
+    }
+    __syncwarp();
+    return true;
+  };
+  // Among the n gathered blocks, the one of smallest rank (key desc, index asc) at which
+  // above + (running sum of weights up to it) >= target; weight = mass or 1.
+  auto resolve = [&](int n, bool by_mass, unsigned long long above, int& rank_out, uint32_t& key_out,
+                     int& idx_out, unsigned long long target) {
+    int best = 0x7fffffff;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int j = lane + 32 * h;
+      if (j < n) {
+        const uint32_t kj = sh.lkey[j], ij = sh.lidx[j];
+        int rank = 0;
+        unsigned long long pre = 0;
+        for (int t = 0; t < n; ++t) {
+          const uint32_t kt = sh.lkey[t], it = sh.lidx[t];
+          const bool before = kt > kj || (kt == kj && it < ij);
+          rank += before ? 1 : 0;
+          if (before || t == j) pre += by_mass ? sh.lw[t] : 1ull;
+        }
+        // a block whose prefix reaches the target codes as its rank; the others code
+        // above every such rank, the last in the order lowest (the whole bucket)
+        best = min(best, above + pre >= target ? rank * 64 + j : (2 * n - 1 - rank) * 64 + j);
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, off));
+    const int j = best & 63;
+    rank_out = best >> 6;
+    key_out = sh.lkey[j];
+    idx_out = static_cast<int>(sh.lidx[j]);
+    __syncwarp();
+  };
+
+  const int floor_k = min(max(k_floor, 0), nB);
+  int m_p = nB;
+  uint32_t ucut = 0u;        // blocks with key > ucut, and key == ucut up to index icut, are kept
+  int icut = -1;
+  bool all = true;
+  if (p < 1.f) {
+    // at least one unit, so that p = 0 still keeps the first block of the order
+    const unsigned long long target =
+        max(1ull, static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(z))));
+    unsigned long long above;
+    int cnt_above;
+    const int b = sel_find_bucket(sh, true, target, above, cnt_above, lane);
+    if (!gather(b, static_cast<int>(sh.hc[b]))) {
+      select_row<MAXW>(g, o, lrow, nB, words, qb, p, k_floor, mrow, cnt_out, lane);
+      return;
+    }
+    int rank;
+    resolve(static_cast<int>(sh.hc[b]), true, above, rank, ucut, icut, target);
+    m_p = cnt_above + rank + 1;
+    all = false;
+  }
+  const int M = max(max(m_p, floor_k), 1);
+  if (M >= nB) {
+    all = true;
+  } else if (M > m_p) {
+    unsigned long long above;
+    int cnt_above;
+    const int b = sel_find_bucket(sh, false, static_cast<unsigned long long>(M), above, cnt_above, lane);
+    if (!gather(b, static_cast<int>(sh.hc[b]))) {
+      select_row<MAXW>(g, o, lrow, nB, words, qb, p, k_floor, mrow, cnt_out, lane);
+      return;
+    }
+    int rank;
+    resolve(static_cast<int>(sh.hc[b]), false, above, rank, ucut, icut, static_cast<unsigned long long>(M));
+    all = false;
+  }
+  int cnt = 0;
+#pragma unroll
+  for (int c = 0; c < MAXW; ++c) {
+    if (c < words) {
+      const int i = c * 32 + lane;
+      const bool valid = key[c] != 0u;
+      const bool kept = valid && (all || key[c] > ucut || (key[c] == ucut && i <= icut) || i == qb ||
+                                  keyframe_block(g, o, i));
       const uint32_t word = __ballot_sync(0xffffffffu, kept);
       cnt += __popc(word);
       if (lane == 0) mrow[c] = word;
@@ -381,7 +640,7 @@ __global__ void __launch_bounds__(kRouteThreads) route_kernel(Geo g, const float
   }
   const int qb = row0 + warp;
   if (qb < nB)
-    select_row<MAXW>(sL + warp * nBpad, nB, words, qb, p, k_floor,
+    select_row<MAXW>(g, RouteOpts{}, sL + warp * nBpad, nB, words, qb, p, k_floor,
                      mask + (static_cast<size_t>(bhi) * nB + qb) * words,
                      counts + static_cast<size_t>(bhi) * nB + qb, lane);
 }
@@ -427,349 +686,167 @@ cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p
 }
 
 // ----------------------------------------------------------------------------
-// Routing in two kernels, for callers that pass a workspace (fvattn_route_ws): the
-// logits of every (query block, key block) pair go to the workspace as an fp32 matrix
-// per (b, h), rows padded to words * 32; then one warp per query block runs the same
-// selection as route_kernel from its row.  The per-logit arithmetic is the fused
-// kernel's (two partial sums over the even and odd components of each float4 of d, in
-// ascending d, added at the end, times scale), so both paths give the same mask.
+// Routing in two kernels, for callers that pass a workspace (fvattn_route_ws,
+// fvattn_route_ex, fvattn_pool_route): the logits of every (query block, key block) pair go
+// to the workspace as an fp32 matrix per (b, h), rows padded to words * 32, computed on
+// the tensor cores (fv_route_tc.cu); then one warp per query block selects from its row
+// by mass histogram (select_row_hist).
 // ----------------------------------------------------------------------------
-
-// One 64 x 64 tile of logits: query blocks [64 qt, +64) against key blocks [64 kt, +64)
-// of slice bhi.  sQ and sK are [64][D + 4] floats of shared memory each.  kL2 reads the
-// pooled rows from L2 only (ld.global.cg): set when they were written earlier in the
-// same kernel, by other CTAs.
-// kSplit loads each float4 step's (x, y) operands, runs their 16 products, then the
-// (z, w) ones: every accumulator sees the same operations in the same order as without
-// it, with half the operand registers live (for the fused kernel's register budget).
-template <int D, bool kL2, bool kSplit>
-__device__ __forceinline__ void logits_tile(const Geo& g, const float* __restrict__ qp,
-                                            const float* __restrict__ kp, float scale,
-                                            float* __restrict__ logits, int qt, int kt, int bhi,
-                                            float* sQ, float* sK) {
-  constexpr int RS = D + 4;            // padded row (floats)
-  const int nB = g.nB, nBpad = g.words * 32;
-  const int q0 = qt * kLogitTile, k0 = kt * kLogitTile;
-  const float* qh = qp + static_cast<size_t>(bhi) * nB * D;
-  const float* kh = kp + static_cast<size_t>(bhi) * nB * D;
-  for (int e = threadIdx.x; e < kLogitTile * D / 4; e += 256) {
-    const int r = e / (D / 4), d4 = e - r * (D / 4);
-    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    const float4* qs = reinterpret_cast<const float4*>(qh + static_cast<size_t>(q0 + r) * D) + d4;
-    const float4* ks = reinterpret_cast<const float4*>(kh + static_cast<size_t>(k0 + r) * D) + d4;
-    reinterpret_cast<float4*>(sQ + r * RS)[d4] = q0 + r < nB ? (kL2 ? __ldcg(qs) : *qs) : z;
-    reinterpret_cast<float4*>(sK + r * RS)[d4] = k0 + r < nB ? (kL2 ? __ldcg(ks) : *ks) : z;
-  }
-  __syncthreads();
-  // thread (ty, tx) takes query rows ty + 16 i and key blocks tx + 16 j, i, j < 4
-  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
-  uint64_t acc[4][4];
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
-  if constexpr (kSplit) {
-#pragma unroll 2
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-#pragma unroll
-      for (int h = 0; h < 2; ++h) {    // h = 0: (x, y) components, h = 1: (z, w)
-        uint64_t qv[4], kv[4];
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-          const float2 x = reinterpret_cast<const float2*>(sQ + (ty + 16 * i) * RS)[2 * d4 + h];
-          qv[i] = f32x2(x.x, x.y);
-          const float2 k2 = reinterpret_cast<const float2*>(sK + (tx + 16 * i) * RS)[2 * d4 + h];
-          kv[i] = f32x2(k2.x, k2.y);
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i)
-#pragma unroll
-          for (int j = 0; j < 4; ++j) acc[i][j] = ffma2(qv[i], kv[j], acc[i][j]);
-      }
-    }
-  } else {
-#pragma unroll 4
-    for (int d4 = 0; d4 < D / 4; ++d4) {
-      uint64_t qxy[4], qzw[4], kxy[4], kzw[4];
-#pragma unroll
-      for (int i = 0; i < 4; ++i) {
-        const float4 x = reinterpret_cast<const float4*>(sQ + (ty + 16 * i) * RS)[d4];
-        qxy[i] = f32x2(x.x, x.y);
-        qzw[i] = f32x2(x.z, x.w);
-        const float4 k4 = reinterpret_cast<const float4*>(sK + (tx + 16 * i) * RS)[d4];
-        kxy[i] = f32x2(k4.x, k4.y);
-        kzw[i] = f32x2(k4.z, k4.w);
-      }
-#pragma unroll
-      for (int i = 0; i < 4; ++i)
-#pragma unroll
-        for (int j = 0; j < 4; ++j) {
-          acc[i][j] = ffma2(qxy[i], kxy[j], acc[i][j]);   // a0 += x.x k.x, a1 += x.y k.y
-          acc[i][j] = ffma2(qzw[i], kzw[j], acc[i][j]);   // a0 += x.z k.z, a1 += x.w k.w
-        }
-    }
-  }
-  float* out = logits + static_cast<size_t>(bhi) * nB * nBpad;
-#pragma unroll
-  for (int i = 0; i < 4; ++i) {
-    const int qr = q0 + ty + 16 * i;
-    if (qr >= nB) continue;
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int kc = k0 + tx + 16 * j;
-      if (kc >= nB) continue;
-      float a0, a1;
-      unpack_f32x2(acc[i][j], a0, a1);
-      out[static_cast<size_t>(qr) * nBpad + kc] = (a0 + a1) * scale;
-    }
-  }
-}
-
-template <int D>
-__global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restrict__ qp,
-                                                     const float* __restrict__ kp, float scale,
-                                                     float* __restrict__ logits) {
-  extern __shared__ __align__(16) unsigned char lg_smem[];
-  float* sQ = reinterpret_cast<float*>(lg_smem);   // [64][D + 4]
-  float* sK = sQ + kLogitTile * (D + 4);           // [64][D + 4]
-  logits_tile<D, false, false>(g, qp, kp, scale, logits, blockIdx.x, blockIdx.y, blockIdx.z, sQ, sK);
-}
-
 template <int MAXW>
-__global__ void __launch_bounds__(256) select_kernel(Geo g, const float* __restrict__ logits, float p,
-                                                     int k_floor, uint32_t* __restrict__ mask,
-                                                     int32_t* __restrict__ counts) {
+__global__ void __launch_bounds__(128) select_hist_kernel(Geo g, RouteOpts o, const float* __restrict__ logits,
+                                                          float p, int k_floor, uint32_t* __restrict__ mask,
+                                                          int32_t* __restrict__ counts) {
+  __shared__ SelScratch sh[4];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nB = g.nB, nBpad = g.words * 32;
-  const long long row = static_cast<long long>(blockIdx.x) * 8 + warp;   // (b*h) * nB + qb
+  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;   // (b*h) * nB + qb
   if (row >= static_cast<long long>(g.B) * g.H * nB) return;
   const int qb = static_cast<int>(row % nB);
-  select_row<MAXW>(logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
-                   mask + static_cast<size_t>(row) * g.words, counts + row, lane);
+  select_row_hist<MAXW>(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
+                        mask + static_cast<size_t>(row) * g.words, counts + row, lane, sh[warp]);
 }
 
-size_t route_ws_bytes(const Geo& g) {
+// Route workspace: a 256-byte header (word 1: error bits of the logits kernel's bounded
+// waits), then the logits, [B*H][nB][words * 32] fp32.
+constexpr size_t kRouteHdr = 256;
+
+size_t route_logits_bytes(const Geo& g) {
   return static_cast<size_t>(g.B) * g.H * g.nB * (static_cast<size_t>(g.words) * 32) * 4;
 }
 
+size_t route_ws_bytes(const Geo& g) { return kRouteHdr + route_logits_bytes(g); }
+
 template <int D, int MAXW>
 static cudaError_t launch_route2_t(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                                   float scale, uint32_t* mask, int32_t* counts, float* logits,
-                                   cudaStream_t st) {
-  const int tiles = (g.nB + kLogitTile - 1) / kLogitTile;
-  const int smem = 2 * kLogitTile * (D + 4) * 4;
-  cudaError_t e = cudaFuncSetAttribute(logits_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+                                   float scale, uint32_t* mask, int32_t* counts, void* ws,
+                                   cudaStream_t st, const RouteOpts& o) {
+  uint32_t* hdr = static_cast<uint32_t*>(ws);
+  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kRouteHdr);
+  cudaError_t e = cudaMemsetAsync(hdr, 0, kRouteHdr, st);
   if (e != cudaSuccess) return e;
-  logits_kernel<D><<<dim3(tiles, tiles, g.B * g.H), 256, smem, st>>>(g, qp, kp, scale, logits);
-  e = cudaGetLastError();
+  int dev = 0, nsm = 0;
+  e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+  if (e != cudaSuccess) return e;
+  e = launch_logits_tc(g, qp, kp, scale, logits, hdr + 1, nsm, st);
   if (e != cudaSuccess) return e;
   const long long rows = static_cast<long long>(g.B) * g.H * g.nB;
-  select_kernel<MAXW><<<static_cast<unsigned>((rows + 7) / 8), 256, 0, st>>>(g, logits, p, k_floor, mask, counts);
+  select_hist_kernel<MAXW><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(g, o, logits, p, k_floor,
+                                                                                   mask, counts);
   return cudaGetLastError();
 }
 
 template <int D>
 static cudaError_t launch_route2_d(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                                   float scale, uint32_t* mask, int32_t* counts, float* logits,
-                                   cudaStream_t st) {
-  if (g.words <= 4) return launch_route2_t<D, 4>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 8) return launch_route2_t<D, 8>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 12) return launch_route2_t<D, 12>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 16) return launch_route2_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 20) return launch_route2_t<D, 20>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 24) return launch_route2_t<D, 24>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 32) return launch_route2_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  if (g.words <= 48) return launch_route2_t<D, 48>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
-  return launch_route2_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+                                   float scale, uint32_t* mask, int32_t* counts, void* ws,
+                                   cudaStream_t st, const RouteOpts& o) {
+  if (g.words <= 4) return launch_route2_t<D, 4>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 8) return launch_route2_t<D, 8>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 12) return launch_route2_t<D, 12>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 16) return launch_route2_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 20) return launch_route2_t<D, 20>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 24) return launch_route2_t<D, 24>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 32) return launch_route2_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  if (g.words <= 48) return launch_route2_t<D, 48>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  return launch_route2_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
 }
 
 cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st) {
-  float* logits = static_cast<float*>(ws);
-  return g.d == 128 ? launch_route2_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st)
-                    : launch_route2_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, logits, st);
+                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st,
+                            const RouteOpts& o) {
+  return g.d == 128 ? launch_route2_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o)
+                    : launch_route2_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
 }
 
 // ----------------------------------------------------------------------------
-// Pool and route in one persistent kernel (fvattn_pool_route).  Pooling streams Q and K
-// from HBM and leaves most instruction-issue slots idle; the route is bound by issue and
-// reads only the pooled rows and logits, which stay in L2.  So the route of one (b, h)
-// slice runs while later slices are still being pooled.  One queue holds three kinds of
-// item, one CTA per item at a time:
-//   pool      block j of slice s of Q or K                 (2 nB per slice)
-//   logits    a 64 x 64 tile of slice s's logits           (tiles^2 per slice)
-//   select    8 query blocks of slice s: Top-p / Top-k     (ceil(nB / 8) per slice)
-// in steps: step i holds pool(i), then logits(i - 1), then select(i - 2), for the
-// slices that exist.  A logits item waits for all pool items of its slice, a select item
-// for all logits items of its slice (counters in the workspace header).  Every item
-// waited on comes earlier in the queue, where a running CTA took it, so every wait ends;
-// waits are bounded all the same, and on a timeout the select items write a mask that
-// keeps every block.
+// Runtime mask repair (FVAttn explainer, 核心方法 §1, 运行时修补: the materialized mask
+// is patched locally, without new scores).  In each row, a dropped key block whose two
+// neighbours along the time, height or width axis of the block grid both exist and are
+// both kept is a one-block hole and is restored; every decision reads the mask as given
+// (one pass).  One warp per row: the row is staged in shared memory (so the call may
+// work in place), and lane l writes words l and l + 32.  Per axis, bit j of a word has
+// its neighbours j - step and j + step: two 32-bit windows of the row.  A bit qualifies
+// only when its coordinate along the axis is interior (a table per CTA).
 // ----------------------------------------------------------------------------
-constexpr int kFusedThreads = 256;
-constexpr int kFusedMaxWords = 24;     // larger rows run the separate pool and route kernels
-constexpr size_t kPrHeader = 256;      // queue counter, error bits; then 2 counters per slice
+constexpr int kRepairWarps = 8;
+constexpr int kRepairMaxWords = 64;    // nB <= 2048
 
-size_t pool_route_ws_bytes(const Geo& g) {
-  const size_t S = static_cast<size_t>(g.B) * g.H;
-  const size_t head = ((kPrHeader + 8 * S) + 255) / 256 * 256;
-  return head + route_ws_bytes(g);
+// 32 bits of the row starting at bit `start` (bits outside [0, nB) read as zero).
+__device__ __forceinline__ uint32_t row_window(const uint32_t* row, int words, int start) {
+  const int w = start >> 5, sh = start & 31;   // arithmetic shift: floor for negative starts
+  const uint32_t lo = (w >= 0 && w < words) ? row[w] : 0u;
+  const uint32_t hi = (w + 1 >= 0 && w + 1 < words) ? row[w + 1] : 0u;
+  return sh == 0 ? lo : ((lo >> sh) | (hi << (32 - sh)));
 }
 
-// Thread 0 waits until *cnt >= need: acquire loads, bounded by a clock64 deadline (2 s at
-// up to 2 GHz) and by the error word (another item already gave up).  False on either.
-__device__ __forceinline__ bool pr_wait(const uint32_t* cnt, uint32_t need, uint32_t* err) {
-  long long t0 = clock64();
-  for (uint32_t i = 0;; ++i) {
-    uint32_t v;
-    asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(cnt) : "memory");
-    if (v >= need) return true;
-    if ((i & 15u) == 15u) {
-      if (*reinterpret_cast<volatile uint32_t*>(err) & kErrTimeout) return false;
-      if (static_cast<uint64_t>(clock64() - t0) > 4000000000ull) {
-        atomicOr(err, kErrTimeout);
-        return false;
-      }
+__global__ void __launch_bounds__(32 * kRepairWarps) mask_repair_kernel(Geo g, const uint32_t* in,
+                                                                        uint32_t* out, int32_t* counts) {
+  __shared__ uint32_t interior[3][kRepairMaxWords];        // per axis: bits with both neighbours
+  __shared__ uint32_t rowbuf[kRepairWarps][kRepairMaxWords];
+  const int words = g.words, nB = g.nB;
+  for (int w = threadIdx.x; w < 3 * words; w += blockDim.x) {
+    const int axis = w / words, wi = w - axis * words;
+    uint32_t bits = 0u;
+    for (int b = 0; b < 32; ++b) {
+      const int j = wi * 32 + b;
+      if (j >= nB) break;
+      const BlockInfo bi = block_info(g, j);
+      const int c = axis == 0 ? bi.tb : (axis == 1 ? bi.yb : bi.xb);
+      const int ext = axis == 0 ? g.nBt : (axis == 1 ? g.nBy : g.nBx);
+      if (c > 0 && c < ext - 1) bits |= 1u << b;
     }
-    __nanosleep(128);
+    interior[axis][wi] = bits;
   }
-}
-
-// Every thread's writes of the item, then one count for the slice.
-__device__ __forceinline__ void pr_done(uint32_t* cnt) {
-  __threadfence();
   __syncthreads();
-  if (threadIdx.x == 0) atomicAdd(cnt, 1u);
-}
-
-template <int D, int MAXW>
-__global__ void __launch_bounds__(kFusedThreads, 3) pool_route_kernel(
-    Geo g, const uint4* __restrict__ q, const uint4* __restrict__ k, float* qp, float* kp, float p,
-    int k_floor, float scale, uint32_t* __restrict__ mask, int32_t* __restrict__ counts,
-    uint32_t* hdr, float* logits) {
-  extern __shared__ __align__(16) unsigned char pr_smem[];
-  float* sQ = reinterpret_cast<float*>(pr_smem);    // [64][D + 4]; select rows reuse it
-  float* sK = sQ + kLogitTile * (D + 4);            // [64][D + 4]
-  __shared__ float red[kPoolThreads / 32][D];
-  __shared__ long long s_item;
-  __shared__ int s_ok;
-  uint32_t* err = hdr + 1;
-  const int nB = g.nB, nBpad = g.words * 32;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  for (;;) {
-    if (threadIdx.x == 0) s_item = static_cast<long long>(atomicAdd(reinterpret_cast<unsigned long long*>(hdr + 2), 1ull));
-    __syncthreads();
-    const long long t = s_item;
-    __syncthreads();   // s_item is rewritten by the next iteration
-    // the plan is recomputed per item (a few integer operations) rather than held in
-    // registers across the loop
-    const PrPlan pl = pr_plan(g.B * g.H, nB);
-    if (t >= pl.total) break;
-    uint32_t* cnt_pool = hdr + kPrHeader / 4;
-    uint32_t* cnt_logit = cnt_pool + pl.S;
-    int kind, slice, idx;
-    pr_decode(pl, t, kind, slice, idx);
-    if (kind == 0) {
-      const int tensor = idx >= nB ? 1 : 0;
-      const int j = idx - tensor * nB;
-      pool_item<D>(g, tensor ? k : q, tensor ? kp : qp, j, slice, red);
-      pr_done(cnt_pool + slice);
-    } else if (kind == 1) {
-      if (threadIdx.x == 0) s_ok = pr_wait(cnt_pool + slice, static_cast<uint32_t>(pl.nP), err) ? 1 : 0;
-      __syncthreads();
-      if (s_ok) {
-        logits_tile<D, true, true>(g, qp, kp, scale, logits, idx / pl.tiles, idx - (idx / pl.tiles) * pl.tiles,
-                             slice, sQ, sK);
-        pr_done(cnt_logit + slice);
-      }
-    } else {
-      if (threadIdx.x == 0) s_ok = pr_wait(cnt_logit + slice, static_cast<uint32_t>(pl.nL), err) ? 1 : 0;
-      __syncthreads();
-      const int qb = idx * 8 + warp;
-      const size_t row = static_cast<size_t>(slice) * nB + qb;
-      if (qb < nB) {
-        uint32_t* mrow = mask + row * g.words;
-        if (s_ok) {
-          float* sL = sQ + warp * nBpad;
-          const float* lrow = logits + row * nBpad;
-          for (int c = lane; c < nBpad; c += 32) sL[c] = c < nB ? __ldcg(lrow + c) : 0.f;
-          __syncwarp();
-          select_row<MAXW>(sL, nB, g.words, qb, p, k_floor, mrow, counts + row, lane);
-        } else {
-          // the logits never arrived: keep every block, a mask the attention accepts
-          const int tail = nB & 31;
-          for (int w = lane; w < g.words; w += 32)
-            mrow[w] = (w < g.words - 1 || tail == 0) ? 0xffffffffu : (1u << tail) - 1u;
-          if (lane == 0) counts[row] = nB;
-        }
-      }
+  const long long rows = static_cast<long long>(g.B) * g.H * nB;
+  const long long row = static_cast<long long>(blockIdx.x) * kRepairWarps + warp;
+  if (row >= rows) return;
+  uint32_t* rb = rowbuf[warp];
+  const uint32_t* src = in + row * words;
+  for (int w = lane; w < words; w += 32) rb[w] = src[w];
+  __syncwarp();
+  const int steps[3] = {g.nBy * g.nBx, g.nBx, 1};
+  int cnt = 0;
+  for (int w = lane; w < words; w += 32) {
+    uint32_t m = rb[w];
+#pragma unroll
+    for (int a = 0; a < 3; ++a) {
+      const uint32_t left = row_window(rb, words, w * 32 - steps[a]);
+      const uint32_t right = row_window(rb, words, w * 32 + steps[a]);
+      m |= left & right & interior[a][w];
     }
+    if (w == words - 1 && (nB & 31)) m &= (1u << (nB & 31)) - 1u;   // no block at or past nB
+    cnt += __popc(m);
+    out[row * words + w] = m;
   }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) cnt += __shfl_xor_sync(0xffffffffu, cnt, off);
+  if (lane == 0) counts[row] = cnt;
 }
 
-template <int D, int MAXW>
-static cudaError_t launch_pool_route_t(const Geo& g, const void* q, const void* k, float* qp, float* kp,
-                                       float p, int k_floor, float scale, uint32_t* mask, int32_t* counts,
-                                       void* ws, int nsm, cudaStream_t st) {
-  const PrPlan pl = pr_plan(g.B * g.H, g.nB);
-  const size_t head = pool_route_ws_bytes(g) - route_ws_bytes(g);
-  cudaError_t e = cudaMemsetAsync(ws, 0, head, st);
-  if (e != cudaSuccess) return e;
-  const int smem = 2 * kLogitTile * (D + 4) * 4;
-  e = cudaFuncSetAttribute(pool_route_kernel<D, MAXW>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
-  if (e != cudaSuccess) return e;
-  // resident CTAs per SM, queried once per device (the first call, normally outside any
-  // stream capture) and reused
-  static int per_sm_of[64] = {};
-  int dev = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  int per_sm = dev >= 0 && dev < 64 ? per_sm_of[dev] : 0;
-  if (per_sm == 0) {
-    e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, pool_route_kernel<D, MAXW>, kFusedThreads, smem);
-    if (e != cudaSuccess) return e;
-    if (per_sm < 1) return cudaErrorInvalidConfiguration;
-    if (dev >= 0 && dev < 64) per_sm_of[dev] = per_sm;
-  }
-  const long long want = static_cast<long long>(nsm) * per_sm;
-  const int grid = static_cast<int>(pl.total < want ? pl.total : want);
-  uint32_t* hdr = static_cast<uint32_t*>(ws);
-  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + head);
-  pool_route_kernel<D, MAXW><<<grid, kFusedThreads, smem, st>>>(
-      g, static_cast<const uint4*>(q), static_cast<const uint4*>(k), qp, kp, p, k_floor, scale, mask, counts,
-      hdr, logits);
+cudaError_t launch_mask_repair(const Geo& g, const uint32_t* in, uint32_t* out, int32_t* counts,
+                               cudaStream_t st) {
+  const long long rows = static_cast<long long>(g.B) * g.H * g.nB;
+  mask_repair_kernel<<<static_cast<unsigned>((rows + kRepairWarps - 1) / kRepairWarps), 32 * kRepairWarps, 0,
+                       st>>>(g, in, out, counts);
   return cudaGetLastError();
 }
 
-template <int D>
-static cudaError_t launch_pool_route_d(const Geo& g, const void* q, const void* k, float* qp, float* kp,
-                                       float p, int k_floor, float scale, uint32_t* mask, int32_t* counts,
-                                       void* ws, int nsm, cudaStream_t st) {
-  // MAXW sizes without register spills at three CTAs per SM (20 and, at d = 64, 4 spill);
-  // empty slots of a row hold zero keys and add exact zeros, so the mask does not depend
-  // on MAXW
-  if (g.words <= 8) return launch_pool_route_t<D, 8>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
-  if (g.words <= 12) return launch_pool_route_t<D, 12>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
-  if (g.words <= 16) return launch_pool_route_t<D, 16>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
-  return launch_pool_route_t<D, 24>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
-}
+// ----------------------------------------------------------------------------
+// fvattn_pool_route: pooling, then the workspace route, in one call (three kernels on the
+// caller's stream).  Its workspace is the route workspace.
+// ----------------------------------------------------------------------------
+size_t pool_route_ws_bytes(const Geo& g) { return route_ws_bytes(g); }
 
 cudaError_t launch_pool_route(const Geo& g, const void* q, const void* k, float* qp, float* kp, float p,
                               int k_floor, float scale, uint32_t* mask, int32_t* counts, void* ws, int nsm,
                               cudaStream_t st) {
-  if (g.words > kFusedMaxWords) {
-    // rows of more than 768 blocks: the separate kernels (the fused one would need more
-    // registers per thread than three CTAs per SM leave)
-    const size_t head = pool_route_ws_bytes(g) - route_ws_bytes(g);
-    cudaError_t e = cudaMemsetAsync(ws, 0, head, st);   // clean error word for device_status
-    if (e != cudaSuccess) return e;
-    e = launch_pool(g, q, k, qp, kp, st);
-    if (e != cudaSuccess) return e;
-    return launch_route_ws(g, qp, kp, p, k_floor, scale, mask, counts,
-                           static_cast<unsigned char*>(ws) + head, st);
-  }
-  return g.d == 128 ? launch_pool_route_d<128>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st)
-                    : launch_pool_route_d<64>(g, q, k, qp, kp, p, k_floor, scale, mask, counts, ws, nsm, st);
+  (void)nsm;
+  cudaError_t e = launch_pool(g, q, k, qp, kp, st);
+  if (e != cudaSuccess) return e;
+  return launch_route_ws(g, qp, kp, p, k_floor, scale, mask, counts, ws, st);
 }
 
 }  // namespace fv

@@ -19,8 +19,9 @@
  *   x in [xb*bw, ...), clipped to the latent: edge blocks are partial.  Blocks are
  *   numbered T-major: j = (tb*nBy + yb)*nBx + xb, nBt = ceil(T/bt), nBy =
  *   ceil(Hs/bh), nBx = ceil(Ws/bw), nB = nBt*nBy*nBx.
- * - Every pointer argument is a DEVICE pointer, 16-byte aligned, owned by the
- *   caller.  The library allocates no device memory and keeps no state between
+ * - Every pointer argument is a DEVICE pointer owned by the caller, 16-byte aligned,
+ *   except mask, counts and lse, which need 4-byte alignment only (so that a caller
+ *   can pass views of consecutive (b, h) slices of them).  The library allocates no device memory and keeps no state between
  *   calls apart from cached driver entry points.
  * - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy default
  *   stream) and never synchronise.  Argument errors are detected on the host
@@ -104,51 +105,92 @@ FVATTN_API fvattn_status_t fvattn_route(const fvattn_geom_t* g, const float* q_p
                              float p, int k_floor, float scale,
                              uint32_t* mask, int32_t* counts, fvattn_stream_t stream);
 
-/* Bytes of device workspace fvattn_route_ws needs: one fp32 logit per (query block, key
- * block) pair of every (b, h), rows padded to words * 32 entries
- * (B * H * nB * words * 32 * 4 bytes; 5.4 MB at 21x30x52 with 1x8x16 blocks and 12
- * heads, 181 MB at 121x30x52).  0 for an invalid geometry. */
+/* Bytes of device workspace fvattn_route_ws, fvattn_route_ex and fvattn_pool_route need:
+ * a 256-byte header (a status word) followed by one fp32 logit per (query block, key
+ * block) pair of every (b, h), rows padded to words * 32 entries (256 + B * H * nB *
+ * words * 32 * 4 bytes; 5.4 MB at 21x30x52 with 1x8x16 blocks and 12 heads, 181 MB at
+ * 121x30x52).  0 for an invalid geometry. */
 FVATTN_API size_t fvattn_route_workspace_size(const fvattn_geom_t* g);
 
 /* fvattn_route, computed in two kernels through a caller-owned workspace: the logits of
- * all block pairs first (a tiled fp32 product written to `workspace`), then the
- * selection, one query block per warp.  Same definition, inputs, outputs, argument
- * domains and error behaviour as fvattn_route (FVAttn explainer 核心方法 §1: Top-p with a Top-k
- * floor and the own block over softmax(pooled q . pooled k * scale)).  The per-logit
- * arithmetic is the same as fvattn_route's, so the two calls give the same mask and
- * counts.  This form spreads the logits over many more CTAs, which matters most when nB
- * is large.
+ * all block pairs first, on the tensor cores (tf32 with each fp32 operand split into a
+ * high and a low tf32 part, three products per pair: fp32-grade logits), written to
+ * `workspace`; then the selection, one query block per warp, with the masses summed
+ * exactly in fixed point (2^-32 of the row's largest exp).  Same definition, inputs,
+ * outputs, argument domains and error behaviour as fvattn_route (FVAttn explainer
+ * 核心方法 §1: Top-p with a Top-k floor and the own block over softmax(pooled q . pooled
+ * k * scale)); the arithmetic differs from fvattn_route's, so the two may disagree on
+ * blocks whose scores nearly tie at the cut.
  *   workspace, ws_bytes : >= fvattn_route_workspace_size(g) bytes of device memory,
  *                         16-byte aligned, owned by the caller; its contents on entry
- *                         do not matter and on return are the logits (scaled).
- * Returns FVATTN_ERR_WORKSPACE when the workspace is missing or too small. */
+ *                         do not matter and on return hold the logits (scaled).
+ * Returns FVATTN_ERR_WORKSPACE when the workspace is missing or too small.  The logits
+ * kernel's waits are bounded; one that gives up is reported by
+ * fvattn_device_status(workspace) as FVATTN_ERR_DEVICE_TIMEOUT. */
 FVATTN_API fvattn_status_t fvattn_route_ws(const fvattn_geom_t* g, const float* q_pool, const float* k_pool,
                                            float p, int k_floor, float scale, uint32_t* mask,
                                            int32_t* counts, void* workspace, size_t ws_bytes,
                                            fvattn_stream_t stream);
 
-/* Bytes of device workspace fvattn_pool_route needs: a header (an item queue, an error
- * word and two counters per (b, h) slice, B * H * 8 bytes plus 256, rounded up to 256)
- * followed by the logits of fvattn_route_ws (fvattn_route_workspace_size bytes).  0 for
- * an invalid geometry. */
+/* Options of fvattn_route_ex: the routing rule of fvattn_route plus the pages' further
+ * frontend steps, each off when zero. */
+typedef struct {
+  float p;          /* Top-p mass, as fvattn_route                                     */
+  int k_floor;      /* Top-k floor in blocks, as fvattn_route                          */
+  float scale;      /* logit scale, as fvattn_route                                    */
+  int token_mass;   /* 1: Top-p over tokens.  The FVAttn explainer (核心方法 §1, Top-p 路由)
+                     * keeps the minimal TOKEN set whose mass reaches p, and its 3D blocks
+                     * let that decision be taken per block: every real token of key block j
+                     * takes the block's pooled logit l_j, so blocks keep the order of l_j
+                     * and block j carries the mass n_j exp(l_j) / sum_k n_k exp(l_k), n_j its
+                     * real token count.  0: blocks count equally (fvattn_route's rule).  */
+  int kf_stride;    /* > 0: keyframe blocks (LVSA Long-Video Showcase README, Results and
+                     * Configuration: rotating keyframes).  Latent frame t is a keyframe when
+                     * (t - kf_phase) mod kf_stride == 0; every key block holding a keyframe
+                     * frame is kept by every query block, added after the prefix rule like
+                     * the own block (it counts toward neither p nor the floor).  A caller
+                     * rotates the set by changing kf_phase between calls.              */
+  int kf_phase;     /* keyframe phase, any integer                                     */
+  int repair;       /* 1: then runtime mask repair in place (fvattn_mask_repair)          */
+} fvattn_route_opts_t;
+
+/* fvattn_route_ws with the options above: the same logits and selection, with the
+ * Top-p masses over tokens when opts->token_mass, keyframe blocks added to every row
+ * when opts->kf_stride > 0, and fvattn_mask_repair applied to the result when
+ * opts->repair.  Same buffers, workspace (fvattn_route_workspace_size) and error
+ * behaviour as fvattn_route_ws; kf_stride < 0 or token_mass / repair outside {0, 1}
+ * is FVATTN_ERR_INVALID_ARG.  With every option zero it equals fvattn_route_ws. */
+FVATTN_API fvattn_status_t fvattn_route_ex(const fvattn_geom_t* g, const float* q_pool, const float* k_pool,
+                                           const fvattn_route_opts_t* opts, uint32_t* mask, int32_t* counts,
+                                           void* workspace, size_t ws_bytes, fvattn_stream_t stream);
+
+/* Runtime mask repair (FVAttn explainer, 核心方法 §1, 运行时修补: holes between routing
+ * and attention are patched locally, on the materialized mask, without new scores).
+ * Reading: in every row, a dropped key block whose two neighbours along the time, height
+ * or width axis of the 3D block grid both exist and are both kept is a one-block hole,
+ * and is set.  One pass: every decision reads mask_in as given, so holes that only open
+ * up after a fill stay.  Bits at j >= nB are cleared.
+ *   mask_in  : uint32 [B][H][nB][words]          (read)
+ *   mask_out : uint32 [B][H][nB][words]          (written; may equal mask_in)
+ *   counts   : int32  [B][H][nB]                 (written: popcount of each repaired row) */
+FVATTN_API fvattn_status_t fvattn_mask_repair(const fvattn_geom_t* g, const uint32_t* mask_in, uint32_t* mask_out,
+                                              int32_t* counts, fvattn_stream_t stream);
+
+/* Bytes of device workspace fvattn_pool_route needs: fvattn_route_workspace_size(g).  0
+ * for an invalid geometry. */
 FVATTN_API size_t fvattn_pool_route_workspace_size(const fvattn_geom_t* g);
 
-/* fvattn_block_pool followed by fvattn_route_ws, in one persistent kernel (FVAttn
- * explainer 核心方法 §1: pooled 3D blocks, then Top-p with a Top-k floor and the own
- * block).  Same definitions, outputs and argument domains as those two calls, and the
- * same results bit for bit: q_pool, k_pool, mask and counts equal what the two calls
- * write.  Pooling streams Q and K from HBM; the route of a (b, h) slice runs on the
- * same SMs while later slices are still being pooled.  When a mask row has more than
- * 24 words (nB > 768) the call runs the two separate calls' kernels instead.
+/* fvattn_block_pool followed by fvattn_route_ws in one call (FVAttn explainer 核心方法
+ * §1: pooled 3D blocks, then Top-p with a Top-k floor and the own block): the same
+ * kernels on the caller's stream, so q_pool, k_pool, mask and counts equal what the two
+ * calls write.
  *   q, k              : bf16 [B][H][N][d]           (read)
  *   q_pool, k_pool    : fp32 [B][H][nB][d]          (written)
  *   mask, counts      : as fvattn_route             (written)
  *   workspace, ws_bytes : >= fvattn_pool_route_workspace_size(g) bytes, 16-byte aligned,
  *                       owned by the caller, contents on entry do not matter; not to be
  *                       shared by calls that run concurrently.
- * Its kernel waits, bounded, for its own earlier work items; if a wait gives up, the
- * rows it could not route keep every block and fvattn_device_status(workspace) reports
- * FVATTN_ERR_DEVICE_TIMEOUT. */
+ * A wait that gives up is reported by fvattn_device_status(workspace). */
 FVATTN_API fvattn_status_t fvattn_pool_route(const fvattn_geom_t* g, const void* q, const void* k, float p,
                                              int k_floor, float scale, float* q_pool, float* k_pool,
                                              uint32_t* mask, int32_t* counts, void* workspace,
@@ -172,7 +214,9 @@ FVATTN_API int fvattn_num_sms(void);
  *   mask    : uint32 [B][H][nB][words], as written by fvattn_route (bit j of a row:
  *             key block j kept).  Bits at j >= nB are ignored.  A row with no bit set
  *             (fvattn_route always sets bit i) gives out = 0 and lse = -inf for its
- *             tokens.
+ *             tokens.  The per-row counts fvattn_route also writes are not an
+ *             argument: the kernels derive every row's kept blocks, and their number,
+ *             from the mask alone, so no count can disagree with its row.
  *   out     : bf16 [B][H][N][d]      (written, every token)
  *   lse     : fp32 [B][H][N]         (written, every token)
  *   workspace, ws_bytes : >= fvattn_attn_workspace_size(g) bytes, 16-byte aligned,
@@ -203,18 +247,26 @@ FVATTN_API fvattn_status_t fvattn_block_sparse_attn(const fvattn_geom_t* g, cons
  *   131040 tiles) are rejected with FVATTN_ERR_WORKSPACE.
  * - The first call on a device resolves the scratch area's device address
  *   (cudaGetSymbolAddress) with that device current; make that first call before any
- *   stream capture.
+ *   stream capture.  The address is cached per device together with the identifier of
+ *   the driver context it was resolved in; when the device's current context changes
+ *   (after cudaDeviceReset, or under a context the caller made current), the next call
+ *   resolves it again, so that call too belongs outside a stream capture.
  * - Every call shares the one scratch area, which keeps the last call's contents (the
  *   kernels reset what must start at zero).  Calls that overlap on the GPU (different
  *   streams, or different host threads on one device) race on it: serialise them.
- * - A device-side timeout of this entry point is not reported through
- *   fvattn_device_status (there is no workspace to pass it). */
+ * - A device-side timeout of this entry point is reported by
+ *   fvattn_noalloc_device_status (there is no workspace to pass to fvattn_device_status). */
 FVATTN_API fvattn_status_t fvattn_block_sparse_attn_noalloc(const fvattn_geom_t* g, const void* q,
                                                             const void* k, const void* v,
                                                             const uint32_t* mask, float scale,
                                                             void* out, float* lse,
                                                             unsigned long long* sm_busy_ns,
                                                             fvattn_stream_t stream);
+
+/* fvattn_device_status for fvattn_block_sparse_attn_noalloc: synchronises `stream` and
+ * reports how the last call of that entry point on the current device ran, from the
+ * library's static scratch area.  Same return values as fvattn_device_status. */
+FVATTN_API fvattn_status_t fvattn_noalloc_device_status(fvattn_stream_t stream);
 
 /* Dense attention: fvattn_block_sparse_attn with every key block kept (the p = 1
  * case), without reading a mask.  Same arguments otherwise. */

@@ -104,6 +104,8 @@ class RouteResult:
     csum: np.ndarray      # fp64 [B, H, nB, nB] cumulative mass along `order`
     m_p: np.ndarray       # int  [B, H, nB] Top-p prefix length
     m_keep: np.ndarray    # int  [B, H, nB] prefix length after the Top-k floor
+    mass: Optional[np.ndarray] = None   # fp64 [B, H, nB, nB] mass of each block (= scores
+                                        # unless the Top-p runs over tokens)
 
 
 def routing_scores(Qp: np.ndarray, Kp: np.ndarray, scale: float) -> np.ndarray:
@@ -113,16 +115,35 @@ def routing_scores(Qp: np.ndarray, Kp: np.ndarray, scale: float) -> np.ndarray:
     return e / e.sum(axis=-1, keepdims=True)
 
 
-def route(Qp: np.ndarray, Kp: np.ndarray, p: float, k_floor: int, scale: float) -> RouteResult:
+def token_scores(Qp: np.ndarray, Kp: np.ndarray, scale: float, real_count: np.ndarray) -> np.ndarray:
+    """Top-p over tokens, decided per block: every real token of key block j takes the
+    block's pooled logit l_j = (Qp[i] . Kp[j]) * scale, and the softmax runs over all real
+    tokens.  Returns the score of one token of block j, exp(l_j) / sum_k n_k exp(l_k)
+    (n_k = real token count of block k); the block's mass is n_j times it."""
+    logits = np.einsum("bhid,bhjd->bhij", Qp.astype(np.float64), Kp.astype(np.float64)) * scale
+    e = np.exp(logits - logits.max(axis=-1, keepdims=True))
+    return e / (e * np.asarray(real_count, np.float64)).sum(axis=-1, keepdims=True)
+
+
+def route(Qp: np.ndarray, Kp: np.ndarray, p: float, k_floor: int, scale: float,
+          real_count: Optional[np.ndarray] = None) -> RouteResult:
     """Per (batch, head, query block): sort key blocks by score (desc, ties by lower
     index); m_p = the shortest prefix whose cumulative mass is >= p (every block when
     p >= 1, capped at nB); m = max(m_p, min(k_floor, nB)); keep that prefix plus the
-    query's own block."""
+    query's own block.
+
+    With `real_count` (the real token count of every block) the Top-p runs over tokens
+    (:func:`token_scores`): the blocks keep the order of their routing scores (the order
+    of their pooled logits, which every token of the block takes), and `mass`, what the
+    prefix accumulates, is a block's share of the token mass, n_j times its token score."""
     s = routing_scores(Qp, Kp, scale)
+    if real_count is None:
+        mass = s
+    else:
+        mass = token_scores(Qp, Kp, scale, real_count) * np.asarray(real_count, np.float64)
     B, H, nB, _ = s.shape
     order = np.argsort(-s, axis=-1, kind="stable")
-    s_sorted = np.take_along_axis(s, order, axis=-1)
-    csum = np.cumsum(s_sorted, axis=-1)
+    csum = np.cumsum(np.take_along_axis(mass, order, axis=-1), axis=-1)
     if p >= 1.0:
         m_p = np.full((B, H, nB), nB, dtype=np.int64)
     else:
@@ -134,7 +155,7 @@ def route(Qp: np.ndarray, Kp: np.ndarray, p: float, k_floor: int, scale: float) 
     own = np.arange(nB)
     keep[..., own, own] = True
     return RouteResult(keep=keep, counts=keep.sum(axis=-1), scores=s, order=order,
-                       csum=csum, m_p=m_p, m_keep=m_keep)
+                       csum=csum, m_p=m_p, m_keep=m_keep, mass=mass)
 
 
 def pack_mask(keep: np.ndarray) -> np.ndarray:
@@ -153,6 +174,43 @@ def unpack_mask(words: np.ndarray, nB: int) -> np.ndarray:
     w = words.astype(np.uint64)[..., None]
     bits = (w >> np.arange(32, dtype=np.uint64)) & np.uint64(1)
     return bits.reshape(words.shape[:-1] + (words.shape[-1] * 32,))[..., :nB].astype(bool)
+
+
+def keyframe_blocks(g: BlockGeometry, stride: int, phase: int) -> np.ndarray:
+    """Key blocks that hold a keyframe (LVSA README, rotating keyframes): latent frame t is
+    a keyframe when (t - phase) mod stride == 0, and a block is a keyframe block when one
+    of its real frames is.  bool [nB]; all False when stride <= 0."""
+    kf = np.zeros(g.nB, dtype=bool)
+    if stride <= 0:
+        return kf
+    frames = np.arange(g.T)
+    key_t = ((frames - phase) % stride) == 0
+    for j in range(g.nB):
+        tb = j // (g.nBy * g.nBx)
+        kf[j] = key_t[tb * g.bt:min(g.T, tb * g.bt + g.bt)].any()
+    return kf
+
+
+def add_keyframes(keep: np.ndarray, kf: np.ndarray) -> np.ndarray:
+    """Every query block also keeps every keyframe block (added after the prefix rule, like
+    the own block; they do not count toward Top-p or the floor)."""
+    return keep | kf[None, None, None, :]
+
+
+def repair_mask(keep: np.ndarray, g: BlockGeometry) -> np.ndarray:
+    """Runtime mask repair on the materialized mask, without scores (FVAttn explainer,
+    核心方法 §1, 运行时修补): in each row, a dropped key block whose two neighbours along
+    the time, height or width axis of the 3D block grid both exist and are both kept is a
+    one-block hole, and is restored.  One pass: every decision reads the mask as given."""
+    nB = g.nB
+    out = keep.copy()
+    tb, rem = np.divmod(np.arange(nB), g.nBy * g.nBx)
+    yb, xb = np.divmod(rem, g.nBx)
+    for coord, ext, step in ((tb, g.nBt, g.nBy * g.nBx), (yb, g.nBy, g.nBx), (xb, g.nBx, 1)):
+        inner = np.nonzero((coord > 0) & (coord < ext - 1))[0]
+        hole = keep[..., inner - step] & keep[..., inner + step]
+        out[..., inner] |= hole
+    return out
 
 
 def keep_for_cut(r: RouteResult, m: np.ndarray) -> np.ndarray:
@@ -229,7 +287,8 @@ def comparison_band(r: RouteResult, p: float, k_floor: int, band: float = 1e-5
 
 
 def check_route_invariants(keep_row: np.ndarray, s_row: np.ndarray, own: int, p: float,
-                           k_floor: int, tol: float = 0.0) -> Optional[str]:
+                           k_floor: int, tol: float = 0.0,
+                           mass_row: Optional[np.ndarray] = None) -> Optional[str]:
     """Check that a keep vector is a valid Top-p/Top-k/own-block selection for one row
     of scores, up to `tol` on scores and masses.  Returns None when valid, else why.
 
@@ -237,8 +296,10 @@ def check_route_invariants(keep_row: np.ndarray, s_row: np.ndarray, own: int, p:
     without the own block, when the own block was added after the prefix):
     every block of P scores >= every block outside P (minus tol); |P| >= min(k, nB);
     mass(P) >= p - tol unless P is everything; and P is minimal: when |P| exceeds
-    the floor, dropping its lowest-scoring block leaves mass < p + tol."""
+    the floor, dropping its lowest-scoring block leaves mass < p + tol.  Masses are
+    `mass_row` when given (Top-p over tokens), else the scores."""
     nB = s_row.shape[0]
+    m_row = s_row if mass_row is None else mass_row
     if not keep_row[own]:
         return "own block not kept"
     floor = min(int(k_floor), nB)
@@ -255,14 +316,15 @@ def check_route_invariants(keep_row: np.ndarray, s_row: np.ndarray, own: int, p:
             reasons.append("not a top set"); continue
         if n < floor:
             reasons.append("below the Top-k floor"); continue
-        mass = inside.sum()
+        mass = m_row[P].sum()
         if p >= 1.0:
             if n != nB:
                 reasons.append("p >= 1 must keep every block"); continue
             return None
         if n < nB and mass < p - tol:
             reasons.append("mass below p"); continue
-        if n > floor and n > 1 and mass - inside.min() >= p + tol:
+        last = np.nonzero(P)[0][np.argmin(s_row[P])]
+        if n > floor and n > 1 and mass - m_row[last] >= p + tol:
             reasons.append("not minimal"); continue
         return None
     return "; ".join(reasons)
@@ -296,6 +358,39 @@ def brute_force_route_row(s_row: np.ndarray, own: int, p: float, k_floor: int) -
             best, best_mass = S, mass
     keep = np.zeros(nB, dtype=bool)
     keep[list(best)] = True
+    keep[own] = True
+    return keep
+
+
+def brute_force_token_route_row(tok_score_row: np.ndarray, real_count: np.ndarray, own: int,
+                                p: float, k_floor: int) -> np.ndarray:
+    """Token-level reference for one row of the Top-p over tokens (tiny inputs only).  The
+    row is expanded into real tokens, n_j tokens of score tok_score_row[j] for block j,
+    ordered by score (ties by block index); the shortest token prefix whose exact
+    (rational) mass reaches p selects tokens, and a block is kept when it holds a selected
+    token.  The floor then lengthens the kept blocks, in the same block order, to
+    min(k, nB); the own block is added."""
+    nB = tok_score_row.shape[0]
+    blocks = sorted(range(nB), key=lambda j: (-float(tok_score_row[j]), j))
+    tokens = [j for j in blocks for _ in range(int(real_count[j]))]
+    if p >= 1.0:
+        chosen = set(range(nB))
+    else:
+        target, acc, chosen = Fraction(float(p)), Fraction(0), set()
+        for j in tokens:
+            chosen.add(j)
+            acc += Fraction(float(tok_score_row[j]))
+            if acc >= target:
+                break
+        else:
+            chosen = set(range(nB))
+    floor = min(int(k_floor), nB)
+    for j in blocks:
+        if len(chosen) >= floor:
+            break
+        chosen.add(j)
+    keep = np.zeros(nB, dtype=bool)
+    keep[sorted(chosen)] = True
     keep[own] = True
     return keep
 

@@ -19,9 +19,14 @@ def L():
 
 
 def header_functions():
-    src = open(os.path.join(ROOT, "include", "fvattn.h")).read()
-    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
-    return sorted(set(re.findall(r"\b(fvattn_[a-z_]+)\s*\(", src)))
+    names = set()
+    for h in sorted(os.listdir(os.path.join(ROOT, "include"))):
+        if not h.endswith(".h"):
+            continue
+        src = open(os.path.join(ROOT, "include", h)).read()
+        src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+        names |= set(re.findall(r"\b(fvattn_[a-z_]+)\s*\(", src))
+    return sorted(names)
 
 
 def test_exports_every_declared_symbol(L):
@@ -53,7 +58,8 @@ def test_host_side_argument_checks(L):
     assert call_route(L, G480, p=-0.1) == E["FVATTN_ERR_INVALID_ARG"]
     assert call_route(L, G480, k=-1) == E["FVATTN_ERR_INVALID_ARG"]
     assert call_route(L, G480, scale=0.0) == E["FVATTN_ERR_INVALID_ARG"]
-    assert call_route(L, G480, mask=0x3004) == E["FVATTN_ERR_UNSUPPORTED"]     # misaligned
+    assert call_route(L, G480, mask=0x3002) == E["FVATTN_ERR_UNSUPPORTED"]     # misaligned word
+    assert call_route(L, G480, qp=0x1004) == E["FVATTN_ERR_UNSUPPORTED"]       # pooled rows need 16 B
     bad_d = fv.Geometry(1, 12, 21, 30, 52, 96, 1, 8, 16)
     assert call_route(L, bad_d) == E["FVATTN_ERR_UNSUPPORTED"]
     big_block = fv.Geometry(1, 1, 4, 16, 16, 128, 2, 8, 16)        # 256 tokens per block
@@ -85,17 +91,16 @@ def test_host_side_argument_checks(L):
     assert L.fvattn_device_status(None, None) == E["FVATTN_ERR_INVALID_ARG"]
     # two-kernel route: the route checks, then a missing / short / misaligned workspace
     need = fv.fvattn_route_workspace_size(G480)
-    assert need == 12 * 336 * 11 * 32 * 4
+    assert need == 256 + 12 * 336 * 11 * 32 * 4         # status header + logits
     args = (ctypes.byref(cg), 0x1000, 0x2000, 0.9, 4, 0.088, 0x3000, 0x4000)
     assert L.fvattn_route_ws(*args, None, need, None) == E["FVATTN_ERR_WORKSPACE"]
     assert L.fvattn_route_ws(*args, 0x10000, need - 1, None) == E["FVATTN_ERR_WORKSPACE"]
     assert L.fvattn_route_ws(*args, 0x10008, need, None) == E["FVATTN_ERR_UNSUPPORTED"]
     assert L.fvattn_route_ws(ctypes.byref(cg), 0x1000, 0x2000, -1.0, 4, 0.088, 0x3000, 0x4000,
                              0x10000, need, None) == E["FVATTN_ERR_INVALID_ARG"]
-    # pool and route in one call: a header of queue, error word and two counters per
-    # slice, then the same logits
+    # pool and route in one call: the route workspace
     need_pr = fv.fvattn_pool_route_workspace_size(G480)
-    assert need_pr == -(-(256 + 8 * 12) // 256) * 256 + need
+    assert need_pr == need
     pr = lambda p=0.9, kf=4, qp=0x5000, ws=0x10000, n=need_pr: L.fvattn_pool_route(
         ctypes.byref(cg), 0x1000, 0x2000, p, kf, 0.088, qp, 0x6000, 0x3000, 0x4000, ws, n, None)
     assert pr(qp=None) == E["FVATTN_ERR_INVALID_ARG"]
@@ -104,6 +109,31 @@ def test_host_side_argument_checks(L):
     assert pr(ws=None) == E["FVATTN_ERR_WORKSPACE"]
     assert pr(n=need_pr - 1) == E["FVATTN_ERR_WORKSPACE"]
     assert pr(ws=0x10008) == E["FVATTN_ERR_UNSUPPORTED"]
+
+
+def test_route_ex_and_repair_argument_checks(L):
+    E = {v: k for k, v in fv.STATUS_NAMES.items()}
+    cg = G480.c()
+    need = fv.fvattn_route_workspace_size(G480)
+
+    def ex(ws=0x10000, n=need, mask=0x3000, **kw):
+        o = fv.RouteOpts(**{**dict(p=0.9, k_floor=4, scale=0.088), **kw})
+        return L.fvattn_route_ex(ctypes.byref(cg), 0x1000, 0x2000, ctypes.byref(o), mask, 0x4000, ws, n, None)
+    assert L.fvattn_route_ex(ctypes.byref(cg), 0x1000, 0x2000, None, 0x3000, 0x4000, 0x10000, need,
+                             None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(p=-1.0) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(k_floor=-1) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(scale=0.0) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(token_mass=2) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(repair=-1) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(kf_stride=-3) == E["FVATTN_ERR_INVALID_ARG"]
+    assert ex(ws=None) == E["FVATTN_ERR_WORKSPACE"]
+    assert ex(n=need - 1) == E["FVATTN_ERR_WORKSPACE"]
+    assert ex(ws=0x10008) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert ex(mask=0x3001) == E["FVATTN_ERR_UNSUPPORTED"]
+    assert L.fvattn_mask_repair(None, 0x1000, 0x1000, 0x2000, None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert L.fvattn_mask_repair(ctypes.byref(cg), None, 0x1000, 0x2000, None) == E["FVATTN_ERR_INVALID_ARG"]
+    assert L.fvattn_mask_repair(ctypes.byref(cg), 0x1000, 0x1002, 0x2000, None) == E["FVATTN_ERR_UNSUPPORTED"]
 
 
 def test_status_strings(L):

@@ -40,9 +40,9 @@ def check_line(d, n):
     assert set(["value", "unit", "h2d_bytes_per_step", "d2h_bytes_per_step"]) <= set(e)
     assert e["h2d_bytes_per_step"] == 3 * 12 * 32760 * 128 * 2          # Q, K, V in
     assert e["d2h_bytes_per_step"] == 12 * 32760 * 128 * 2 + 12 * 32760 * 4   # out and lse back
-    # four kernels a layer step (pool and route fused, prep_cost, prep_order, attention),
-    # three steps
-    assert d["gpu_launches"] == 4 * 3
+    # six kernels a layer step (pool, logits, selection, prep_cost, prep_order,
+    # attention), three steps
+    assert d["gpu_launches"] == 6 * 3
     assert set(["sm_mhz", "sm_max_mhz", "reasons"]) <= set(d["clocks"])
     # the stand-in route keeps every block: the layer's effective FLOPs are the dense count,
     # n replicas of it every 4 ms

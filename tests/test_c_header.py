@@ -43,6 +43,10 @@ int main(void) {
                                                              (const void*)0x3000, (const uint32_t*)0x4000,
                                                              0.088f, (void*)0x5000, (float*)0x6000,
                                                              (void*)0x7000, ws - 256, NULL, NULL));
+  /* the attention calls take the mask alone, no per-row counts */
+  printf("small dense ws %d\n", (int)fvattn_dense_attn(&g, (const void*)0x1000, (const void*)0x2000,
+                                                       (const void*)0x3000, 0.088f, (void*)0x5000,
+                                                       (float*)0x6000, (void*)0x7000, ws - 256, NULL, NULL));
   return 0;
 }
 """
@@ -56,11 +60,11 @@ def libdir():
 @pytest.mark.skipif(shutil.which("gcc") is None, reason="needs gcc")
 def test_header_is_strict_c99_and_cxx17(tmp_path):
     src = tmp_path / "h.c"
-    src.write_text('#include "fvattn.h"\nint main(void) { return 0; }\n')
+    src.write_text('#include "fvattn.h"\n#include "fvattn_testing.h"\nint main(void) { return 0; }\n')
     subprocess.run(["gcc", "-std=c99", "-pedantic-errors", "-Wall", "-Wextra", "-Werror", "-I", INC,
                     "-fsyntax-only", str(src)], check=True)
     srcpp = tmp_path / "h.cpp"
-    srcpp.write_text('#include "fvattn.h"\nint main() { return 0; }\n')
+    srcpp.write_text('#include "fvattn.h"\n#include "fvattn_testing.h"\nint main() { return 0; }\n')
     subprocess.run(["g++", "-std=c++17", "-pedantic-errors", "-Wall", "-Wextra", "-Werror", "-I", INC,
                     "-fsyntax-only", str(srcpp)], check=True)
 
@@ -80,7 +84,7 @@ def test_c_program_links_and_runs_host_entry_points(tmp_path, libdir):
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True, env=env).stdout
     lines = out.splitlines()
     assert lines[0].startswith("nB=336 words=11 attn_ws=")
-    assert lines[0].endswith(f" route_ws={12 * 336 * 11 * 32 * 4}")
+    assert lines[0].endswith(f" route_ws={256 + 12 * 336 * 11 * 32 * 4}")
     # the same static strings the binding reads through ctypes
     assert lines[1:8] == [f"status {i} {fv.fvattn_status_string(i)}" for i in range(7)]
     assert lines[8:] == [
@@ -89,4 +93,5 @@ def test_c_program_links_and_runs_host_entry_points(tmp_path, libdir):
         "p<0 route 1",         # FVATTN_ERR_INVALID_ARG
         "small route ws 3",    # FVATTN_ERR_WORKSPACE
         "small attn ws 3",     # FVATTN_ERR_WORKSPACE
+        "small dense ws 3",    # FVATTN_ERR_WORKSPACE
     ]

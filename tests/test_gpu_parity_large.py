@@ -51,9 +51,11 @@ def test_sweep_480p():
     assert f[-1].min() == 1.0          # p = 1 keeps everything
 
 
-def test_route_ws_equals_route_720p():
-    """The two-kernel route gives exactly the one-kernel route's mask at 720p (20 mask
-    words, 630 blocks)."""
+def test_route_forms_720p():
+    """Both route forms against the oracle at 720p (20 mask words, 630 blocks): the
+    one-kernel fvattn_route (fp32 FMA logits, bitwise threshold search) and the workspace
+    form (tensor-core logits, histogram selection).  Their arithmetic differs, so each is
+    held to the oracle's band on its own."""
     import torch
     import free_adaptive_block_b200 as fv
     wl = W.WAN22_720P
@@ -63,9 +65,14 @@ def test_route_ws_equals_route_720p():
     q, k = P.to_dev(x["q"]), P.to_dev(x["k"])
     b = fv.LayerBuffers.allocate(g)
     fv.fvattn_block_pool(g, q, k, b.q_pool, b.k_pool)
-    fv.fvattn_route(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts)
-    m1, c1 = b.mask.clone(), b.counts.clone()
-    b.mask.fill_(-1)
-    fv.fvattn_route_ws(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts, b.route_ws)
-    torch.cuda.synchronize()
-    assert torch.equal(b.mask, m1) and torch.equal(b.counts, c1)
+    og = O.block_geometry(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    qp, kp = O.pool(x["q"], og), O.pool(x["k"], og)
+    for form in ("route", "route_ws"):
+        b.mask.fill_(-1)
+        if form == "route":
+            fv.fvattn_route(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts)
+        else:
+            fv.fvattn_route_ws(g, b.q_pool, b.k_pool, wl.p, wl.k_floor, sc, b.mask, b.counts, b.route_ws)
+        torch.cuda.synchronize()
+        res = dict(mask=b.mask.cpu().numpy().view(np.uint32), counts=b.counts.cpu().numpy())
+        print(form, P.check_route(wl, qp, kp, res, wl.p, wl.k_floor))

@@ -349,3 +349,121 @@ def test_candidate_cuts_and_keep_for_cut():
     keep = O.keep_for_cut(r2, np.full((1, 1, 3), 1))
     assert keep[0, 0].astype(int).tolist() == [[1, 0, 0], [1, 1, 0], [1, 0, 1]]
     assert (O.keep_for_cut(r2, r2.m_keep) == r2.keep).all()
+
+
+# ------------------------------------------------------------------ next rows of the path
+def test_token_topp_against_token_level_brute_force():
+    """Top-p over tokens, decided per block, against an explicit expansion of every row
+    into real tokens (ragged block sizes: partial blocks on every edge)."""
+    wl = W.SMALL_RAGGED_T
+    x = W.generate(wl)
+    g = O.block_geometry(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    assert len(set(g.real_count.tolist())) > 2
+    Qp, Kp = O.pool(x["q"], g), O.pool(x["k"], g)
+    scale = 1.0 / math.sqrt(wl.d)
+    rng = np.random.default_rng(11)
+    ts = O.token_scores(Qp, Kp, scale, g.real_count)
+    for p, k in [(0.5, 1), (0.8, 3), (0.95, 0), (1.0, 0), (0.3, 30)]:
+        r = O.route(Qp, Kp, p, k, scale, real_count=g.real_count)
+        assert np.allclose(r.mass.sum(-1), 1.0)
+        for b, h, qb in zip(rng.integers(0, wl.B, 12), rng.integers(0, wl.H, 12), rng.integers(0, g.nB, 12)):
+            want = O.brute_force_token_route_row(ts[b, h, qb], g.real_count, qb, p, k)
+            assert (r.keep[b, h, qb] == want).all(), (p, k, b, h, qb)
+            assert O.check_route_invariants(r.keep[b, h, qb], r.scores[b, h, qb], qb, p, k, 1e-12,
+                                            r.mass[b, h, qb]) is None
+
+
+def test_token_topp_equals_block_topp_when_blocks_are_equal():
+    w = W.TINY                                   # every block holds 32 tokens
+    x = W.generate(w)
+    g = O.block_geometry(w.T, w.Hs, w.Ws, w.bt, w.bh, w.bw)
+    Qp, Kp = O.pool(x["q"], g), O.pool(x["k"], g)
+    for p, k in [(0.6, 1), (0.9, 2)]:
+        a = O.route(Qp, Kp, p, k, 0.125)
+        t = O.route(Qp, Kp, p, k, 0.125, real_count=g.real_count)
+        assert (a.keep == t.keep).all()
+        np.testing.assert_allclose(t.mass, a.scores, rtol=1e-12)
+
+
+def test_token_topp_hand_row():
+    # blocks 0 and 1 share one pooled logit, block 2's is ln 0.5 lower; block 0 holds 96
+    # tokens and blocks 1, 2 hold 32 each, so the token masses are 96, 32 and 16 over 144
+    # (0.667, 0.222, 0.111) although blocks 0 and 1 tie by score.  At p = 0.6 block 0
+    # alone reaches p by token mass.
+    nB = 3
+    logits = np.log(np.array([1.0, 1.0, 0.5]))
+    Qp = np.tile(logits, (nB, 1))[None, None]
+    counts = np.array([96, 32, 32])
+    r = O.route(Qp, np.eye(nB)[None, None], 0.6, 1, 1.0, real_count=counts)
+    np.testing.assert_allclose(r.mass[0, 0, 2], np.array([96, 32, 16]) / 144.0)
+    assert r.keep[0, 0, 2].astype(int).tolist() == [1, 0, 1]     # block 0, plus own 2
+    # the plain block rule needs both tied blocks (scores 0.4, 0.4, 0.2)
+    r0 = O.route(Qp, np.eye(nB)[None, None], 0.6, 1, 1.0)
+    assert r0.keep[0, 0, 2].astype(int).tolist() == [1, 1, 1]
+
+
+def test_keyframe_blocks_hand_cases():
+    g = O.block_geometry(10, 4, 4, 1, 4, 4)         # 10 frames, one block per frame
+    assert np.nonzero(O.keyframe_blocks(g, 4, 1))[0].tolist() == [1, 5, 9]
+    assert np.nonzero(O.keyframe_blocks(g, 4, 0))[0].tolist() == [0, 4, 8]
+    assert np.nonzero(O.keyframe_blocks(g, 20, 0))[0].tolist() == [0]
+    assert not O.keyframe_blocks(g, 0, 0).any()
+    g2 = O.block_geometry(7, 4, 8, 2, 4, 4)         # 2-frame blocks, 4 time blocks x 2 columns
+    # keyframes 1 and 4 (stride 3, phase 1; frame 7 does not exist): time blocks 0 and 2
+    assert np.nonzero(O.keyframe_blocks(g2, 3, 1))[0].tolist() == [0, 1, 4, 5]
+    # phase 2: frames 2 and 5 -> time blocks 1 and 2
+    assert np.nonzero(O.keyframe_blocks(g2, 3, 2))[0].tolist() == [2, 3, 4, 5]
+    keep = np.zeros((1, 1, 8, 8), bool)
+    keep[..., 3, 6] = True
+    got = O.add_keyframes(keep, O.keyframe_blocks(g2, 3, 2))
+    assert np.nonzero(got[0, 0, 3])[0].tolist() == [2, 3, 4, 5, 6]
+    assert np.nonzero(got[0, 0, 0])[0].tolist() == [2, 3, 4, 5]
+
+
+def test_keyframes_do_not_move_the_topp_cut():
+    w = W.SMALL_RAGGED
+    x = W.generate(w)
+    g = O.block_geometry(w.T, w.Hs, w.Ws, w.bt, w.bh, w.bw)
+    Qp, Kp = O.pool(x["q"], g), O.pool(x["k"], g)
+    r = O.route(Qp, Kp, 0.8, 2, 1 / math.sqrt(w.d))
+    kf = O.keyframe_blocks(g, 2, 1)
+    got = O.add_keyframes(r.keep, kf)
+    assert (got == (r.keep | kf)).all() and got[..., kf].all()
+
+
+def _repair_by_coordinates(keep, g):
+    out = keep.copy()
+    for j in range(g.nB):
+        tb, r = divmod(j, g.nBy * g.nBx)
+        yb, xb = divmod(r, g.nBx)
+        for dt, dy, dx in ((1, 0, 0), (0, 1, 0), (0, 0, 1)):
+            a = (tb - dt, yb - dy, xb - dx)
+            c = (tb + dt, yb + dy, xb + dx)
+            if min(a) < 0 or c[0] >= g.nBt or c[1] >= g.nBy or c[2] >= g.nBx:
+                continue
+            ja = (a[0] * g.nBy + a[1]) * g.nBx + a[2]
+            jc = (c[0] * g.nBy + c[1]) * g.nBx + c[2]
+            out[..., j] |= keep[..., ja] & keep[..., jc]
+    return out
+
+
+def test_repair_mask_against_coordinate_loops():
+    rng = np.random.default_rng(3)
+    for dims in [(4, 3, 5), (1, 1, 7), (3, 1, 1), (2, 4, 4)]:
+        g = O.block_geometry(dims[0] * 2, dims[1] * 4, dims[2] * 8 - 3, 2, 4, 8)
+        assert (g.nBt, g.nBy, g.nBx) == dims
+        for dens in (0.2, 0.5, 0.8):
+            keep = rng.random((2, 3, g.nB, g.nB)) < dens
+            np.testing.assert_array_equal(O.repair_mask(keep, g), _repair_by_coordinates(keep, g))
+
+
+def test_repair_mask_hand_case():
+    g = O.block_geometry(1, 1, 5, 1, 1, 1)          # five blocks in a row (x axis)
+    keep = np.array([1, 0, 1, 0, 0], bool)[None, None, None, :]
+    # block 1 is a hole between kept 0 and 2; block 3 is not (4 is dropped); one pass only
+    assert O.repair_mask(keep, g)[0, 0, 0].astype(int).tolist() == [1, 1, 1, 0, 0]
+    keep2 = np.array([1, 0, 1, 0, 1], bool)[None, None, None, :]
+    assert O.repair_mask(keep2, g)[0, 0, 0].astype(int).tolist() == [1, 1, 1, 1, 1]
+    # blocks at the ends of an axis have no hole to fill
+    keep3 = np.array([0, 1, 0, 0, 1], bool)[None, None, None, :]
+    assert O.repair_mask(keep3, g)[0, 0, 0].astype(int).tolist() == [0, 1, 0, 0, 1]
