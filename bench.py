@@ -506,8 +506,46 @@ def run_reference(args):
             "e2e": {"value": round(value, 6), "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def _graph_of(fn, stream):
+    """Captures fn() once in a CUDA graph (after one uncaptured run on a side stream)."""
+    import torch
+    side = torch.cuda.Stream()
+    side.wait_stream(stream)
+    with torch.cuda.stream(side):
+        fn()
+    stream.wait_stream(side)
+    gr = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(gr):
+        fn()
+    return gr
+
+
+def _timed_replays(gr, prepare, flush, reps, direct=None):
+    """Device times of `reps` replays of gr, each in its place in a layer: L2 flushed, then
+    prepare() (pool and route for the point, untimed; it also absorbs the write-back of the
+    flush's dirty lines), then the timed replay.  With `direct`, the same for a direct call
+    of the function the graph holds.  Returns (replay times, direct times)."""
+    import torch
+    ts, td = [], []
+    for i in range(3 + reps):
+        for fn, out in ((lambda: gr.replay(), ts),) + (((direct, td),) if direct else ()):
+            a = torch.cuda.Event(enable_timing=True)
+            b = torch.cuda.Event(enable_timing=True)
+            flush.fill_(float(i))
+            prepare()
+            a.record()
+            fn()
+            b.record()
+            torch.cuda.synchronize()
+            if i >= 3:
+                out.append(a.elapsed_time(b))
+    return ts, td
+
+
 def run_sweep(args, local_rank):
-    """Config-5 sweep: p x k_floor at the 480p shape; one JSON line per point (stdout)."""
+    """Config-5 sweep: p x k_floor at the 480p shape; one JSON line per point (stdout).  Each
+    point times the attention call as the headline does: a graph replay after an L2 flush,
+    pool and route; the direct (uncaptured) call is timed the same way beside it."""
     import torch
     import free_adaptive_block_b200 as fv
     torch.cuda.set_device(local_rank)
@@ -521,46 +559,106 @@ def run_sweep(args, local_rank):
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
     real = MX.real_counts(wl0.T, wl0.Hs, wl0.Ws, wl0.bt, wl0.bh, wl0.bw)
     peaks = load_peaks()
-
-    def timed(fn, p, k_floor, reps):
-        """Median device time of one call in its place in the layer, as on the headline
-        line: L2 flushed, then pool and route for this point (untimed; they also absorb
-        the write-back of the flush's dirty lines), then the timed call."""
-        ts = []
-        for i in range(3 + reps):
-            a = torch.cuda.Event(enable_timing=True)
-            b = torch.cuda.Event(enable_timing=True)
-            flush.fill_(float(i))
-            fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
-            fv.fvattn_route(g, buf.q_pool, buf.k_pool, p, k_floor, scale, buf.mask, buf.counts)
-            a.record()
-            fn()
-            b.record()
-            torch.cuda.synchronize()
-            if i >= 3:
-                ts.append(a.elapsed_time(b))
-        return statistics.median(ts)
-
-    dense_ms = timed(lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace),
-                     wl0.p, wl0.k_floor, args.steps)
+    stream = torch.cuda.current_stream(dev)
+    attn = lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,  # noqa: E731
+                                               buf.workspace, buf.sm_busy_ns)
+    dense = lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace)  # noqa: E731
+    route = lambda p, kf: fv.fvattn_pool_route(g, q, k, p, kf, scale, buf.q_pool, buf.k_pool,  # noqa: E731
+                                               buf.mask, buf.counts, buf.pool_route_ws)
+    route(wl0.p, wl0.k_floor)
+    dense_ts, _ = _timed_replays(_graph_of(dense, stream), lambda: route(wl0.p, wl0.k_floor), flush, args.steps)
+    dense_ms = statistics.median(dense_ts)
+    attn_graph = None
     for wl in W.sweep():
-        fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
-        fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale, buf.mask, buf.counts)
+        route(wl.p, wl.k_floor)
         torch.cuda.synchronize()
         keep = MX.unpack_words(buf.mask.cpu().numpy().view(np.uint32), g.nB)
         eff = MX.effective_flops(keep, real, wl.d)
-        ms = timed(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
-                                                        buf.workspace, buf.sm_busy_ns),
-                   wl.p, wl.k_floor, args.steps)
+        if attn_graph is None:
+            attn_graph = _graph_of(attn, stream)   # the mask buffer is an input: one graph serves
+        ts, td = _timed_replays(attn_graph, lambda: route(wl.p, wl.k_floor), flush, args.steps, direct=attn)
+        ms, ms_direct = statistics.median(ts), statistics.median(td)
         busy = buf.sm_busy_ns.cpu().numpy()
         busy = busy[busy > 0]
         print(json.dumps({"sweep_point": wl.name, "p": wl.p, "k_floor": wl.k_floor,
                           "kept_block_frac": round(float(keep.mean()), 4), "attn_ms": round(ms, 4),
+                          "attn_ms_direct_call": round(ms_direct, 4),
                           "effective_tflops": round(eff / (ms * 1e-3) / 1e12, 2),
                           "frac_of_bf16_peak": round(eff / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
                           "dense_attn_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / ms, 3),
+                          "timing": "graph replay after L2 flush + pool + route (median); direct call beside it",
                           "sm_busy_max_over_mean": (round(float(busy.max() / busy.mean()), 4)
                                                     if busy.size else None)}), flush=True)
+
+
+def run_next(args, local_rank):
+    """The rows beyond Top-p / Top-k routing, one JSON line each: keyframe blocks at the 6x
+    horizon, Top-p over tokens, runtime mask repair and slack-aware augmentation at 480p.
+    Each line reports the kept fraction, the attention time (graph replay after L2 flush
+    and the row's routing), and its speedup over the dense path on the same inputs."""
+    import torch
+    import free_adaptive_block_b200 as fv
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    peaks = load_peaks()
+    stream = torch.cuda.current_stream(dev)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)
+    for wl, modes in ((W.WAN21_6X, ("plain", "keyframes")),
+                      (W.WAN21_480P, ("plain", "token_mass", "repair", "slack_augment"))):
+        g = fv.Geometry(**wl.geom())
+        scale = float(np.float32(1.0 / math.sqrt(wl.d)))
+        x = W.generate(wl)
+        q, k, v = (torch.from_numpy(W.bf16_bits(x[n])).view(torch.bfloat16).to(dev) for n in ("q", "k", "v"))
+        del x
+        buf = fv.LayerBuffers.allocate(g, dev)
+        real = MX.real_counts(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+        attn = lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,  # noqa: E731
+                                                   buf.workspace, buf.sm_busy_ns)
+        dense = lambda: fv.fvattn_dense_attn(g, q, k, v, scale, buf.out, buf.lse, buf.workspace)  # noqa: E731
+        base_opts = dict(p=wl.p, k_floor=wl.k_floor, scale=scale)
+        tau = 1.0 / g.nB                        # a block above the uniform score
+
+        def prepare(mode):
+            fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool)
+            o = dict(base_opts)
+            if mode == "keyframes":
+                o.update(kf_stride=20, kf_phase=0)
+            elif mode == "token_mass":
+                o.update(token_mass=1)
+            elif mode == "repair":
+                o.update(repair=1)
+            fv.fvattn_route_ex(g, buf.q_pool, buf.k_pool, fv.RouteOpts(**o), buf.mask, buf.counts, buf.route_ws)
+            if mode == "slack_augment":
+                fv.fvattn_slack_augment(g, buf.route_ws, tau, buf.mask, buf.counts, buf.workspace)
+
+        prepare("plain")
+        dense_reps = 2 if wl.N > 100000 else 6
+        dense_ms = statistics.median(_timed_replays(_graph_of(dense, stream), lambda: prepare("plain"), flush,
+                                                    dense_reps)[0])
+        gr = _graph_of(attn, stream)
+        for mode in modes:
+            prepare(mode)
+            torch.cuda.synchronize()
+            keep = MX.unpack_words(buf.mask.cpu().numpy().view(np.uint32), g.nB)
+            eff = MX.effective_flops(keep, real, wl.d)
+            reps = min(args.steps, 5 if wl.N > 100000 else 10)
+            ts, _ = _timed_replays(gr, lambda: prepare(mode), flush, reps)
+            ms = statistics.median(ts)
+            busy = buf.sm_busy_ns.cpu().numpy()
+            busy = busy[busy > 0]
+            line = {"next_row": mode, "workload": wl.name, "p": wl.p, "k_floor": wl.k_floor,
+                    "kept_block_frac": round(float(keep.mean()), 4), "attn_ms": round(ms, 4),
+                    "effective_tflops": round(eff / (ms * 1e-3) / 1e12, 2),
+                    "frac_of_bf16_peak": round(eff / (ms * 1e-3) / 1e12 / peaks["bf16"], 4),
+                    "dense_attn_ms": round(dense_ms, 4), "speedup_vs_dense": round(dense_ms / ms, 3),
+                    "sm_busy_max_over_mean": round(float(busy.max() / busy.mean()), 4) if busy.size else None}
+            if mode == "keyframes":
+                line["keyframes"] = "stride 20, phase 0 (latent frames 0, 20, ..., 120)"
+            if mode == "slack_augment":
+                line["tau"] = tau
+            print(json.dumps(line), flush=True)
+        del buf, q, k, v
+        torch.cuda.empty_cache()
 
 
 def main():
@@ -570,6 +668,8 @@ def main():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
     ap.add_argument("--sweep", action="store_true", help="also time the 15 p/k points (config 5)")
+    ap.add_argument("--next", dest="next_rows", action="store_true",
+                    help="also time keyframes (6x), Top-p over tokens, mask repair, slack augmentation (480p)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--all-configs", action="store_true",
                     help="after the 480p line, one line per other workload (tiny, 720p, 6x horizon)")
@@ -608,6 +708,8 @@ def main():
                 print(json.dumps(extra), flush=True)
         if args.sweep and rank == 0:
             run_sweep(args, local_rank)
+        if args.next_rows and rank == 0:
+            run_next(args, local_rank)
     finally:
         if world > 1:
             import torch

@@ -27,7 +27,7 @@ __all__ = [
     "Geometry", "FvattnError", "lib", "fvattn_num_blocks", "fvattn_block_pool", "fvattn_route",
     "fvattn_attn_workspace_size", "fvattn_num_sms", "fvattn_block_sparse_attn",
     "fvattn_route_workspace_size", "fvattn_route_ws", "fvattn_pool_route_workspace_size",
-    "fvattn_pool_route", "RouteOpts", "fvattn_route_ex", "fvattn_mask_repair",
+    "fvattn_pool_route", "RouteOpts", "fvattn_route_ex", "fvattn_mask_repair", "fvattn_slack_augment",
     "fvattn_dense_attn", "fvattn_block_sparse_attn_noalloc", "fvattn_noalloc_device_status", "fvattn_device_status", "fvattn_status_string", "attention_layer",
     "LayerBuffers", "LayerGraph", "HostPipeline",
 ]
@@ -128,6 +128,9 @@ _SIGS = {
                                        ctypes.c_void_p]),
     "fvattn_mask_repair": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                           ctypes.c_void_p]),
+    "fvattn_slack_augment": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_size_t, ctypes.c_float,
+                                            ctypes.c_int, ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
+                                            ctypes.c_size_t, ctypes.c_void_p]),
     "fvattn_testing_attn_stall": (ctypes.c_int, [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_float,
                                                  ctypes.c_void_p, ctypes.c_void_p, ctypes.c_void_p,
@@ -263,6 +266,19 @@ def fvattn_mask_repair(g: Geometry, mask_in, mask_out, counts, stream=None) -> N
     _ok("fvattn_mask_repair", lib().fvattn_mask_repair(
         ctypes.byref(cg), _ptr(mask_in, torch.int32, shape, "mask_in"), _ptr(mask_out, torch.int32, shape, "mask_out"),
         _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"), _stream(stream)))
+
+
+def fvattn_slack_augment(g: Geometry, route_workspace, tau: float, mask, counts, scratch, n_sm: int = 0,
+                         stream=None) -> None:
+    """Slack-aware augmentation of the final wave of tiles, in place on mask and counts;
+    route_workspace holds the logits of the route call that wrote the mask."""
+    import torch
+    cg = g.c()
+    _ok("fvattn_slack_augment", lib().fvattn_slack_augment(
+        ctypes.byref(cg), _ptr(route_workspace, torch.uint8, None, "route_workspace"), route_workspace.numel(),
+        float(tau), int(n_sm), _ptr(mask, torch.int32, (g.B, g.H, g.nB, g.words), "mask"),
+        _ptr(counts, torch.int32, (g.B, g.H, g.nB), "counts"), _ptr(scratch, torch.uint8, None, "scratch"),
+        scratch.numel(), _stream(stream)))
 
 
 def fvattn_pool_route_workspace_size(g: Geometry) -> int:

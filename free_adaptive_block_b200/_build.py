@@ -9,7 +9,7 @@ PKG = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(PKG)
 CSRC = os.path.join(PKG, "csrc")
 LIB = os.path.join(PKG, "libfvattn.so")
-SOURCES = ["fv_api.cu", "fv_pool_route.cu", "fv_route_tc.cu", "fv_attn.cu"]
+SOURCES = ["fv_api.cu", "fv_pool_route.cu", "fv_route_tc.cu", "fv_augment.cu", "fv_attn.cu"]
 
 
 def nvcc() -> str:

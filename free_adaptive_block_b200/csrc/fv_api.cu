@@ -85,6 +85,25 @@ PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
   return fn;
 }
 
+}  // namespace
+
+// 3D map over an fp32 [slices][rows][d] array (pooled rows split for the tensor cores): box
+// 32 channels x 128 rows x 1 slice, 128-byte swizzle, rows past the slice's end read zero.
+bool fv::encode_rows_fp32(CUtensorMap* m, const void* ptr, int slices, int rows, int d) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  cuuint64_t dims[3] = {static_cast<cuuint64_t>(d), static_cast<cuuint64_t>(rows), static_cast<cuuint64_t>(slices)};
+  cuuint64_t strides[2] = {static_cast<cuuint64_t>(d) * 4, static_cast<cuuint64_t>(rows) * d * 4};
+  cuuint32_t box[3] = {32u, 128u, 1u};
+  cuuint32_t estr[3] = {1, 1, 1};
+  const CUresult r = fn(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 3, const_cast<void*>(ptr), dims, strides, box, estr,
+                        CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                        CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+namespace {
+
 // 5D map over a bf16 [B*H][T][Hs][Ws][d] tensor; box = 64 channels x box_x columns x
 // bh rows x bt frames x 1 slice, 128-byte swizzle, zero fill out of range.
 bool encode_map(CUtensorMap* m, const void* ptr, const Geo& g, int box_x) {
@@ -131,13 +150,36 @@ fvattn_status_t run_attn(const fvattn_geom_t* gi, const void* q, const void* k, 
   if (reinterpret_cast<uintptr_t>(ws) & 15u) return FVATTN_ERR_UNSUPPORTED;
   const int nsm = current_num_sms();
   if (nsm <= 0) return cuda_status(cudaGetLastError() == cudaSuccess ? cudaErrorNoDevice : cudaGetLastError());
-  const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
-  fv::AttnMaps maps;
-  if (!encode_map(&maps.q, q, g, g.bw) || !encode_map(&maps.qe, q, g, rx_edge) ||
-      !encode_map(&maps.k, k, g, g.bw) || !encode_map(&maps.ke, k, g, rx_edge) ||
-      !encode_map(&maps.v, v, g, g.bw) || !encode_map(&maps.ve, v, g, rx_edge))
-    return FVATTN_ERR_CUDA;
-  return cuda_status(fv::launch_attn(g, maps, mask, scale, out, lse, ws, busy, nsm,
+  // The six tensor maps depend only on the geometry and the Q, K, V addresses: a thread
+  // keeps the last set it encoded and reuses it while they stay the same.
+  struct MapCache {
+    unsigned long long ctx;
+    const void *q, *k, *v;
+    fvattn_geom_t g;
+    fv::AttnMaps maps;
+    bool valid;
+  };
+  thread_local MapCache mc = {};
+  const unsigned long long ctx = fv::current_ctx_id();
+  const bool hit = mc.valid && ctx != 0 && mc.ctx == ctx && mc.q == q && mc.k == k && mc.v == v &&
+                   mc.g.B == gi->B && mc.g.H == gi->H && mc.g.T == gi->T && mc.g.Hs == gi->Hs &&
+                   mc.g.Ws == gi->Ws && mc.g.d == gi->d && mc.g.bt == gi->bt && mc.g.bh == gi->bh &&
+                   mc.g.bw == gi->bw;
+  if (!hit) {
+    const int rx_edge = g.Ws - (g.nBx - 1) * g.bw;
+    mc.valid = false;
+    if (!encode_map(&mc.maps.q, q, g, g.bw) || !encode_map(&mc.maps.qe, q, g, rx_edge) ||
+        !encode_map(&mc.maps.k, k, g, g.bw) || !encode_map(&mc.maps.ke, k, g, rx_edge) ||
+        !encode_map(&mc.maps.v, v, g, g.bw) || !encode_map(&mc.maps.ve, v, g, rx_edge))
+      return FVATTN_ERR_CUDA;
+    mc.ctx = ctx;
+    mc.q = q;
+    mc.k = k;
+    mc.v = v;
+    mc.g = *gi;
+    mc.valid = true;
+  }
+  return cuda_status(fv::launch_attn(g, mc.maps, mask, scale, out, lse, ws, busy, nsm,
                                      reinterpret_cast<cudaStream_t>(stream), stall_ns));
 }
 
@@ -158,7 +200,9 @@ NoAllocSlot g_noalloc_slot[kMaxDevices] = {};
 // Identifier of the calling thread's current driver context (0 when there is none).  A
 // device reset or a new context loads the library's module again, and the static array
 // may then sit at another address, so the cached address is keyed on this identifier.
-unsigned long long current_ctx_id() {
+}  // namespace
+
+unsigned long long fv::current_ctx_id() {
   static PFN_cuCtxGetCurrent_v4000 get_cur = nullptr;
   static PFN_cuCtxGetId_v12000 get_id = nullptr;
   static std::once_flag once;
@@ -181,6 +225,8 @@ unsigned long long current_ctx_id() {
   return id;
 }
 
+namespace {
+
 // Device address of g_noalloc_scratch in the current context.  Host code only holds a
 // host-side stand-in for the symbol, so the address is asked of the runtime
 // (cudaGetSymbolAddress) the first time a device's context is seen, and again whenever
@@ -192,13 +238,13 @@ fvattn_status_t noalloc_scratch(void** out) {
   if (dev < 0 || dev >= kMaxDevices) return FVATTN_ERR_UNSUPPORTED;
   std::lock_guard<std::mutex> lock(g_noalloc_mu);
   NoAllocSlot& slot = g_noalloc_slot[dev];
-  const unsigned long long id = current_ctx_id();
+  const unsigned long long id = fv::current_ctx_id();
   if (slot.addr == nullptr || id == 0 || id != slot.ctx_id) {
     void* p = nullptr;
     st = cuda_status(cudaGetSymbolAddress(&p, g_noalloc_scratch));
     if (st != FVATTN_OK) return st;
     slot.addr = p;
-    slot.ctx_id = current_ctx_id();   // the runtime call made the primary context current
+    slot.ctx_id = fv::current_ctx_id();   // the runtime call made the primary context current
   }
   *out = slot.addr;
   return FVATTN_OK;
@@ -295,6 +341,30 @@ fvattn_status_t fvattn_route_ex(const fvattn_geom_t* gi, const float* q_pool, co
                                                       workspace, st, o));
   if (s != FVATTN_OK || !opts->repair) return s;
   return cuda_status(fv::launch_mask_repair(g, mask, mask, counts, st));
+}
+
+fvattn_status_t fvattn_slack_augment(const fvattn_geom_t* gi, const void* route_workspace, size_t route_ws_bytes,
+                                     float tau, int n_sm, uint32_t* mask, int32_t* counts, void* scratch,
+                                     size_t scratch_bytes, fvattn_stream_t stream) {
+  Geo g;
+  FV_CHECK(make_geo(gi, &g));
+  FV_CHECK(check_ptr4(mask));
+  FV_CHECK(check_ptr4(counts));
+  if (!(tau >= 0.f) || !isfinite(tau)) return FVATTN_ERR_INVALID_ARG;
+  if (n_sm < 0) return FVATTN_ERR_INVALID_ARG;
+  // tile costs (real query tokens x real key tokens) are held in 26 bits
+  if (static_cast<long long>(g.bt) * g.bh * g.bw * g.N >= (1LL << 26)) return FVATTN_ERR_UNSUPPORTED;
+  if (route_workspace == nullptr || route_ws_bytes < fv::route_ws_bytes(g)) return FVATTN_ERR_WORKSPACE;
+  if (scratch == nullptr || scratch_bytes < fv::augment_scratch_bytes(g)) return FVATTN_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(route_workspace) | reinterpret_cast<uintptr_t>(scratch)) & 15u)
+    return FVATTN_ERR_UNSUPPORTED;
+  if (n_sm == 0) {
+    n_sm = current_num_sms();
+    if (n_sm <= 0) return cuda_status(cudaGetLastError() == cudaSuccess ? cudaErrorNoDevice : cudaGetLastError());
+  }
+  const float* logits = reinterpret_cast<const float*>(static_cast<const unsigned char*>(route_workspace) + 256);
+  return cuda_status(fv::launch_augment(g, logits, tau, n_sm, mask, counts, scratch,
+                                        reinterpret_cast<cudaStream_t>(stream)));
 }
 
 fvattn_status_t fvattn_mask_repair(const fvattn_geom_t* gi, const uint32_t* mask_in, uint32_t* mask_out,

@@ -51,16 +51,16 @@ constexpr int kMaxBlocks = 2048;       // blocks per (b, h) slice, the mask row 
 constexpr int kTR = 2;                 // tile-id ring depth
 constexpr int kChunkBytes = 128 * 128; // 128 rows x 64 bf16 (one 128-byte swizzle column)
 constexpr uint32_t kTmemCols = 512;
-// Tensor memory (512 columns x 128 lanes, lane = query row): two S slots of 128 fp32
-// columns, O (d columns) and two P slots of 64 columns (bf16 pairs).  An S slot is
-// free as soon as its softmax group has loaded it into registers, and P_c only waits
-// for the P.V two blocks back, so no tensor-core product waits on the one before it.
-constexpr int kNS = 2;                 // S ring depth
-constexpr int kNP = 2;                 // P ring depth
-constexpr uint32_t kColS = 0;          // S slot r: columns [128r, 128r+128)
-constexpr uint32_t kColO = 128 * kNS;  // O: columns [256, 256 + d)
-template <int D> __host__ __device__ constexpr uint32_t col_p() { return kColO + D; }   // P slot r: +64r
-static_assert(col_p<128>() + 64 * kNP <= 512, "tensor memory layout exceeds 512 columns");
+// Tensor memory (512 columns x 128 lanes, lane = query row): three S slots of 128 fp32
+// columns and O (d columns).  P_c (bf16 pairs, 64 columns) is written over S_c in its
+// own slot: the softmax group holds the whole row of S_c in registers before it stores
+// any P, so nothing else waits for a P slot.  S slot c mod 3 takes S_c+3 once P.V c has
+// read P_c, three blocks of slack for the tensor core.
+constexpr int kNS = 3;                 // S / P ring depth
+constexpr int kPV = 6;                 // P.V completion barriers (block c commits [c % 6])
+constexpr uint32_t kColS = 0;          // S slot r: columns [128r, 128r+128), P_c over its first 64
+constexpr uint32_t kColO = 128 * kNS;  // O: columns [384, 384 + d)
+static_assert(kColO + 128 <= 512, "tensor memory layout exceeds 512 columns");
 constexpr float kRebase = 8.0f;        // lazy re-basing threshold, log2 units
 
 __device__ __forceinline__ float max3f(float a, float b, float c) {
@@ -91,11 +91,12 @@ struct __align__(8) AttnBars {
   uint64_t q_full, q_empty;
   uint64_t k_full[kNK], k_empty[kNK];
   uint64_t v_full[kNV], v_empty[kNV];
-  uint64_t s_full[kNS];   // per S slot: written by the MMA ...
-  uint64_t s_empty[kNS];  //   ... and loaded into registers by its softmax group
-  uint64_t p_full[kNP];   // per P slot
-  uint64_t pv_done[3];    // P.V of block c commits [c % 3]: a group waiting for P.V c-1 or
-                          // c-2 has itself seen P.V c-4 complete, so no wait aliases a phase
+  uint64_t s_full[kNS];   // per S slot: S_c written by the MMA
+  uint64_t p_full[kNS];   // per S slot: P_c stored over S_c by the softmax group
+  uint64_t pv_done[kPV];  // P.V of block c commits [c % 6].  A wait for P.V x on it needs
+                          // P.V x-6 complete; every waiter knows P.V c-3 complete for a
+                          // block c it has seen S of (S_c is issued only after P.V c-3),
+                          // and waits only for P.V of c-3 .. c, so no wait aliases a phase
   uint64_t o_empty;
   uint64_t hb[2][4];      // reference hand-off, [writing group][TMEM lane quarter]
   uint64_t xbar[4];       // end-of-tile row-sum exchange, per TMEM lane quarter: written
@@ -230,10 +231,9 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     for (int i = 0; i < kNV; ++i) { mbar_init(&bars.v_full[i], 1); mbar_init(&bars.v_empty[i], 1); }
     for (int i = 0; i < kNS; ++i) {
       mbar_init(&bars.s_full[i], 1);
-      mbar_init(&bars.s_empty[i], kSoftWarps / 2);
+      mbar_init(&bars.p_full[i], kSoftWarps / 2);
     }
-    for (int i = 0; i < kNP; ++i) mbar_init(&bars.p_full[i], kSoftWarps / 2);
-    for (int i = 0; i < 3; ++i) mbar_init(&bars.pv_done[i], 1);
+    for (int i = 0; i < kPV; ++i) mbar_init(&bars.pv_done[i], 1);
     for (int i = 0; i < 4; ++i) {
       mbar_init(&bars.xbar[i], 2);
       mbar_init(&bars.xread[i], 2);
@@ -453,7 +453,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
    } else if (warp == 1) {
     // ------------------------------------------------------------ S issuer
     // Block j of the call's running block count c: S_c = Q K_c^T into S slot c mod kNS,
-    // once the softmax group has loaded S_c-kNS out of it.  The S and the P.V products come
+    // once P.V c-kNS has read P_c-kNS out of it.  The S and the P.V products come
     // from two warps: an MMA issue blocks while the tensor core's queue is full, so one
     // warp's waits and bookkeeping overlap the other warp's issue.
     uint32_t tcount = 0, mqc = 0;
@@ -482,7 +482,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const ItemRange ir = item_range(n, nw, nn, prm.pack);
         const uint32_t idesc_s = idesc_bf16_f32(128, item_npad(bars.blist[slot], n, nw, ir, prm.rows_e), 0, 0);
         if (!wwait(&bars.k_full[ks], (c / kNK) & 1)) { ok = false; break; }
-        if (c >= kNS && !wwait(&bars.s_empty[ss], ((c - kNS) / kNS) & 1)) { ok = false; break; }
+        if (c >= kNS && !wwait(&bars.pv_done[(c - kNS) % kPV], ((c - kNS) / kPV) & 1)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dK = dK0 + static_cast<uint64_t>((ks * TILE) >> 4);
         const uint32_t tS = tmem + kColS + ss * 128;
@@ -505,7 +505,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     }
    } else if (warp == 2) {
     // ------------------------------------------------------------ P.V issuer
-    // O += P_c V_c in block order (one accumulator), P_c from P slot c mod kNP.
+    // O += P_c V_c in block order (one accumulator), P_c from S slot c mod kNS.
     uint32_t tcount = 0, tiles = 0;
     uint32_t gc = 0;
     const uint32_t idesc_pv = idesc_bf16_f32(128, D, 0, 1);
@@ -522,15 +522,15 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       int n = 0;
       for (; n < nitems; ++n) {
         const uint32_t c = gc + n;
-        const int ps = c % kNP;
+        const int ps = c % kNS;
         const int vs = c % kNV;
         const int nk = item_npad(bars.blist[slot], n, nw, item_range(n, nw, nn, prm.pack), prm.rows_e) >> 4;
-        if (!wwait(&bars.p_full[ps], (c / kNP) & 1)) { ok = false; break; }
+        if (!wwait(&bars.p_full[ps], (c / kNS) & 1)) { ok = false; break; }
         if (!wwait(&bars.v_full[vs], (c / kNV) & 1)) { ok = false; break; }
         if (n == 0 && !wwait(&bars.o_empty, (tiles & 1) ^ 1)) { ok = false; break; }
         tc_fence_after();
         const uint64_t dV = dV0 + static_cast<uint64_t>((vs * TILE) >> 4);
-        const uint32_t tP = tmem + col_p<D>() + ps * 64;
+        const uint32_t tP = tmem + kColS + ps * 128;
         if (elect_one()) {
 #pragma unroll
           for (int q = 0; q < 8; ++q) {
@@ -539,7 +539,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
                      (n == 0 && q == 0) ? 0u : 1u);
           }
           mma_commit(&bars.v_empty[vs]);
-          mma_commit(&bars.pv_done[c % 3]);
+          mma_commit(&bars.pv_done[c % kPV]);
         }
         __syncwarp();
       }
@@ -566,7 +566,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
     const int row = quarter * 32 + lane;
     const uint32_t lane_off = static_cast<uint32_t>(quarter * 32) << 16;
     const uint32_t tS0 = tmem + lane_off + kColS;
-    const uint32_t tP0 = tmem + lane_off + col_p<D>();
     const uint32_t tO = tmem + lane_off + kColO;
     uint32_t tcount = 0, xn = 0, hr = 0;
     uint32_t gc = 0;                    // blocks of all earlier tiles: S ring position
@@ -605,7 +604,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         const uint32_t c = gc + j;
         const int ss = c % kNS;
         const uint32_t tS = tS0 + ss * 128;
-        const uint32_t tP = tP0 + (c % kNP) * 64;
+        const uint32_t tP = tS;                     // P_c goes over S_c
         const int npad = item_npad(bl, j, nw, ir, prm.rows_e);
         const int nact = (npad + 31) >> 5;          // 32-column chunks below npad (uniform)
         // member: this warp's query block keeps the item (some sub-block of a packed item)
@@ -639,7 +638,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         }
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.s_empty[ss]);    // the slot may take S_c+2
         // Keys that are not real tokens (a partial last 16-key group, or the gaps of a box
         // cut at the time and height edges at once) to -inf.  One warp-uniform branch,
         // taken only by such blocks, so the common path carries none of this code.
@@ -712,7 +710,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         if (__any_sync(0xffffffffu, rebase)) {
           const float alpha = rebase ? ex2(mp - mx) : 1.f;
           const uint32_t cp = c - 1;
-          if (!sync_wait(&bars.pv_done[cp % 3], (cp / 3) & 1)) { ok = false; break; }
+          if (!sync_wait(&bars.pv_done[cp % kPV], (cp / kPV) & 1)) { ok = false; break; }
           tc_fence_after();
 #pragma unroll 1
           for (int q = 0; q < D / 32; ++q) {
@@ -731,13 +729,6 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
           if (lscale) l *= ex2(m - mref);
         }
         m = mref;
-        // P slot c mod kNP is free once P.V c-kNP has read it (long done: it is this
-        // group's previous block)
-        if (c >= kNP) {
-          const uint32_t cp = c - kNP;
-          if (!sync_wait(&bars.pv_done[cp % 3], (cp / 3) & 1)) { ok = false; break; }
-          tc_fence_after();
-        }
         // P = 2^(s * scale * log2 e - m), packed to bf16 pairs and stored 16 keys at a
         // time (P column k/2 holds keys k, k+1).  Chunks at or past npad are neither
         // computed nor stored: the P.V reads keys < npad only.
@@ -774,7 +765,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
         tmem_wait_st();
         tc_fence_before();
         __syncwarp();
-        if (lane == 0) mbar_arrive(&bars.p_full[c % kNP]);
+        if (lane == 0) mbar_arrive(&bars.p_full[c % kNS]);
       }
       if (!ok) break;
       // ---- epilogue
@@ -788,7 +779,7 @@ __global__ void __launch_bounds__(kAttnThreads, 1)
       if (mf != m) l = (m == -INFINITY) ? 0.f : l * ex2(m - mf);
       if (nkv > 0) {
         const uint32_t cl = gc - 1;      // the tile's last P.V
-        if (!sync_wait(&bars.pv_done[cl % 3], (cl / 3) & 1)) break;
+        if (!sync_wait(&bars.pv_done[cl % kPV], (cl / kPV) & 1)) break;
       }
       if (xn > 0 && !sync_wait(&bars.xread[quarter], (xn - 1) & 1)) break;
       bars.xl[grp][row] = l;
@@ -1086,7 +1077,8 @@ template <int D>
 static cudaError_t launch_attn_d(const Geo& g, const AttnMaps& maps, const AttnParams& prm, int grid,
                                  cudaStream_t st) {
   constexpr int smem = attn_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(attn_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static SmemAttrCache attr_ctx = {};
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(attn_kernel<D>), smem, attr_ctx);
   if (e != cudaSuccess) return e;
   attn_kernel<D><<<grid, kAttnThreads, smem, st>>>(maps.q, maps.qe, maps.k, maps.ke, maps.v, maps.ve, prm);
   return cudaGetLastError();

@@ -307,35 +307,68 @@ __device__ __forceinline__ void select_row(const Geo& g, const RouteOpts& o, con
 // ----------------------------------------------------------------------------
 // Selection by mass histogram (the form fvattn_route_ws, fvattn_route_ex and
 // fvattn_pool_route use).  Same rule as select_row, with the masses summed exactly: every
-// block's mass exp(l - max) (times its real token count for the Top-p over tokens) is
+// block's mass 2^((l - max) log2 e) (times its real token count for the Top-p over tokens) is
 // rounded once to a fixed-point integer of 2^-32 units, and all sums are integer sums, so
 // they do not depend on summation order and the prefix test "mass >= p" reads
 // sum >= ceil(p * Z) in integers.  Per row (one warp):
-//   1. logits into registers (lane l holds blocks c * 32 + l), row maximum;
-//   2. a 256-bucket histogram of mass and count in shared memory, bucket
-//      b = min(255, floor((max - l) * 16)): buckets are contiguous ranges of the logit
-//      order, 1/16 logit wide, the last one holding everything 16 or more below the max
-//      (at most e^-16 of the row's mass per block);
+//   1. logits into registers (lane l holds blocks c * 32 + l) as order keys, row maximum;
+//   2. a 512-bucket histogram of mass and count in shared memory over t = (max - l) * 32:
+//      bucket floor(t), the last one holding everything 16 or more below the max (its
+//      sums are kept in registers: the blocks of a sparse row pile up there);
 //   3. a warp scan over the buckets finds the bucket where the prefix mass reaches p;
-//   4. that bucket's blocks (a few at these shapes) are gathered and ranked exactly by
-//      (logit desc, index asc); the cut is the first rank at which the prefix reaches p;
-//   5. the Top-k floor, when it lengthens the prefix, repeats 3-4 on counts;
-//   6. the mask: blocks above the cut's key, tied blocks up to the cut's index, the own
+//   4. when that bucket holds more than 32 blocks, a second histogram over its fraction
+//      of t (512 sub-buckets) narrows it;
+//   5. the bucket's blocks are gathered and ranked exactly by (logit desc, index asc); the
+//      cut is the first rank at which the prefix reaches p;
+//   6. the Top-k floor, when it lengthens the prefix, repeats 2-5 on counts;
+//   7. the mask: blocks above the cut's key, tied blocks up to the cut's index, the own
 //      block and keyframe blocks.
-// A bucket with more than kSelCap blocks (a cut far down a nearly flat tail) runs
-// select_row on the row instead.
+// A sub-bucket with more than 32 blocks (near-ties by the dozen) runs select_row.
 // ----------------------------------------------------------------------------
-constexpr int kSelBuckets = 256;
-constexpr float kSelPerLogit = 16.f;
-constexpr int kSelCap = 64;
+__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
+}
+__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
+template <int N>
+__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
-struct SelScratch {                      // one per warp
-  unsigned long long hm[kSelBuckets];    // mass per bucket (2^-32 units)
-  uint32_t hc[kSelBuckets];              // blocks per bucket
-  unsigned long long lw[kSelCap];        // gathered bucket: mass,
-  uint32_t lkey[kSelCap];                //   order key,
-  uint32_t lidx[kSelCap];                //   block index
+constexpr int kSelBuckets = 512;
+constexpr float kSelPerLogit = 32.f;
+constexpr int kSelCap = 32;             // gathered blocks: one per lane
+constexpr int kSelWarps = 4;            // rows (warps) per CTA
+
+// Shared memory of one warp (one row at a time): the mass histogram, the gathered list and
+// the row's order keys, lane l's keys in column l ([c][32], so a lane touches only its own
+// words and no synchronisation is needed for them).
+struct SelScratch {
+  uint32_t* hh;                          // mass per bucket (2^-32 units): high parts (w >> 20) ...
+  uint32_t* hl;                          //   ... and low parts (w & 0xfffff), both exact in 32 bits
+  uint32_t* hc;                          // blocks per bucket
+  unsigned long long* lw;                // gathered bucket: mass,
+  uint32_t* lkey;                        //   order key,
+  uint32_t* lidx;                        //   block index
+  uint32_t* key;                         // the row: key[c * 32 + lane] for block c * 32 + lane
 };
+
+__host__ __device__ constexpr size_t sel_warp_bytes(int words) {
+  return 3 * kSelBuckets * 4 + kSelCap * 8 + 2 * kSelCap * 4 + static_cast<size_t>(words) * 32 * 4;
+}
+
+__device__ __forceinline__ SelScratch sel_scratch(unsigned char* base) {
+  SelScratch sh;
+  sh.hh = reinterpret_cast<uint32_t*>(base);
+  sh.hl = sh.hh + kSelBuckets;
+  sh.hc = sh.hl + kSelBuckets;
+  sh.lw = reinterpret_cast<unsigned long long*>(sh.hc + kSelBuckets);
+  sh.lkey = reinterpret_cast<uint32_t*>(sh.lw + kSelCap);
+  sh.lidx = sh.lkey + kSelCap;
+  sh.key = sh.lidx + kSelCap;
+  return sh;
+}
+
+__device__ __forceinline__ float key_value(uint32_t k) {   // inverse of order_key
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
 
 __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
 #pragma unroll
@@ -343,30 +376,37 @@ __device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v)
   return v;
 }
 
-__device__ __forceinline__ int sel_bucket(float mx, float x) {
-  return min(kSelBuckets - 1, __float2int_rz((mx - x) * kSelPerLogit));
-}
-
 __device__ __forceinline__ unsigned long long sel_fixed(float w) {
   return __float2ull_rn(w * 4294967296.0f);
 }
 
+// Bucket coordinate of a logit: t = (max - x) * 32; level-0 bucket floor(t) (capped), and
+// inside level-0 bucket b0 the level-1 bucket floor((t - b0) * 512) (exact in fp32: t < 512
+// carries at most 14 fraction bits, so t - b0 and the scaling round nothing).
+__device__ __forceinline__ float sel_t(float mx, float x) { return (mx - x) * kSelPerLogit; }
+__device__ __forceinline__ int sel_b0(float t) { return min(kSelBuckets - 1, __float2int_rz(t)); }
+__device__ __forceinline__ int sel_b1(float t, int b0) {
+  return min(kSelBuckets - 1, __float2int_rz((t - static_cast<float>(b0)) * static_cast<float>(kSelBuckets)));
+}
+
+__device__ __forceinline__ unsigned long long sel_bucket_mass(const SelScratch& sh, int b) {
+  return (static_cast<unsigned long long>(sh.hh[b]) << 20) + sh.hl[b];
+}
+
 // Finds the bucket where the running sum (mass when `by_mass`, else count) first reaches
-// `target`, scanning buckets from the top of the order.  Returns the bucket and, through
-// `above`, the sum over the buckets before it (and `cnt_above`, their block count).
+// `target`, scanning buckets from the top of the order.  Lane l owns buckets 16 l .. 16 l + 15.
+// Returns the bucket; `above` / `cnt_above` get the sum and block count before it.
 __device__ __forceinline__ int sel_find_bucket(const SelScratch& sh, bool by_mass, unsigned long long target,
                                                unsigned long long& above, int& cnt_above, int lane) {
-  unsigned long long loc[8];
-  int cl[8];
+  constexpr int PER = kSelBuckets / 32;
   unsigned long long run = 0;
   int crun = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    const int b = lane * 8 + e;
-    cl[e] = static_cast<int>(sh.hc[b]);
-    loc[e] = by_mass ? sh.hm[b] : static_cast<unsigned long long>(cl[e]);
-    run += loc[e];
-    crun += cl[e];
+#pragma unroll 4
+  for (int e = 0; e < PER; ++e) {
+    const int b = lane * PER + e;
+    const uint32_t n = sh.hc[b];
+    run += by_mass ? sel_bucket_mass(sh, b) : static_cast<unsigned long long>(n);
+    crun += static_cast<int>(n);
   }
   unsigned long long incl = run;
   int cincl = crun;
@@ -381,15 +421,21 @@ __device__ __forceinline__ int sel_find_bucket(const SelScratch& sh, bool by_mas
   int found = kSelBuckets;
   unsigned long long f_above = 0;
   int f_cnt = 0;
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    if (found == kSelBuckets && excl + loc[e] >= target) {
-      found = lane * 8 + e;
-      f_above = excl;
-      f_cnt = cexcl;
+  if (incl >= target && excl < target) {      // the crossing lies in this lane's buckets
+#pragma unroll 1
+    for (int e = 0; e < PER; ++e) {
+      const int b = lane * PER + e;
+      const uint32_t n = sh.hc[b];
+      const unsigned long long v = by_mass ? sel_bucket_mass(sh, b) : static_cast<unsigned long long>(n);
+      if (excl + v >= target) {
+        found = b;
+        f_above = excl;
+        f_cnt = cexcl;
+        break;
+      }
+      excl += v;
+      cexcl += static_cast<int>(n);
     }
-    excl += loc[e];
-    cexcl += cl[e];
   }
   const uint32_t hit = __ballot_sync(0xffffffffu, found < kSelBuckets);
   const int src = hit ? __ffs(hit) - 1 : 31;
@@ -398,88 +444,129 @@ __device__ __forceinline__ int sel_find_bucket(const SelScratch& sh, bool by_mas
   return hit ? __shfl_sync(0xffffffffu, found, src) : kSelBuckets - 1;
 }
 
-template <int MAXW>
-__device__ __forceinline__ void select_row_hist(const Geo& g, const RouteOpts& o, const float* lrow, int nB,
-                                                int words, int qb, float p, int k_floor, uint32_t* mrow,
-                                                int32_t* cnt_out, int lane, SelScratch& sh) {
-  uint32_t key[MAXW];
-  float x[MAXW];
+__device__ void select_row_hist(const Geo& g, const RouteOpts& o, const float* lrow, int nB, int words, int qb,
+                                float p, int k_floor, uint32_t* mrow, int32_t* cnt_out, int lane,
+                                const SelScratch& sh) {
+  // the row's words * 32 logits into shared memory in one round trip (16-byte cp.async,
+  // all in flight), then each lane turns its column into order keys
+  {
+    const uint32_t dst = smem_u32(sh.key);
+    const int chunks = words * 8;            // 16-byte chunks of the row
+    for (int q = lane; q < chunks; q += 32) cp_async16(dst + q * 16, lrow + q * 4, 16u);
+    cp_async_commit();
+    cp_async_wait<0>();
+    __syncwarp();
+  }
+  uint32_t* key = sh.key + lane;   // this lane's column: key[c * 32]
   float mx = -INFINITY;
-#pragma unroll
-  for (int c = 0; c < MAXW; ++c) {
+#pragma unroll 4
+  for (int c = 0; c < words; ++c) {
     const int i = c * 32 + lane;
-    const bool v = c < words && i < nB;
-    x[c] = v ? __ldcg(lrow + i) : -INFINITY;
-    key[c] = v ? order_key(x[c]) : 0u;
-    mx = fmaxf(mx, x[c]);
+    const float x = i < nB ? __uint_as_float(key[c * 32]) : -INFINITY;
+    key[c * 32] = i < nB ? order_key(x) : 0u;
+    mx = fmaxf(mx, x);
   }
   mx = warp_max(mx);
-#pragma unroll
-  for (int e = 0; e < 8; ++e) {
-    sh.hm[lane * 8 + e] = 0ull;
-    sh.hc[lane * 8 + e] = 0u;
-  }
-  __syncwarp();
-  auto mass_of = [&](int c) -> float {
-    float w = expf(x[c] - mx);
+  const float nmx = -mx;
+  // a block's mass in 2^-32 units: 2^((x - max) log2 e), times its real token count for
+  // the Top-p over tokens; the same rounded operations wherever it is evaluated
+  auto mass_of = [&](int c, float x) -> unsigned long long {
+    float w = ex2(__fmul_rn(__fadd_rn(x, nmx), 1.4426950408889634f));
     if (o.token_mass) w *= static_cast<float>(block_info(g, c * 32 + lane).nvalid);
-    return w;
+    return sel_fixed(w);
   };
-  unsigned long long z = 0;
-#pragma unroll
-  for (int c = 0; c < MAXW; ++c) {
-    if (key[c] != 0u) {
-      const unsigned long long w = sel_fixed(mass_of(c));
-      const int b = sel_bucket(mx, x[c]);
-      atomicAdd(&sh.hm[b], w);
-      atomicAdd(&sh.hc[b], 1u);
-      z += w;
+  // Histogram of the blocks of level-0 bucket in0 (all blocks when in0 < 0): 32-bit
+  // shared-memory atomics per block (a mass w < 2^40 goes in as w >> 20 and w & 0xfffff,
+  // so over at most 2^11 blocks the sums stay below 2^31), except for the last bucket
+  // (the tail, where the blocks of a sparse row pile up), which each lane sums in
+  // registers and one lane stores.  Returns the row's (or bucket's) mass.
+  auto histogram = [&](int in0) -> unsigned long long {
+#pragma unroll 4
+    for (int e = lane; e < kSelBuckets; e += 32) {
+      sh.hh[e] = 0u;
+      sh.hl[e] = 0u;
+      sh.hc[e] = 0u;
     }
-  }
-  z = warp_sum_u64(z);
-  __syncwarp();
-
-  // Gathers bucket b's blocks into the list; false when they do not fit.
-  auto gather = [&](int b, int n) -> bool {
-    if (n > kSelCap) return false;
+    __syncwarp();
+    unsigned long long z = 0, tail_w = 0;
+    uint32_t tail_c = 0;
+#pragma unroll 2
+    for (int c = 0; c < words; ++c) {
+      const uint32_t k = key[c * 32];
+      if (k != 0u) {
+        const float x = key_value(k);
+        const float t = sel_t(mx, x);
+        const int b0 = sel_b0(t);
+        const int b = in0 < 0 ? b0 : (b0 == in0 ? sel_b1(t, b0) : -1);
+        if (b >= 0) {
+          const unsigned long long w = mass_of(c, x);
+          z += w;
+          if (b == kSelBuckets - 1) {
+            tail_w += w;
+            ++tail_c;
+          } else {
+            atomicAdd(&sh.hh[b], static_cast<uint32_t>(w >> 20));
+            atomicAdd(&sh.hl[b], static_cast<uint32_t>(w & 0xfffffu));
+            atomicAdd(&sh.hc[b], 1u);
+          }
+        }
+      }
+    }
+    tail_w = warp_sum_u64(tail_w);
+    tail_c = static_cast<uint32_t>(warp_sum_i(static_cast<int>(tail_c)));
+    __syncwarp();
+    if (lane == 0) {
+      sh.hh[kSelBuckets - 1] = static_cast<uint32_t>(tail_w >> 20);
+      sh.hl[kSelBuckets - 1] = static_cast<uint32_t>(tail_w & 0xfffffu);
+      sh.hc[kSelBuckets - 1] = tail_c;
+    }
+    __syncwarp();
+    return warp_sum_u64(z);
+  };
+  // Gathers the n <= 32 blocks of level-0 bucket b0 (and level-1 bucket b1 >= 0).
+  auto gather = [&](int b0, int b1) {
     int base = 0;
-#pragma unroll
-    for (int c = 0; c < MAXW; ++c) {
-      const bool in = key[c] != 0u && sel_bucket(mx, x[c]) == b;
+#pragma unroll 2
+    for (int c = 0; c < words; ++c) {
+      const uint32_t k = key[c * 32];
+      bool in = false;
+      float x = 0.f;
+      if (k != 0u) {
+        x = key_value(k);
+        const float t = sel_t(mx, x);
+        const int c0 = sel_b0(t);
+        in = c0 == b0 && (b1 < 0 || sel_b1(t, c0) == b1);
+      }
       const uint32_t bal = __ballot_sync(0xffffffffu, in);
       if (in) {
         const int pos = base + __popc(bal & ((1u << lane) - 1u));
-        sh.lkey[pos] = key[c];
+        sh.lkey[pos] = k;
         sh.lidx[pos] = static_cast<uint32_t>(c * 32 + lane);
-        sh.lw[pos] = sel_fixed(mass_of(c));
+        sh.lw[pos] = mass_of(c, x);
       }
       base += __popc(bal);
     }
     __syncwarp();
-    return true;
   };
-  // Among the n gathered blocks, the one of smallest rank (key desc, index asc) at which
-  // above + (running sum of weights up to it) >= target; weight = mass or 1.
-  auto resolve = [&](int n, bool by_mass, unsigned long long above, int& rank_out, uint32_t& key_out,
-                     int& idx_out, unsigned long long target) {
+  // Among the n <= 32 gathered blocks (lane j holds block j), the one of smallest rank
+  // (key desc, index asc) at which above + (running sum of weights up to it) >= target;
+  // weight = mass or 1.
+  auto resolve = [&](int n, bool by_mass, unsigned long long above, unsigned long long target, int& rank_out,
+                     uint32_t& key_out, int& idx_out) {
     int best = 0x7fffffff;
-#pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      const int j = lane + 32 * h;
-      if (j < n) {
-        const uint32_t kj = sh.lkey[j], ij = sh.lidx[j];
-        int rank = 0;
-        unsigned long long pre = 0;
-        for (int t = 0; t < n; ++t) {
-          const uint32_t kt = sh.lkey[t], it = sh.lidx[t];
-          const bool before = kt > kj || (kt == kj && it < ij);
-          rank += before ? 1 : 0;
-          if (before || t == j) pre += by_mass ? sh.lw[t] : 1ull;
-        }
-        // a block whose prefix reaches the target codes as its rank; the others code
-        // above every such rank, the last in the order lowest (the whole bucket)
-        best = min(best, above + pre >= target ? rank * 64 + j : (2 * n - 1 - rank) * 64 + j);
+    if (lane < n) {
+      const uint32_t kj = sh.lkey[lane], ij = sh.lidx[lane];
+      int rank = 0;
+      unsigned long long pre = 0;
+      for (int t = 0; t < n; ++t) {
+        const uint32_t kt = sh.lkey[t], it = sh.lidx[t];
+        const bool before = kt > kj || (kt == kj && it <= ij);
+        rank += (before && t != lane) ? 1 : 0;
+        pre += before ? (by_mass ? sh.lw[t] : 1ull) : 0ull;
       }
+      // a block whose prefix reaches the target codes as its rank; the others code above
+      // every such rank, the last in the order lowest (the whole bucket)
+      best = above + pre >= target ? rank * 64 + lane : (2 * n - 1 - rank) * 64 + lane;
     }
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, off));
@@ -489,7 +576,80 @@ __device__ __forceinline__ void select_row_hist(const Geo& g, const RouteOpts& o
     idx_out = static_cast<int>(sh.lidx[j]);
     __syncwarp();
   };
+  // Exact fallback for a bucket of more than 32 near-tied blocks: a bitwise search for the
+  // cut's key over the whole row (u = the largest key whose prefix of keys >= u reaches the
+  // target), then tied keys in index order.
+  auto search = [&](bool by_mass, unsigned long long target, int& m_out, uint32_t& ucut, int& icut) {
+    uint32_t u = 0;
+#pragma unroll 1
+    for (int bit = 31; bit >= 0; --bit) {
+      const uint32_t cand = u | (1u << bit);
+      unsigned long long m = 0;
+#pragma unroll 1
+      for (int c = 0; c < words; ++c) {
+        const uint32_t k = key[c * 32];
+        if (k != 0u && k >= cand) m += by_mass ? mass_of(c, key_value(k)) : 1ull;
+      }
+      if (warp_sum_u64(m) >= target) u = cand;
+    }
+    unsigned long long acc = 0;
+    int gt = 0;
+#pragma unroll 1
+    for (int c = 0; c < words; ++c) {
+      const uint32_t k = key[c * 32];
+      if (k != 0u && k > u) {
+        acc += by_mass ? mass_of(c, key_value(k)) : 1ull;
+        ++gt;
+      }
+    }
+    acc = warp_sum_u64(acc);
+    gt = warp_sum_i(gt);
+    int r = 0, last = -1;
+#pragma unroll 1
+    for (int c = 0; c < words && acc < target; ++c) {
+      const uint32_t k = key[c * 32];
+      uint32_t tb = __ballot_sync(0xffffffffu, k != 0u && k == u);
+      while (tb != 0u && acc < target) {
+        const int l = __ffs(tb) - 1;
+        tb &= tb - 1u;
+        const unsigned long long w = by_mass ? mass_of(c, key_value(u)) : 1ull;
+        acc += __shfl_sync(0xffffffffu, w, l);
+        ++r;
+        last = c * 32 + l;
+      }
+    }
+    m_out = gt + r;
+    ucut = u;
+    icut = last;
+  };
+  // The cut: the block of the order at which the running sum reaches target (the level-0
+  // histogram is in place).
+  auto cut = [&](bool by_mass, unsigned long long target, int& m_out, uint32_t& ucut, int& icut) {
+    unsigned long long above;
+    int cnt_above;
+    const int b0 = sel_find_bucket(sh, by_mass, target, above, cnt_above, lane);
+    int b1 = -1;
+    int n = static_cast<int>(sh.hc[b0]);
+    if (n > kSelCap) {
+      histogram(b0);
+      unsigned long long above1;
+      int cnt1;
+      b1 = sel_find_bucket(sh, by_mass, target - above, above1, cnt1, lane);
+      above += above1;
+      cnt_above += cnt1;
+      n = static_cast<int>(sh.hc[b1]);
+      if (n > kSelCap) {
+        search(by_mass, target, m_out, ucut, icut);
+        return;
+      }
+    }
+    gather(b0, b1);
+    int rank;
+    resolve(n, by_mass, above, target, rank, ucut, icut);
+    m_out = cnt_above + rank + 1;
+  };
 
+  const unsigned long long z = histogram(-1);
   const int floor_k = min(max(k_floor, 0), nB);
   int m_p = nB;
   uint32_t ucut = 0u;        // blocks with key > ucut, and key == ucut up to index icut, are kept
@@ -499,55 +659,31 @@ __device__ __forceinline__ void select_row_hist(const Geo& g, const RouteOpts& o
     // at least one unit, so that p = 0 still keeps the first block of the order
     const unsigned long long target =
         max(1ull, static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(z))));
-    unsigned long long above;
-    int cnt_above;
-    const int b = sel_find_bucket(sh, true, target, above, cnt_above, lane);
-    if (!gather(b, static_cast<int>(sh.hc[b]))) {
-      select_row<MAXW>(g, o, lrow, nB, words, qb, p, k_floor, mrow, cnt_out, lane);
-      return;
-    }
-    int rank;
-    resolve(static_cast<int>(sh.hc[b]), true, above, rank, ucut, icut, target);
-    m_p = cnt_above + rank + 1;
+    cut(true, target, m_p, ucut, icut);
     all = false;
   }
   const int M = max(max(m_p, floor_k), 1);
   if (M >= nB) {
     all = true;
   } else if (M > m_p) {
-    unsigned long long above;
-    int cnt_above;
-    const int b = sel_find_bucket(sh, false, static_cast<unsigned long long>(M), above, cnt_above, lane);
-    if (!gather(b, static_cast<int>(sh.hc[b]))) {
-      select_row<MAXW>(g, o, lrow, nB, words, qb, p, k_floor, mrow, cnt_out, lane);
-      return;
-    }
-    int rank;
-    resolve(static_cast<int>(sh.hc[b]), false, above, rank, ucut, icut, static_cast<unsigned long long>(M));
+    histogram(-1);           // the cut may have left a finer histogram in place
+    int m;
+    cut(false, static_cast<unsigned long long>(M), m, ucut, icut);
     all = false;
   }
   int cnt = 0;
-#pragma unroll
-  for (int c = 0; c < MAXW; ++c) {
-    if (c < words) {
-      const int i = c * 32 + lane;
-      const bool valid = key[c] != 0u;
-      const bool kept = valid && (all || key[c] > ucut || (key[c] == ucut && i <= icut) || i == qb ||
+#pragma unroll 2
+  for (int c = 0; c < words; ++c) {
+    const int i = c * 32 + lane;
+    const uint32_t k = key[c * 32];
+    const bool kept = k != 0u && (all || k > ucut || (k == ucut && i <= icut) || i == qb ||
                                   keyframe_block(g, o, i));
-      const uint32_t word = __ballot_sync(0xffffffffu, kept);
-      cnt += __popc(word);
-      if (lane == 0) mrow[c] = word;
-    }
+    const uint32_t word = __ballot_sync(0xffffffffu, kept);
+    cnt += __popc(word);
+    if (lane == 0) mrow[c] = word;
   }
   if (lane == 0) *cnt_out = cnt;
 }
-
-__device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
-  asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
-}
-__device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
-template <int N>
-__device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
 
 constexpr int kRouteKT = 128;          // key blocks per staged tile
 constexpr int kRouteDC = 32;           // channels per staged tile
@@ -656,8 +792,8 @@ static cudaError_t launch_route_t(const Geo& g, const float* qp, const float* kp
                                   float scale, uint32_t* mask, int32_t* counts, cudaStream_t st) {
   dim3 grid((g.nB + kRouteRows - 1) / kRouteRows, g.B * g.H);
   const size_t smem = route_smem_bytes(g);
-  cudaError_t e = cudaFuncSetAttribute(route_kernel<D, MAXW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                       static_cast<int>(smem));
+  static SmemAttrCache attr_ctx = {};
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(route_kernel<D, MAXW>), static_cast<int>(smem), attr_ctx);
   if (e != cudaSuccess) return e;
   route_kernel<D, MAXW><<<grid, kRouteThreads, smem, st>>>(g, qp, kp, p, k_floor, scale, mask, counts);
   return cudaGetLastError();
@@ -692,34 +828,153 @@ cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p
 // the tensor cores (fv_route_tc.cu); then one warp per query block selects from its row
 // by mass histogram (select_row_hist).
 // ----------------------------------------------------------------------------
-template <int MAXW>
-__global__ void __launch_bounds__(128) select_hist_kernel(Geo g, RouteOpts o, const float* __restrict__ logits,
-                                                          float p, int k_floor, uint32_t* __restrict__ mask,
-                                                          int32_t* __restrict__ counts) {
-  __shared__ SelScratch sh[4];
+__global__ void __launch_bounds__(32 * kSelWarps) select_hist_kernel(Geo g, RouteOpts o,
+                                                                     const float* __restrict__ logits, float p,
+                                                                     int k_floor, uint32_t* __restrict__ mask,
+                                                                     int32_t* __restrict__ counts) {
+  extern __shared__ __align__(16) unsigned char sel_smem[];
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int nB = g.nB, nBpad = g.words * 32;
-  const long long row = static_cast<long long>(blockIdx.x) * 4 + warp;   // (b*h) * nB + qb
+  const long long row = static_cast<long long>(blockIdx.x) * kSelWarps + warp;   // (b*h) * nB + qb
   if (row >= static_cast<long long>(g.B) * g.H * nB) return;
   const int qb = static_cast<int>(row % nB);
-  select_row_hist<MAXW>(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
-                        mask + static_cast<size_t>(row) * g.words, counts + row, lane, sh[warp]);
+  const SelScratch sh = sel_scratch(sel_smem + warp * sel_warp_bytes(g.words));
+  select_row_hist(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
+                  mask + static_cast<size_t>(row) * g.words, counts + row, lane, sh);
+}
+
+// For rows of at most kHistMinWords mask words the route is the fp32 pair: logits_kernel
+// (64 x 64 block pairs per CTA, each thread 4 x 4 pairs in f32x2 FMA, in the per-logit
+// operation order of route_kernel) and the bitwise selection below.  At those sizes the
+// tensor-core path's split and fill cost more than its products save.
+constexpr int kHistMinWords = 16;
+constexpr int kLogitTile = 64;         // query x key blocks per CTA
+
+template <int D>
+__global__ void __launch_bounds__(256) logits_kernel(Geo g, const float* __restrict__ qp,
+                                                     const float* __restrict__ kp, float scale,
+                                                     float* __restrict__ logits) {
+  constexpr int RS = D + 4;            // padded row (floats)
+  extern __shared__ __align__(16) unsigned char lg_smem[];
+  float* sQ = reinterpret_cast<float*>(lg_smem);   // [64][D + 4]
+  float* sK = sQ + kLogitTile * RS;                // [64][D + 4]
+  const int nB = g.nB, nBpad = g.words * 32;
+  const int bhi = blockIdx.z;
+  const int q0 = blockIdx.x * kLogitTile, k0 = blockIdx.y * kLogitTile;
+  const float* qh = qp + static_cast<size_t>(bhi) * nB * D;
+  const float* kh = kp + static_cast<size_t>(bhi) * nB * D;
+  for (int e = threadIdx.x; e < kLogitTile * D / 4; e += 256) {
+    const int r = e / (D / 4), d4 = e - r * (D / 4);
+    const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
+    reinterpret_cast<float4*>(sQ + r * RS)[d4] =
+        q0 + r < nB ? reinterpret_cast<const float4*>(qh + static_cast<size_t>(q0 + r) * D)[d4] : z;
+    reinterpret_cast<float4*>(sK + r * RS)[d4] =
+        k0 + r < nB ? reinterpret_cast<const float4*>(kh + static_cast<size_t>(k0 + r) * D)[d4] : z;
+  }
+  __syncthreads();
+  // thread (ty, tx) takes query rows ty + 16 i and key blocks tx + 16 j, i, j < 4
+  const int tx = threadIdx.x & 15, ty = threadIdx.x >> 4;
+  uint64_t acc[4][4];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) acc[i][j] = 0ull;
+#pragma unroll 4
+  for (int d4 = 0; d4 < D / 4; ++d4) {
+    uint64_t qxy[4], qzw[4], kxy[4], kzw[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float4 x = reinterpret_cast<const float4*>(sQ + (ty + 16 * i) * RS)[d4];
+      qxy[i] = f32x2(x.x, x.y);
+      qzw[i] = f32x2(x.z, x.w);
+      const float4 k4 = reinterpret_cast<const float4*>(sK + (tx + 16 * i) * RS)[d4];
+      kxy[i] = f32x2(k4.x, k4.y);
+      kzw[i] = f32x2(k4.z, k4.w);
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        acc[i][j] = ffma2(qxy[i], kxy[j], acc[i][j]);   // a0 += x.x k.x, a1 += x.y k.y
+        acc[i][j] = ffma2(qzw[i], kzw[j], acc[i][j]);   // a0 += x.z k.z, a1 += x.w k.w
+      }
+  }
+  float* out = logits + static_cast<size_t>(bhi) * nB * nBpad;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int qr = q0 + ty + 16 * i;
+    if (qr >= nB) continue;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int kc = k0 + tx + 16 * j;
+      if (kc >= nB) continue;
+      float a0, a1;
+      unpack_f32x2(acc[i][j], a0, a1);
+      out[static_cast<size_t>(qr) * nBpad + kc] = (a0 + a1) * scale;
+    }
+  }
+}
+
+// The selection of select_row (bitwise threshold search, one warp per row, the row's
+// logits in registers), for rows of at most kHistMinWords mask words: there its fixed cost
+// is below the histogram's (a 512-bucket scan and a gathered list per row).
+template <int MAXW>
+__global__ void __launch_bounds__(256) select_bitwise_kernel(Geo g, RouteOpts o, const float* __restrict__ logits,
+                                                             float p, int k_floor, uint32_t* __restrict__ mask,
+                                                             int32_t* __restrict__ counts) {
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int nB = g.nB, nBpad = g.words * 32;
+  const long long row = static_cast<long long>(blockIdx.x) * 8 + warp;   // (b*h) * nB + qb
+  if (row >= static_cast<long long>(g.B) * g.H * nB) return;
+  const int qb = static_cast<int>(row % nB);
+  select_row<MAXW>(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
+                   mask + static_cast<size_t>(row) * g.words, counts + row, lane);
+}
+
+
+
+static cudaError_t launch_select(const Geo& g, const RouteOpts& o, const float* logits, float p, int k_floor,
+                                 uint32_t* mask, int32_t* counts, cudaStream_t st) {
+  const long long rows = static_cast<long long>(g.B) * g.H * g.nB;
+  if (g.words <= kHistMinWords) {
+    const unsigned grid = static_cast<unsigned>((rows + 7) / 8);
+#define FV_SELECT(W) select_bitwise_kernel<W><<<grid, 256, 0, st>>>(g, o, logits, p, k_floor, mask, counts)
+    if (g.words <= 4) FV_SELECT(4);
+    else if (g.words <= 8) FV_SELECT(8);
+    else if (g.words <= 12) FV_SELECT(12);
+    else if (g.words <= 16) FV_SELECT(16);
+    else if (g.words <= 20) FV_SELECT(20);
+    else if (g.words <= 24) FV_SELECT(24);
+    else if (g.words <= 32) FV_SELECT(32);
+    else if (g.words <= 48) FV_SELECT(48);
+    else FV_SELECT(64);
+#undef FV_SELECT
+    return cudaGetLastError();
+  }
+  const int smem = static_cast<int>(kSelWarps * sel_warp_bytes(g.words));
+  static SmemAttrCache sel_attr = {};
+  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(select_hist_kernel), smem, sel_attr);
+  if (e != cudaSuccess) return e;
+  select_hist_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), 32 * kSelWarps, smem, st>>>(
+      g, o, logits, p, k_floor, mask, counts);
+  return cudaGetLastError();
 }
 
 // Route workspace: a 256-byte header (word 1: error bits of the logits kernel's bounded
-// waits), then the logits, [B*H][nB][words * 32] fp32.
+// waits), then the logits, [B*H][nB][words * 32] fp32 ...
 constexpr size_t kRouteHdr = 256;
 
 size_t route_logits_bytes(const Geo& g) {
   return static_cast<size_t>(g.B) * g.H * g.nB * (static_cast<size_t>(g.words) * 32) * 4;
 }
 
-size_t route_ws_bytes(const Geo& g) { return kRouteHdr + route_logits_bytes(g); }
+// ... followed by the pooled rows split into tf32 high and low parts (4 planes of
+// B*H*nB*d floats) for the tensor-core logits.
+size_t route_ws_bytes(const Geo& g) { return kRouteHdr + route_logits_bytes(g) + logits_split_bytes(g); }
 
-template <int D, int MAXW>
-static cudaError_t launch_route2_t(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                                   float scale, uint32_t* mask, int32_t* counts, void* ws,
-                                   cudaStream_t st, const RouteOpts& o) {
+cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st,
+                            const RouteOpts& o) {
   uint32_t* hdr = static_cast<uint32_t*>(ws);
   float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kRouteHdr);
   cudaError_t e = cudaMemsetAsync(hdr, 0, kRouteHdr, st);
@@ -729,34 +984,25 @@ static cudaError_t launch_route2_t(const Geo& g, const float* qp, const float* k
   if (e != cudaSuccess) return e;
   e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
   if (e != cudaSuccess) return e;
-  e = launch_logits_tc(g, qp, kp, scale, logits, hdr + 1, nsm, st);
+  if (g.words <= kHistMinWords) {
+    const int tiles = (g.nB + kLogitTile - 1) / kLogitTile;
+    const int smem = 2 * kLogitTile * (g.d + 4) * 4;
+    static SmemAttrCache lg_attr = {};
+    const void* fn = g.d == 128 ? reinterpret_cast<const void*>(logits_kernel<128>)
+                                : reinterpret_cast<const void*>(logits_kernel<64>);
+    e = set_smem_once(fn, smem, lg_attr);
+    if (e != cudaSuccess) return e;
+    const dim3 grid(tiles, tiles, g.B * g.H);
+    if (g.d == 128) logits_kernel<128><<<grid, 256, smem, st>>>(g, qp, kp, scale, logits);
+    else logits_kernel<64><<<grid, 256, smem, st>>>(g, qp, kp, scale, logits);
+  } else {
+    float* split = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(logits) + route_logits_bytes(g));
+    e = launch_logits_tc(g, qp, kp, scale, logits, split, hdr + 1, nsm, st);
+  }
   if (e != cudaSuccess) return e;
-  const long long rows = static_cast<long long>(g.B) * g.H * g.nB;
-  select_hist_kernel<MAXW><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, st>>>(g, o, logits, p, k_floor,
-                                                                                   mask, counts);
-  return cudaGetLastError();
-}
-
-template <int D>
-static cudaError_t launch_route2_d(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                                   float scale, uint32_t* mask, int32_t* counts, void* ws,
-                                   cudaStream_t st, const RouteOpts& o) {
-  if (g.words <= 4) return launch_route2_t<D, 4>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 8) return launch_route2_t<D, 8>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 12) return launch_route2_t<D, 12>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 16) return launch_route2_t<D, 16>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 20) return launch_route2_t<D, 20>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 24) return launch_route2_t<D, 24>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 32) return launch_route2_t<D, 32>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  if (g.words <= 48) return launch_route2_t<D, 48>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-  return launch_route2_t<D, 64>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
-}
-
-cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st,
-                            const RouteOpts& o) {
-  return g.d == 128 ? launch_route2_d<128>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o)
-                    : launch_route2_d<64>(g, qp, kp, p, k_floor, scale, mask, counts, ws, st, o);
+  e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  return launch_select(g, o, logits, p, k_floor, mask, counts, st);
 }
 
 // ----------------------------------------------------------------------------

@@ -12,14 +12,15 @@
 // from Tensor Cores while surpassing the FP32 theoretical peak performance", 2022):
 // the dropped terms are below 2^-21 of |a||b| per product.
 //
-// One CTA per work unit = (slice, 128 query blocks, a range of 128-key-block tiles):
-//   warps 0-3  load Qp / Kp rows from global memory (L2), split them into hi and lo and
-//              store both into shared memory in the 128-byte-swizzled K-major layout the
-//              MMA descriptors read (the query tile once, key tiles 32 channels at a time
-//              through a ring of stages);
-//   warp 4     issues the MMAs (one elected lane) into one of two 128-column fp32
+// split_kernel writes the hi and lo parts of every pooled row once, into the route
+// workspace.  Then one CTA per work unit = (slice, 128 query blocks, a range of
+// 128-key-block tiles):
+//   warp 0     loads the query tile's hi and lo parts, then the key tiles' 32 channels at a
+//              time through a ring of stages, with TMA in the 128-byte-swizzled K-major
+//              layout the MMA descriptors read;
+//   warp 1     issues the MMAs (one elected lane) into one of two 128-column fp32
 //              accumulators in tensor memory;
-//   warps 5-8  read an accumulator (one TMEM lane = one query row per thread), scale it
+//   warps 2-5  read an accumulator (one TMEM lane = one query row per thread), scale it
 //              and store the row's 128 logits, while the other accumulator fills.
 // Every wait is bounded; a stuck pipeline raises the workspace's error word and the
 // kernel drains and returns (fv::mbar_wait).
@@ -28,14 +29,15 @@
 
 namespace fv {
 
-constexpr int kLgThreads = 288;           // 9 warps
+constexpr int kLgThreads = 192;           // 6 warps
 constexpr int kLgChunk = 128 * 128;       // bytes: 128 rows x 32 fp32 (one swizzle column)
 constexpr int kLgTile = 128;              // query / key blocks per tile
 
-template <int D> __host__ __device__ constexpr int lg_stages() { return D == 128 ? 3 : 4; }
+template <int D> __host__ __device__ constexpr int lg_stages() { return D == 128 ? 2 : 4; }
+constexpr int kLgXpose = 4 * 32 * 33 * 4;   // bytes: a 32 x 33 fp32 transpose buffer per epilogue warp
 
 struct __align__(8) LgBars {
-  uint64_t a_full;
+  uint64_t a_full, a_empty;
   uint64_t st_full[4], st_empty[4];
   uint64_t acc_full[2], acc_empty[2];
   uint64_t fin;
@@ -45,39 +47,81 @@ struct __align__(8) LgBars {
 
 template <int D>
 __host__ __device__ constexpr int lg_smem_bytes() {
-  return 2 * (D / 32) * kLgChunk + lg_stages<D>() * 2 * kLgChunk + static_cast<int>(sizeof(LgBars));
+  return 2 * (D / 32) * kLgChunk + lg_stages<D>() * 2 * kLgChunk + kLgXpose + static_cast<int>(sizeof(LgBars));
 }
 static_assert(lg_smem_bytes<128>() <= 232448, "logits kernel exceeds 227 KB of shared memory");
+static_assert(lg_smem_bytes<64>() <= 232448, "logits kernel exceeds 227 KB of shared memory");
 
 struct LgParams {
   Geo g;
-  const float* qp;
-  const float* kp;
   float* logits;      // [B*H][nB][words*32]
   float scale;
   uint32_t* err;      // error word of the route workspace
-  int qtiles, ktiles, kper;   // 128-block tiles per slice (rows, keys); key tiles per unit
-  int nsplit;                 // units per (slice, query tile)
+  int tiles;          // 128-block tiles per slice side
+  int ksplit, kper;   // key-tile ranges per (slice, query tile), key tiles per range
+  long long items;    // (slice, query tile, key range) items, in that order
 };
 
-// 16 bytes (4 channels) of pooled row `row` of a 128-row tile, split and stored at 16-byte
-// unit `col16` of the row in the swizzled chunk.
-__device__ __forceinline__ void lg_store_split(uint32_t hi_base, uint32_t lo_base, int row, int col16, float4 x) {
-  const uint32_t off = static_cast<uint32_t>(row * 128 + ((col16 ^ (row & 7)) << 4));
-  const float h0 = to_tf32(x.x), h1 = to_tf32(x.y), h2 = to_tf32(x.z), h3 = to_tf32(x.w);
-  const float l0 = to_tf32(x.x - h0), l1 = to_tf32(x.y - h1), l2 = to_tf32(x.z - h2), l3 = to_tf32(x.w - h3);
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(hi_base + off), "f"(h0), "f"(h1), "f"(h2), "f"(h3)
-               : "memory");
-  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(lo_base + off), "f"(l0), "f"(l1), "f"(l2), "f"(l3)
-               : "memory");
+struct LgMaps {
+  CUtensorMap qh, ql, kh, kl;   // the split pooled rows, [B*H][nB][d] fp32 each
+};
+
+// x = hi + lo with hi = tf32(x), lo = tf32(x - hi), both rounded to nearest; stored as the
+// fp32 bit patterns the kind::tf32 MMA reads.
+template <int D>
+__global__ void __launch_bounds__(256) split_kernel(const float4* __restrict__ qp, const float4* __restrict__ kp,
+                                                    float4* __restrict__ split, long long n4) {
+  const long long i = static_cast<long long>(blockIdx.x) * 256 + threadIdx.x;
+  if (i >= n4) return;
+#pragma unroll
+  for (int src = 0; src < 2; ++src) {
+    const float4 x = __ldg((src ? kp : qp) + i);
+    const float4 h = make_float4(to_tf32(x.x), to_tf32(x.y), to_tf32(x.z), to_tf32(x.w));
+    const float4 l = make_float4(to_tf32(x.x - h.x), to_tf32(x.y - h.y), to_tf32(x.z - h.z), to_tf32(x.w - h.w));
+    split[(2 * src) * n4 + i] = h;
+    split[(2 * src + 1) * n4 + i] = l;
+  }
 }
 
+__device__ __forceinline__ void tma_load_3d(uint32_t dst, const CUtensorMap* m, uint64_t* bar, int c0, int c1,
+                                            int c2) {
+  asm volatile(
+      "cp.async.bulk.tensor.3d.shared::cluster.global.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5}], [%2];" ::"r"(dst),
+      "l"(reinterpret_cast<uint64_t>(m)), "r"(smem_u32(bar)), "r"(c0), "r"(c1), "r"(c2)
+      : "memory");
+}
+
+// Item w -> slice, query tile, key tiles [kt0, kt1).
+struct LgItem {
+  int bhi, qt, kt0, kt1;
+};
+__device__ __forceinline__ LgItem lg_item(long long w, const LgParams& p) {
+  const long long per_slice = static_cast<long long>(p.tiles) * p.ksplit;
+  LgItem r;
+  r.bhi = static_cast<int>(w / per_slice);
+  const int rem = static_cast<int>(w - r.bhi * per_slice);
+  r.qt = rem / p.ksplit;
+  const int ks = rem - r.qt * p.ksplit;
+  r.kt0 = ks * p.kper;
+  r.kt1 = min(p.tiles, r.kt0 + p.kper);
+  return r;
+}
+
+// Persistent: CTA i takes items i, i + P, i + 2P, ...  The items in flight at any moment
+// are consecutive, so the CTAs on one slice sweep the same key tiles at about the same
+// time: a key tile comes from DRAM once and from L2 for the slice's other query tiles.  A
+// CTA loads its query tile once per item.
 template <int D>
-__global__ void __launch_bounds__(kLgThreads, 1) logits_tc_kernel(const LgParams prm) {
+__global__ void __launch_bounds__(kLgThreads, 1)
+    logits_tc_kernel(const __grid_constant__ CUtensorMap tmQh, const __grid_constant__ CUtensorMap tmQl,
+                     const __grid_constant__ CUtensorMap tmKh, const __grid_constant__ CUtensorMap tmKl,
+                     const LgParams prm) {
   constexpr int NC = D / 32;                // 32-channel chunks per row
   constexpr int S = lg_stages<D>();
   extern __shared__ __align__(1024) unsigned char lg_dsm[];
-  LgBars& bars = *reinterpret_cast<LgBars*>(lg_dsm + 2 * NC * kLgChunk + S * 2 * kLgChunk);
+  float* xpose = reinterpret_cast<float*>(lg_dsm + 2 * NC * kLgChunk + S * 2 * kLgChunk);
+  LgBars& bars = *reinterpret_cast<LgBars*>(lg_dsm + 2 * NC * kLgChunk + S * 2 * kLgChunk + kLgXpose);
   const Geo& g = prm.g;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   volatile int* abort = &bars.abort;
@@ -92,85 +136,83 @@ __global__ void __launch_bounds__(kLgThreads, 1) logits_tc_kernel(const LgParams
   auto sBhi = [&](int s) { return base + static_cast<uint32_t>(2 * NC * kLgChunk + s * 2 * kLgChunk); };
   auto sBlo = [&](int s) { return sBhi(s) + static_cast<uint32_t>(kLgChunk); };
 
-  // work unit -> slice, query tile, key tiles [kt0, kt1)
-  const int unit = blockIdx.x;
-  const int per_slice = prm.qtiles * prm.nsplit;
-  const int bhi = unit / per_slice;
-  const int rem = unit - bhi * per_slice;
-  const int qt = rem / prm.nsplit, sp = rem - qt * prm.nsplit;
-  const int kt0 = sp * prm.kper, kt1 = min(prm.ktiles, kt0 + prm.kper);
-  const int nt = kt1 - kt0;
   const int nB = g.nB, nBpad = g.words * 32;
-  const int q0 = qt * kLgTile;
 
   if (threadIdx.x == 0) {
-    mbar_init(&bars.a_full, 128);
-    for (int i = 0; i < S; ++i) { mbar_init(&bars.st_full[i], 128); mbar_init(&bars.st_empty[i], 1); }
+    mbar_init(&bars.a_full, 1);
+    mbar_init(&bars.a_empty, 1);
+    for (int i = 0; i < S; ++i) { mbar_init(&bars.st_full[i], 1); mbar_init(&bars.st_empty[i], 1); }
     for (int i = 0; i < 2; ++i) { mbar_init(&bars.acc_full[i], 1); mbar_init(&bars.acc_empty[i], 4); }
     mbar_init(&bars.fin, 1);
     bars.abort = 0;
     fence_barrier_init();
   }
-  if (warp == 4) {
+  if (warp == 1) {
     tmem_alloc(&bars.tmem_base, 256);
     tmem_relinquish();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tmQh); tma_prefetch_desc(&tmQl);
+    tma_prefetch_desc(&tmKh); tma_prefetch_desc(&tmKl);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = bars.tmem_base;
+  uint32_t loads = 0, aloads = 0;           // B chunks / query tiles whose copies were issued
 
-  if (warp < 4) {
-    // ------------------------------------------------------------ operand staging
-    const int t = threadIdx.x;
-    const float4* qrows = reinterpret_cast<const float4*>(prm.qp + static_cast<size_t>(bhi) * nB * D);
-    const float4* krows = reinterpret_cast<const float4*>(prm.kp + static_cast<size_t>(bhi) * nB * D);
-    const float4 zero = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (warp == 0) {
+    // ------------------------------------------------------------ TMA producer (lane 0)
+    if (lane == 0) {
+      uint32_t i = 0;
+      bool ok = true;
 #pragma unroll 1
-    for (int c = 0; c < NC; ++c) {
-#pragma unroll 2
-      for (int u = t; u < 1024; u += 128) {
-        const int row = u >> 3, col16 = u & 7;
-        const int r = q0 + row;
-        const float4 x = r < nB ? __ldcg(qrows + static_cast<size_t>(r) * (D / 4) + c * 8 + col16) : zero;
-        lg_store_split(sAhi + c * kLgChunk, sAlo + c * kLgChunk, row, col16, x);
-      }
-    }
-    fence_proxy_async_smem();
-    mbar_arrive(&bars.a_full);
-    uint32_t i = 0;
-    bool ok = true;
+      for (long long w = blockIdx.x; w < prm.items && ok; w += gridDim.x) {
+        const LgItem t = lg_item(w, prm);
+        // the previous query tile's MMAs have finished reading it
+        if (aloads > 0 && !mbar_wait(&bars.a_empty, (aloads - 1) & 1, abort, err)) break;
+        mbar_arrive_expect_tx(&bars.a_full, static_cast<uint32_t>(2 * NC * kLgChunk));
 #pragma unroll 1
-    for (int kt = kt0; kt < kt1 && ok; ++kt) {
-#pragma unroll 1
-      for (int c = 0; c < NC; ++c, ++i) {
-        const int s = i % S;
-        if (!mbar_wait(&bars.st_empty[s], ((i / S) & 1) ^ 1, abort, err)) { ok = false; break; }
-#pragma unroll 2
-        for (int u = t; u < 1024; u += 128) {
-          const int row = u >> 3, col16 = u & 7;
-          const int r = kt * kLgTile + row;
-          const float4 x = r < nB ? __ldcg(krows + static_cast<size_t>(r) * (D / 4) + c * 8 + col16) : zero;
-          lg_store_split(sBhi(s), sBlo(s), row, col16, x);
+        for (int c = 0; c < NC; ++c) {
+          tma_load_3d(sAhi + c * kLgChunk, &tmQh, &bars.a_full, c * 32, t.qt * kLgTile, t.bhi);
+          tma_load_3d(sAlo + c * kLgChunk, &tmQl, &bars.a_full, c * 32, t.qt * kLgTile, t.bhi);
         }
-        fence_proxy_async_smem();
-        mbar_arrive(&bars.st_full[s]);
+        ++aloads;
+#pragma unroll 1
+        for (int kt = t.kt0; kt < t.kt1 && ok; ++kt) {
+#pragma unroll 1
+          for (int c = 0; c < NC; ++c, ++i) {
+            const int s = i % S;
+            if (!mbar_wait(&bars.st_empty[s], ((i / S) & 1) ^ 1, abort, err)) { ok = false; break; }
+            mbar_arrive_expect_tx(&bars.st_full[s], static_cast<uint32_t>(2 * kLgChunk));
+            tma_load_3d(sBhi(s), &tmKh, &bars.st_full[s], c * 32, kt * kLgTile, t.bhi);
+            tma_load_3d(sBlo(s), &tmKl, &bars.st_full[s], c * 32, kt * kLgTile, t.bhi);
+            loads = i + 1;
+          }
+        }
       }
     }
-  } else if (warp == 4) {
+    __syncwarp();
+  } else if (warp == 1) {
     // ------------------------------------------------------------ MMA issue
     const uint32_t idesc = idesc_tf32_f32(128, 128);
     auto wwait = [&](uint64_t* bar, uint32_t parity) -> bool {
       return __all_sync(0xffffffffu, mbar_wait(bar, parity, abort, err));
     };
-    bool ok = wwait(&bars.a_full, 0);
-    tc_fence_after();
-    uint32_t i = 0;
+    uint32_t i = 0, na = 0;
+    bool ok = true;
+    int j = 0;
 #pragma unroll 1
-    for (int j = 0; j < nt && ok; ++j) {
+    for (long long w = blockIdx.x; w < prm.items && ok; w += gridDim.x) {
+      const LgItem t = lg_item(w, prm);
+      if (!wwait(&bars.a_full, na & 1)) break;
+      ++na;
+#pragma unroll 1
+    for (int kt = t.kt0; kt < t.kt1 && ok; ++kt, ++j) {
       const int slot = j & 1;
-      if (!wwait(&bars.acc_empty[slot], ((j >> 1) & 1) ^ 1)) break;
+      if (!wwait(&bars.acc_empty[slot], ((j >> 1) & 1) ^ 1)) { ok = false; break; }
       const uint32_t tacc = tmem + static_cast<uint32_t>(slot * 128);
+      const bool last_of_a = kt + 1 == t.kt1;
 #pragma unroll 1
       for (int c = 0; c < NC; ++c, ++i) {
         const int s = i % S;
@@ -189,91 +231,149 @@ __global__ void __launch_bounds__(kLgThreads, 1) logits_tc_kernel(const LgParams
             mma_ss_tf32(tacc, dAh + o, dBh + o, idesc, 1u);
           }
           mma_commit(&bars.st_empty[s]);
-          if (c == NC - 1) mma_commit(&bars.acc_full[slot]);
+          if (c == NC - 1) {
+            mma_commit(&bars.acc_full[slot]);
+            if (last_of_a) mma_commit(&bars.a_empty);
+          }
         }
         __syncwarp();
       }
     }
+    }
   } else {
-    // ------------------------------------------------------------ epilogue
+    // ------------------------------------------------------------ epilogue (warps 2-5)
+    // Each 32 x 32 block of the accumulator (this warp's 32 rows, 32 key columns) goes
+    // through a padded shared buffer: thread r writes its row, then the warp stores row by
+    // row, 32 consecutive logits (128 bytes) per instruction.
     const int quarter = warp & 3;
-    const int row = quarter * 32 + lane;
-    const int r = q0 + row;
-    float* out = prm.logits + (static_cast<size_t>(bhi) * nB + (r < nB ? r : 0)) * nBpad;
+    float* xb = xpose + (warp - 2) * 32 * 33;
     const float sc = prm.scale;
+    int j = 0;
+    bool ok = true;
 #pragma unroll 1
-    for (int j = 0; j < nt; ++j) {
+    for (long long w = blockIdx.x; w < prm.items && ok; w += gridDim.x) {
+      const LgItem t = lg_item(w, prm);
+#pragma unroll 1
+    for (int kt = t.kt0; kt < t.kt1; ++kt, ++j) {
       const int slot = j & 1;
-      if (!__all_sync(0xffffffffu, mbar_wait(&bars.acc_full[slot], (j >> 1) & 1, abort, err))) break;
+      if (!__all_sync(0xffffffffu, mbar_wait(&bars.acc_full[slot], (j >> 1) & 1, abort, err))) { ok = false; break; }
       tc_fence_after();
-      const int k0 = (kt0 + j) * kLgTile;
+      const int row0 = t.qt * kLgTile + quarter * 32;
+      const int nrows = min(32, nB - row0);
 #pragma unroll 1
       for (int g4 = 0; g4 < 4; ++g4) {
         uint32_t v[32];
         tmem_ld32(tmem + (static_cast<uint32_t>(quarter * 32) << 16) + static_cast<uint32_t>(slot * 128 + 32 * g4), v);
         tmem_wait_ld();
-        const int col = k0 + 32 * g4;
-        if (r < nB && col < nBpad) {
-          float4* dst = reinterpret_cast<float4*>(out + col);
+        const int col = kt * kLgTile + 32 * g4;
+        if (col < nBpad) {                          // uniform over the warp
 #pragma unroll
-          for (int e = 0; e < 8; ++e)
-            dst[e] = make_float4(__uint_as_float(v[4 * e]) * sc, __uint_as_float(v[4 * e + 1]) * sc,
-                                 __uint_as_float(v[4 * e + 2]) * sc, __uint_as_float(v[4 * e + 3]) * sc);
+          for (int e = 0; e < 32; ++e) xb[lane * 33 + e] = __uint_as_float(v[e]) * sc;
+          __syncwarp();
+#pragma unroll 4
+          for (int r = 0; r < nrows; ++r)
+            prm.logits[(static_cast<size_t>(t.bhi) * nB + row0 + r) * nBpad + col + lane] = xb[r * 33 + lane];
+          __syncwarp();
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(&bars.acc_empty[slot]);
     }
+    }
   }
 
   // ------------------------------------------------------------ teardown
   __syncthreads();
-  if (bars.abort && warp == 4 && lane == 0) {
-    // let every issued MMA finish before tensor and shared memory are released
+  if (bars.abort) {
+    // let every armed copy land and every issued MMA finish before shared and tensor
+    // memory are released (bounded, the abort flag ignored)
     int never = 0;
     volatile int* nv = &never;
-    mma_commit(&bars.fin);
-    mbar_wait(&bars.fin, 0, nv, nullptr, 100000000ull);
+    if (warp == 0 && lane == 0) {
+      if (aloads > 0) mbar_wait(&bars.a_full, (aloads - 1) & 1, nv, nullptr, 100000000ull);
+      for (uint32_t i = (loads > static_cast<uint32_t>(S) ? loads - S : 0); i < loads; ++i)
+        mbar_wait(&bars.st_full[i % S], (i / S) & 1, nv, nullptr, 100000000ull);
+    }
+    if (warp == 1 && lane == 0) {
+      mma_commit(&bars.fin);
+      mbar_wait(&bars.fin, 0, nv, nullptr, 100000000ull);
+    }
   }
   tc_fence_before();
   __syncthreads();
-  if (warp == 4) {
+  if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem, 256);
   }
 }
 
+size_t logits_split_bytes(const Geo& g) {
+  return 4 * static_cast<size_t>(g.B) * g.H * g.nB * g.d * 4;
+}
+
 template <int D>
 static cudaError_t launch_logits_tc_d(const Geo& g, const float* qp, const float* kp, float scale, float* logits,
-                                      uint32_t* err, int nsm, cudaStream_t st) {
+                                      float* split, uint32_t* err, int nsm, cudaStream_t st) {
+  const int S = g.B * g.H;
+  const long long n4 = static_cast<long long>(S) * g.nB * D / 4;
+  split_kernel<D><<<static_cast<unsigned>((n4 + 255) / 256), 256, 0, st>>>(
+      reinterpret_cast<const float4*>(qp), reinterpret_cast<const float4*>(kp), reinterpret_cast<float4*>(split), n4);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  const size_t plane = static_cast<size_t>(S) * g.nB * D;
+  // the four maps depend only on the split buffer and the geometry: the last set a thread
+  // encoded is reused while they stay the same
+  struct MapCache {
+    unsigned long long ctx;
+    const float* split;
+    int S, nB;
+    LgMaps maps;
+    bool valid;
+  };
+  thread_local MapCache mc = {};
+  const unsigned long long ctx = current_ctx_id();
+  if (!(mc.valid && ctx != 0 && mc.ctx == ctx && mc.split == split && mc.S == S && mc.nB == g.nB)) {
+    mc.valid = false;
+    if (!encode_rows_fp32(&mc.maps.qh, split, S, g.nB, D) ||
+        !encode_rows_fp32(&mc.maps.ql, split + plane, S, g.nB, D) ||
+        !encode_rows_fp32(&mc.maps.kh, split + 2 * plane, S, g.nB, D) ||
+        !encode_rows_fp32(&mc.maps.kl, split + 3 * plane, S, g.nB, D))
+      return cudaErrorInvalidValue;
+    mc.ctx = ctx;
+    mc.split = split;
+    mc.S = S;
+    mc.nB = g.nB;
+    mc.valid = true;
+  }
   LgParams prm;
   prm.g = g;
-  prm.qp = qp;
-  prm.kp = kp;
   prm.logits = logits;
   prm.scale = scale;
   prm.err = err;
-  prm.qtiles = (g.nB + kLgTile - 1) / kLgTile;
-  prm.ktiles = prm.qtiles;
-  // split the key tiles of a (slice, query tile) over enough units for two waves
-  const long long base = static_cast<long long>(g.B) * g.H * prm.qtiles;
-  int nsplit = 1;
-  while (nsplit < prm.ktiles && base * nsplit < 2LL * nsm) ++nsplit;
-  prm.kper = (prm.ktiles + nsplit - 1) / nsplit;
-  prm.nsplit = (prm.ktiles + prm.kper - 1) / prm.kper;
-  const long long units = base * prm.nsplit;
+  prm.tiles = (g.nB + kLgTile - 1) / kLgTile;
+  // key ranges: enough items for about three rounds over the SMs, each item at least two
+  // key tiles (so that its query tile is used for more than one)
+  const long long base = static_cast<long long>(S) * prm.tiles;
+  int ksplit = 1;
+  while (ksplit < prm.tiles / 2 && base * ksplit < 3LL * nsm) ++ksplit;
+  prm.kper = (prm.tiles + ksplit - 1) / ksplit;
+  prm.ksplit = (prm.tiles + prm.kper - 1) / prm.kper;
+  prm.items = base * prm.ksplit;
+  const long long grid = prm.items < nsm ? prm.items : nsm;
   constexpr int smem = lg_smem_bytes<D>();
-  cudaError_t e = cudaFuncSetAttribute(logits_tc_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
+  static SmemAttrCache attr_ctx = {};
+  e = set_smem_once(reinterpret_cast<const void*>(logits_tc_kernel<D>), smem, attr_ctx);
   if (e != cudaSuccess) return e;
-  logits_tc_kernel<D><<<static_cast<unsigned>(units), kLgThreads, smem, st>>>(prm);
+  logits_tc_kernel<D><<<static_cast<unsigned>(grid), kLgThreads, smem, st>>>(mc.maps.qh, mc.maps.ql, mc.maps.kh,
+                                                                             mc.maps.kl, prm);
   return cudaGetLastError();
 }
 
 cudaError_t launch_logits_tc(const Geo& g, const float* qp, const float* kp, float scale, float* logits,
-                             uint32_t* err, int nsm, cudaStream_t st) {
-  return g.d == 128 ? launch_logits_tc_d<128>(g, qp, kp, scale, logits, err, nsm, st)
-                    : launch_logits_tc_d<64>(g, qp, kp, scale, logits, err, nsm, st);
+                             float* split, uint32_t* err, int nsm, cudaStream_t st) {
+  return g.d == 128 ? launch_logits_tc_d<128>(g, qp, kp, scale, logits, split, err, nsm, st)
+                    : launch_logits_tc_d<64>(g, qp, kp, scale, logits, split, err, nsm, st);
 }
 
 }  // namespace fv

@@ -106,21 +106,24 @@ FVATTN_API fvattn_status_t fvattn_route(const fvattn_geom_t* g, const float* q_p
                              uint32_t* mask, int32_t* counts, fvattn_stream_t stream);
 
 /* Bytes of device workspace fvattn_route_ws, fvattn_route_ex and fvattn_pool_route need:
- * a 256-byte header (a status word) followed by one fp32 logit per (query block, key
- * block) pair of every (b, h), rows padded to words * 32 entries (256 + B * H * nB *
- * words * 32 * 4 bytes; 5.4 MB at 21x30x52 with 1x8x16 blocks and 12 heads, 181 MB at
- * 121x30x52).  0 for an invalid geometry. */
+ * a 256-byte header (a status word), one fp32 logit per (query block, key block) pair of
+ * every (b, h) with rows padded to words * 32 entries, and the pooled rows split into
+ * tf32 high and low parts (256 + B*H*nB*words*32*4 + 4*B*H*nB*d*4 bytes; 13.7 MB at
+ * 21x30x52 with 1x8x16 blocks, d = 128 and 12 heads, 229 MB at 121x30x52).  0 for an
+ * invalid geometry. */
 FVATTN_API size_t fvattn_route_workspace_size(const fvattn_geom_t* g);
 
-/* fvattn_route, computed in two kernels through a caller-owned workspace: the logits of
- * all block pairs first, on the tensor cores (tf32 with each fp32 operand split into a
- * high and a low tf32 part, three products per pair: fp32-grade logits), written to
- * `workspace`; then the selection, one query block per warp, with the masses summed
- * exactly in fixed point (2^-32 of the row's largest exp).  Same definition, inputs,
- * outputs, argument domains and error behaviour as fvattn_route (FVAttn explainer
- * 核心方法 §1: Top-p with a Top-k floor and the own block over softmax(pooled q . pooled
- * k * scale)); the arithmetic differs from fvattn_route's, so the two may disagree on
- * blocks whose scores nearly tie at the cut.
+/* fvattn_route, computed through a caller-owned workspace: the logits of all block pairs
+ * first, written to `workspace`, then the selection, one query block per warp.  Rows of
+ * up to 16 mask words (nB <= 512) take fvattn_route's arithmetic in two kernels (a tiled
+ * fp32 product, then the bitwise threshold search), so the two calls give the same mask.
+ * Longer rows take the tensor cores for the logits (tf32 with each fp32 operand split into
+ * a high and a low tf32 part, three products per pair: fp32-grade logits) and select by a
+ * mass histogram with the masses summed exactly in fixed point (2^-32 of the row's
+ * largest exp); there the two calls may disagree on blocks whose scores nearly tie at the
+ * cut.  Same definition, inputs, outputs, argument domains and error behaviour as
+ * fvattn_route (FVAttn explainer 核心方法 §1: Top-p with a Top-k floor and the own block
+ * over softmax(pooled q . pooled k * scale)).
  *   workspace, ws_bytes : >= fvattn_route_workspace_size(g) bytes of device memory,
  *                         16-byte aligned, owned by the caller; its contents on entry
  *                         do not matter and on return hold the logits (scaled).
@@ -175,6 +178,31 @@ FVATTN_API fvattn_status_t fvattn_route_ex(const fvattn_geom_t* g, const float* 
  *   counts   : int32  [B][H][nB]                 (written: popcount of each repaired row) */
 FVATTN_API fvattn_status_t fvattn_mask_repair(const fvattn_geom_t* g, const uint32_t* mask_in, uint32_t* mask_out,
                                               int32_t* counts, fvattn_stream_t stream);
+
+/* Slack-aware sparse augmentation (FVAttn explainer, 核心方法 §3 Slack-Aware Sparse
+ * Augmentation: the slack that idle workers leave before the critical path ends is filled
+ * with high-value blocks, filtered by a score threshold; 工程落地 item 5).  Reading for one
+ * GPU, whose workers are the SMs of the persistent attention kernel: the cost of a
+ * (b, h, query block) tile is its real query tokens times the real key tokens of its kept
+ * blocks; tiles run longest first (cost descending, ties by tile index), and the last n_sm
+ * tiles of that order form the final wave, whose largest tile sets the end, cost c*.
+ * Every tile of the wave takes its dropped key blocks of routing score >= tau, in score
+ * order (descending, ties by lower index), each while its cost stays <= c*, and stops at
+ * the first that does not fit.  Call it after a route that left its logits in
+ * route_workspace (fvattn_route_ws, fvattn_route_ex, fvattn_pool_route) and before the
+ * attention.
+ *   route_workspace, route_ws_bytes : that route call's workspace (read)
+ *   tau    : score threshold, >= 0 (routing score = softmax over key blocks of the logits)
+ *   n_sm   : workers; 0 = the current device's SM count
+ *   mask, counts : updated in place (only the wave's rows change)
+ *   scratch, scratch_bytes : >= fvattn_attn_workspace_size(g) bytes of device memory, the
+ *            attention call's workspace may serve (its contents are rewritten anyway)
+ * Geometries whose tile cost needs 26 bits or more (bt*bh*bw * N >= 2^26) return
+ * FVATTN_ERR_UNSUPPORTED. */
+FVATTN_API fvattn_status_t fvattn_slack_augment(const fvattn_geom_t* g, const void* route_workspace,
+                                                size_t route_ws_bytes, float tau, int n_sm, uint32_t* mask,
+                                                int32_t* counts, void* scratch, size_t scratch_bytes,
+                                                fvattn_stream_t stream);
 
 /* Bytes of device workspace fvattn_pool_route needs: fvattn_route_workspace_size(g).  0
  * for an invalid geometry. */

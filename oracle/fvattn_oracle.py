@@ -213,6 +213,50 @@ def repair_mask(keep: np.ndarray, g: BlockGeometry) -> np.ndarray:
     return out
 
 
+def tile_costs(keep: np.ndarray, real_count: np.ndarray) -> np.ndarray:
+    """Attention work of every (b, h, query block) tile: its real query tokens times the
+    real key tokens of its kept blocks.  int [B, H, nB]."""
+    rc = np.asarray(real_count, np.int64)
+    return rc[None, None, :] * (keep.astype(np.int64) @ rc)
+
+
+def slack_augment(keep: np.ndarray, scores: np.ndarray, real_count: np.ndarray, n_sm: int,
+                  tau: float) -> np.ndarray:
+    """Slack-aware sparse augmentation on one GPU (FVAttn explainer, 核心方法 §3: the slack
+    that idle workers leave before the critical path ends is filled with high-value blocks,
+    filtered by a score threshold).
+
+    The tiles run longest first (cost descending, ties by tile index).  The last n_sm
+    tiles of that order form the final wave, where workers fall idle: its largest tile
+    sets the end, cost c*.  Every tile of the wave takes its dropped blocks of routing
+    score >= tau, in score order (descending, ties by lower index), each while the tile's
+    cost stays <= c*, stopping at the first that does not fit."""
+    B, H, nB, _ = keep.shape
+    rc = np.asarray(real_count, np.int64)
+    cost = tile_costs(keep, rc).reshape(-1)
+    T = cost.size
+    order = np.lexsort((np.arange(T), -cost))          # cost desc, then index asc
+    wave = order[max(0, T - int(n_sm)):]
+    out = keep.copy()
+    if wave.size == 0:
+        return out
+    cap = cost[wave].max()
+    flat_keep = out.reshape(T, nB)
+    flat_s = scores.reshape(T, nB)
+    for t in wave:
+        qb = t % nB
+        c = cost[t]
+        cand = [j for j in np.lexsort((np.arange(nB), -flat_s[t]))
+                if not flat_keep[t, j] and flat_s[t, j] >= tau]
+        for j in cand:
+            add = rc[qb] * rc[j]
+            if c + add > cap:
+                break
+            flat_keep[t, j] = True
+            c += add
+    return out
+
+
 def keep_for_cut(r: RouteResult, m: np.ndarray) -> np.ndarray:
     """The keep matrix for prefix lengths m [B,H,nB] (instead of r.m_keep): the first m
     key blocks of each row's order, plus the query's own block."""

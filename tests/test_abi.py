@@ -91,7 +91,7 @@ def test_host_side_argument_checks(L):
     assert L.fvattn_device_status(None, None) == E["FVATTN_ERR_INVALID_ARG"]
     # two-kernel route: the route checks, then a missing / short / misaligned workspace
     need = fv.fvattn_route_workspace_size(G480)
-    assert need == 256 + 12 * 336 * 11 * 32 * 4         # status header + logits
+    assert need == 256 + 12 * 336 * 11 * 32 * 4 + 4 * 12 * 336 * 128 * 4   # header, logits, split rows
     args = (ctypes.byref(cg), 0x1000, 0x2000, 0.9, 4, 0.088, 0x3000, 0x4000)
     assert L.fvattn_route_ws(*args, None, need, None) == E["FVATTN_ERR_WORKSPACE"]
     assert L.fvattn_route_ws(*args, 0x10000, need - 1, None) == E["FVATTN_ERR_WORKSPACE"]

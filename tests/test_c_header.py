@@ -84,7 +84,7 @@ def test_c_program_links_and_runs_host_entry_points(tmp_path, libdir):
     out = subprocess.run([str(exe)], check=True, capture_output=True, text=True, env=env).stdout
     lines = out.splitlines()
     assert lines[0].startswith("nB=336 words=11 attn_ws=")
-    assert lines[0].endswith(f" route_ws={256 + 12 * 336 * 11 * 32 * 4}")
+    assert lines[0].endswith(f" route_ws={256 + 12 * 336 * 11 * 32 * 4 + 4 * 12 * 336 * 128 * 4}")
     # the same static strings the binding reads through ctypes
     assert lines[1:8] == [f"status {i} {fv.fvattn_status_string(i)}" for i in range(7)]
     assert lines[8:] == [

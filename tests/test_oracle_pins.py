@@ -467,3 +467,68 @@ def test_repair_mask_hand_case():
     # blocks at the ends of an axis have no hole to fill
     keep3 = np.array([0, 1, 0, 0, 1], bool)[None, None, None, :]
     assert O.repair_mask(keep3, g)[0, 0, 0].astype(int).tolist() == [0, 1, 0, 0, 1]
+
+
+def test_tile_costs_by_token_pairs():
+    g = O.block_geometry(3, 5, 7, 2, 4, 4)          # ragged on every axis
+    rng = np.random.default_rng(4)
+    keep = rng.random((1, 2, g.nB, g.nB)) < 0.4
+    cost = O.tile_costs(keep, g.real_count)
+    for h in range(2):
+        for qb in range(g.nB):
+            pairs = sum(len(g.tokens_of_block[qb]) * len(g.tokens_of_block[kb])
+                        for kb in range(g.nB) if keep[0, h, qb, kb])
+            assert cost[0, h, qb] == pairs
+
+
+def test_slack_augment_hand_case():
+    # a 1 x 1 x 4 latent cut into 1-token blocks: four tiles whose costs are their kept
+    # counts.  Rows keep {0}, {0,1}, {0,1,2}, {0,1,2,3}: costs 1, 2, 3, 4.  With 2 SMs the
+    # final wave is the two cheapest tiles (rows 0 and 1), c* = 2: row 0 may add one block,
+    # row 1 none.
+    g = O.block_geometry(1, 1, 4, 1, 1, 1)
+    keep = np.zeros((1, 1, 4, 4), bool)
+    for i in range(4):
+        keep[0, 0, i, :i + 1] = True
+    s = np.array([[0.1, 0.2, 0.3, 0.4]] * 4)[None, None]      # block 3 scores highest
+    got = O.slack_augment(keep, s, g.real_count, 2, 0.0)
+    assert got[0, 0, 0].astype(int).tolist() == [1, 0, 0, 1]      # block 3, then full
+    assert (got[0, 0, 1:] == keep[0, 0, 1:]).all()
+    # a threshold above every candidate adds nothing
+    assert (O.slack_augment(keep, s, g.real_count, 2, 0.5) == keep).all()
+    # a threshold between: row 0's best candidate (0.4) passes
+    assert O.slack_augment(keep, s, g.real_count, 2, 0.35)[0, 0, 0].astype(int).tolist() == [1, 0, 0, 1]
+    # with 4 SMs every tile is in the final wave and c* = 4: rows 0-2 fill to 4 blocks
+    got4 = O.slack_augment(keep, s, g.real_count, 4, 0.0)
+    assert got4.all()
+    # ties in cost: the later index is later in the order (row 1 and a second row 1')
+    keep2 = np.zeros((1, 2, 4, 4), bool)
+    keep2[0, :, :, 0] = True                       # every tile costs 1
+    got2 = O.slack_augment(keep2, np.broadcast_to(s, (1, 2, 4, 4)), g.real_count, 3, 0.0)
+    # the final wave is the last three tiles in index order: (h=1, qb 1..3); c* = 1, nothing fits
+    assert (got2 == keep2).all()
+
+
+def test_slack_augment_never_exceeds_the_wave_cap():
+    w = W.SMALL_RAGGED
+    x = W.generate(w)
+    g = O.block_geometry(w.T, w.Hs, w.Ws, w.bt, w.bh, w.bw)
+    r = O.route(O.pool(x["q"], g), O.pool(x["k"], g), 0.6, 1, 1 / math.sqrt(w.d))
+    for n_sm in (4, 16, 64):
+        got = O.slack_augment(r.keep, r.scores, g.real_count, n_sm, 1e-4)
+        assert (got >= r.keep).all()
+        c0 = O.tile_costs(r.keep, g.real_count).reshape(-1)
+        c1 = O.tile_costs(got, g.real_count).reshape(-1)
+        order = np.lexsort((np.arange(c0.size), -c0))
+        wave = order[-n_sm:]
+        assert (c1[wave] <= c0[wave].max()).all()
+        changed = np.nonzero(c1 != c0)[0]
+        assert set(changed.tolist()) <= set(wave.tolist())
+        # added blocks pass the threshold and are the best dropped ones of their row
+        fk, fg, fs = r.keep.reshape(c0.size, -1), got.reshape(c0.size, -1), r.scores.reshape(c0.size, -1)
+        for t in changed:
+            added = fg[t] & ~fk[t]
+            assert (fs[t][added] >= 1e-4).all()
+            dropped = ~fg[t] & (fs[t] >= 1e-4)
+            if dropped.any():
+                assert fs[t][added].min() >= fs[t][dropped].max()
