@@ -85,6 +85,8 @@ fv.fvattn_dense_attn = lambda *a, **k: None
 fv.fvattn_device_status = lambda *a, **k: 0
 fv.fvattn_pool_route_workspace_size = lambda g: 1024
 fv.fvattn_pool_route = lambda g, q, k, p, kf, sc, qp, kp, mask, counts, ws, stream=None: mask.fill_(-1)
+fv.fvattn_route_ex = lambda g, qp, kp, opts, mask, counts, ws, stream=None: mask.fill_(-1)
+fv.fvattn_slack_augment = lambda *a, **k: None
 
 
 class FakeLayerGraph:

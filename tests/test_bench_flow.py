@@ -70,3 +70,21 @@ def test_two_ranks_over_gloo():
     assert len(lines) == 1                       # rank 0 only
     check_line(lines[0], 2)
     assert "cpu_baseline" not in lines[0] or lines[0]["cpu_baseline"] is None   # N = 1 only
+
+
+def test_sweep_lines_world_size_1():
+    """--sweep prints the headline line, then one line per p x k point, each timed by graph
+    replay with the direct call beside it."""
+    env = dict(os.environ, PYTHONPATH=ROOT)
+    out = subprocess.run([sys.executable, HARNESS, "--steps", "3", "--warmup", "3", "--sweep",
+                          "--no-cpu-baseline"], capture_output=True, text=True, env=env, timeout=900)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = json_lines(out.stdout)
+    assert "metric" in lines[0]
+    pts = [d for d in lines[1:] if "sweep_point" in d]
+    assert len(pts) == 15
+    for d in pts:
+        for key in ("p", "k_floor", "kept_block_frac", "attn_ms", "attn_ms_direct_call", "speedup_vs_dense",
+                    "effective_tflops", "frac_of_bf16_peak", "timing"):
+            assert key in d, key
+        assert d["kept_block_frac"] == 1.0          # the stand-in route keeps every block
