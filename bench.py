@@ -41,7 +41,7 @@ METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16
 # DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
 # ncu capture of dram__bytes_read.sum + dram__bytes_write.sum; valid only for the
 # kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "d1a9d3edfb431bc0", "bytes": 388617984}
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "c3520db57f7689b4", "bytes": 389974272}
 
 
 def attn_traffic():
