@@ -293,31 +293,33 @@ def run_ours(args, rank, world, local_rank, wl=None):
         return ts
 
     def back_to_back(fn, reps=20):
-        """Device time per launch of `reps` launches in a row (no host gaps)."""
-        for _ in range(3):
-            fn()
+        """Device time per call of `reps` calls in a row, captured in one CUDA graph (no host
+        work between them; the timing protocol of the layer).  fn(s) issues the call on
+        stream s; inside a capture s is None, the capturing stream."""
+        gr = graph_of(lambda: [fn(None) for _ in range(reps)])
+        for _ in range(2):
+            gr.replay()
         a = torch.cuda.Event(enable_timing=True)
         b = torch.cuda.Event(enable_timing=True)
         flush.fill_(0.5)
         a.record(stream)
-        for _ in range(reps):
-            fn()
+        gr.replay()
         b.record(stream)
         torch.cuda.synchronize(dev)
         return a.elapsed_time(b) / reps
 
     # Per-stage device times (not added to the layer time above).  Pool streams 201 MB
     # (more than L2); route reads the pooled rows pool has just written.
-    t_pool = back_to_back(lambda: fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, stream))
-    t_route = back_to_back(lambda: fv.fvattn_route_ws(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
-                                                      buf.mask, buf.counts, buf.route_ws, stream))
-    t_route1 = back_to_back(lambda: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
-                                                    buf.mask, buf.counts, stream))
-    # the layer's pool and route (fvattn_pool_route: pool, tensor-core logits, selection)
+    t_pool = back_to_back(lambda s: fv.fvattn_block_pool(g, q, k, buf.q_pool, buf.k_pool, s))
+    t_route = back_to_back(lambda s: fv.fvattn_route_ws(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
+                                                        buf.mask, buf.counts, buf.route_ws, s))
+    t_route1 = back_to_back(lambda s: fv.fvattn_route(g, buf.q_pool, buf.k_pool, wl.p, wl.k_floor, scale,
+                                                      buf.mask, buf.counts, s), reps=5)
+    # the layer's pool and route (fvattn_pool_route: pool, then the workspace route)
     fused = buf.pool_route_ws is not None
-    t_pool_route = back_to_back(lambda: fv.fvattn_pool_route(g, q, k, wl.p, wl.k_floor, scale, buf.q_pool,
-                                                             buf.k_pool, buf.mask, buf.counts,
-                                                             buf.pool_route_ws, stream))
+    t_pool_route = back_to_back(lambda s: fv.fvattn_pool_route(g, q, k, wl.p, wl.k_floor, scale, buf.q_pool,
+                                                               buf.k_pool, buf.mask, buf.counts,
+                                                               buf.pool_route_ws, s))
     # (inside a capture the calls must use the capturing stream: stream=None = current)
     attn_graph = graph_of(lambda: fv.fvattn_block_sparse_attn(g, q, k, v, buf.mask, scale, buf.out, buf.lse,
                                                               buf.workspace, buf.sm_busy_ns))
@@ -409,12 +411,12 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "attn_frac_of_bf16_peak": round(attn_tflops / peaks["bf16"], 4),
         "pool_ms": round(t_pool, 4), "route_ms": round(t_route, 4),
         "pool_route_ms": round(t_pool_route, 4),
-        "pool_route_kernel": ("fvattn_pool_route: pool, tensor-core logits, histogram selection" if fused
+        "pool_route_kernel": ("fvattn_pool_route: pool, then the workspace route (logits, selection)" if fused
                               else "pool + two-kernel route"),
         "route_one_kernel_ms": round(t_route1, 4),
         "stage_timing": "pool, route (fvattn_route_ws), pool_route (fvattn_pool_route, the layer's): device "
-                        "time per launch over 20 "
-                        "back-to-back launches; attention: one captured call after L2 flush + pool + route "
+                        "time per call of 20 back-to-back calls replayed from one CUDA graph (route_one_kernel: "
+                        "5); attention: one captured call after L2 flush + pool + route "
                         "(attn_ms median, attn_ms_mean and roofline mean)",
         "layer_step": "CUDA graph of pool -> route -> attention (LayerGraph)" if args.graph else "direct calls",
         "pool_route_gbs": round(pr_bytes / (pr_ms * 1e-3) / 1e9, 1),
@@ -679,6 +681,9 @@ def main():
                     help="chunks of (b, h) slices in the end-to-end leg (HostPipeline)")
     ap.add_argument("--layer-only", action="store_true",
                     help="time the layer steps only (no dense, e2e or CPU legs); for profilers")
+    ap.add_argument("--workload", default=None, choices=sorted(W.ALL),
+                    help="one line for this workload only, on one GPU (for profilers; the "
+                         "headline is the default, Wan2.1-480p)")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     rank = int(os.environ.get("RANK", 0))
@@ -695,6 +700,14 @@ def main():
         import torch
         torch.cuda.set_device(local_rank)
         torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
+    if args.workload is not None and args.workload != W.WAN21_480P.name:
+        if world > 1:
+            raise SystemExit("--workload runs on one GPU")
+        wl = W.ALL[args.workload]
+        line = run_ours(args, 0, 1, local_rank, wl)
+        line["metric"] = f"same measurements on the {wl.name} workload (not the headline)"
+        print(json.dumps(line), flush=True)
+        return
     try:
         line = run_ours(args, rank, world, local_rank)
         if rank == 0:

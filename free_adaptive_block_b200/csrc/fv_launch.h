@@ -18,12 +18,13 @@ bool encode_rows_fp32(CUtensorMap* m, const void* ptr, int slices, int rows, int
 // Sets `fn`'s dynamic shared-memory limit to at least `bytes`, unless a limit at least that
 // large was set already in the current context (the attribute lives with the context's copy
 // of the function; setting it on every call costs host time).  `cache` holds, per device
-// ordinal, the context id and the limit last set there.
+// ordinal, the context id and the limit last set there.  carveout >= 0 also sets the
+// preferred shared-memory carveout (percent of the unified L1 / shared array) with it.
 struct SmemAttrCache {
   unsigned long long ctx[64];
   int bytes[64];
 };
-inline cudaError_t set_smem_once(const void* fn, int bytes, SmemAttrCache& cache) {
+inline cudaError_t set_smem_once(const void* fn, int bytes, SmemAttrCache& cache, int carveout = -1) {
   int dev = 0;
   cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
@@ -31,6 +32,8 @@ inline cudaError_t set_smem_once(const void* fn, int bytes, SmemAttrCache& cache
   const unsigned long long id = current_ctx_id();
   if (slot && id != 0 && cache.ctx[dev] == id && cache.bytes[dev] >= bytes) return cudaSuccess;
   e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes);
+  if (e == cudaSuccess && carveout >= 0)
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributePreferredSharedMemoryCarveout, carveout);
   if (e == cudaSuccess && slot) {
     cache.ctx[dev] = current_ctx_id();
     cache.bytes[dev] = bytes;

@@ -305,385 +305,474 @@ __device__ __forceinline__ void select_row(const Geo& g, const RouteOpts& o, con
 }
 
 // ----------------------------------------------------------------------------
-// Selection by mass histogram (the form fvattn_route_ws, fvattn_route_ex and
-// fvattn_pool_route use).  Same rule as select_row, with the masses summed exactly: every
-// block's mass 2^((l - max) log2 e) (times its real token count for the Top-p over tokens) is
-// rounded once to a fixed-point integer of 2^-32 units, and all sums are integer sums, so
-// they do not depend on summation order and the prefix test "mass >= p" reads
-// sum >= ceil(p * Z) in integers.  Per row (one warp):
-//   1. logits into registers (lane l holds blocks c * 32 + l) as order keys, row maximum;
-//   2. a 512-bucket histogram of mass and count in shared memory over t = (max - l) * 32:
-//      bucket floor(t), the last one holding everything 16 or more below the max (its
-//      sums are kept in registers: the blocks of a sparse row pile up there);
-//   3. a warp scan over the buckets finds the bucket where the prefix mass reaches p;
-//   4. when that bucket holds more than 32 blocks, a second histogram over its fraction
-//      of t (512 sub-buckets) narrows it;
-//   5. the bucket's blocks are gathered and ranked exactly by (logit desc, index asc); the
-//      cut is the first rank at which the prefix reaches p;
-//   6. the Top-k floor, when it lengthens the prefix, repeats 2-5 on counts;
-//   7. the mask: blocks above the cut's key, tied blocks up to the cut's index, the own
-//      block and keyframe blocks.
-// A sub-bucket with more than 32 blocks (near-ties by the dozen) runs select_row.
+// Selection by mass histogram, for rows of more than kHistMinWords mask words (the form
+// fvattn_route_ws, fvattn_route_ex and fvattn_pool_route take there).  Same rule as
+// select_row, with the masses summed exactly: every block's mass 2^((l - max) log2 e)
+// (times its real token count for the Top-p over tokens) is rounded once to a fixed-point
+// integer of 2^-32 units, held as two int32 parts, and all sums are integer sums: they do
+// not depend on summation order, and the prefix test "mass >= p" reads sum >= ceil(p Z) in
+// integers.  Blocks are ordered by (logit desc, index asc), logits compared as floats.
+// One warp per row:
+//   1. the row into shared memory with 16-byte loads (blocks at or past nB as -inf) and
+//      its maximum;
+//   2. a 512-bucket histogram of mass (two 32-bit shared atomics per block), bucket
+//      round(32 (max - l)) clamped to 511: monotone in l;
+//   3. a warp scan over the buckets gives Z and the bucket where the prefix reaches
+//      ceil(p Z), and a pass lists that bucket's blocks (up to 256, in index order);
+//   4. at most 32 listed blocks are ranked exactly against each other, one per lane, and
+//      the cut is the first in the order at which the prefix reaches the target; a longer
+//      list is narrowed first by histograms over the 9 key bits below its highest
+//      differing bit, level after level;
+//   5. the mask: the blocks up to the cut, the own block, keyframe blocks.  The pass also
+//      counts m_p, and when the Top-k floor lengthens the prefix the cut is found again
+//      on counts and the mask rewritten.
+// More than 256 blocks in the cut bucket, or more than 32 blocks of one logit, fall back
+// to an exact bitwise search over the row.
 // ----------------------------------------------------------------------------
+constexpr int kHB = 512;                // buckets (and sub-buckets of the list levels)
+constexpr int kSelList = 256;           // listed blocks of the cut bucket
+constexpr int kSelWarps = 4;            // rows (warps) per CTA
+
+struct SelSmem {
+  int* hh;        // [kHB] per bucket: sum of the mass high parts (or a block count) ...
+  int* hl;        // [kHB]   ... and of the low parts (signed); hh, hl contiguous
+  float* lx;      // [kSelList] listed blocks: logit ...
+  int* li;        //   ... and block index
+  float* x;       // [words * 32] the row
+};
+
+__host__ __device__ constexpr size_t sel_warp_bytes(int words) {
+  return 2 * kHB * 4 + kSelList * 8 + static_cast<size_t>(words) * 128;
+}
+
+__device__ __forceinline__ SelSmem sel_smem_at(unsigned char* base) {
+  SelSmem s;
+  s.hh = reinterpret_cast<int*>(base);
+  s.hl = s.hh + kHB;
+  s.lx = reinterpret_cast<float*>(s.hl + kHB);
+  s.li = reinterpret_cast<int*>(s.lx + kSelList);
+  s.x = reinterpret_cast<float*>(s.li + kSelList);
+  return s;
+}
+
+// Order key of a logit with -0 taken as +0, so that key order is float order.
+__device__ __forceinline__ uint32_t sel_key(float x) { return order_key(__fadd_rn(x, 0.f)); }
+__device__ __forceinline__ float key_value(uint32_t k) {   // inverse of order_key
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
+}
+
+__device__ __forceinline__ long long warp_sum_ll(long long v) {
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+  return v;
+}
+
+// Bucket of a logit: the bits of fma(l, -32, cb) with cb = fl(32 max + 1.5 * 2^23), which
+// hold round(32 (max - l) + delta) (delta, the rounding of cb, is one constant for the
+// row), clamped to [0, 511]; -inf lands in 511.  A higher logit never lands later.
+__device__ __forceinline__ int sel_bucket(float x, float cb) {
+  return min(max(__float_as_int(__fmaf_rn(x, -32.f, cb)) - 0x4B400000, 0), kHB - 1);
+}
+
+// A block's mass in 2^-32 units as hh * 2^20 + hl: a = w * 2^12, hh = round(a),
+// hl = round((a - hh) * 2^20), each rounded by the 1.5 * 2^23 shifter (exact: a <= 2^19
+// since a block holds at most 2^7 tokens, and |a - hh| <= 1/2).  Over at most 2^11 blocks
+// sum(hh) <= 2^30 and |sum(hl)| <= 2^30.  TOKEN: times the block's real token count.
+struct MassParts {
+  int hh, hl;
+};
+template <bool TOKEN>
+__device__ __forceinline__ MassParts sel_mass(const Geo& g, float x, float nmx, int i) {
+  float w = ex2(__fmul_rn(__fadd_rn(x, nmx), 1.4426950408889634f));
+  if (TOKEN) w = __fmul_rn(w, static_cast<float>(block_info(g, i).nvalid));
+  const float a = __fmul_rn(w, 4096.f);
+  const float t1 = __fadd_rn(a, 12582912.f);
+  const float lo = __fsub_rn(a, __fsub_rn(t1, 12582912.f));
+  const float t2 = __fmaf_rn(lo, 1048576.f, 12582912.f);
+  return MassParts{__float_as_int(t1) - 0x4B400000, __float_as_int(t2) - 0x4B400000};
+}
+__device__ __forceinline__ long long parts64(int hh, int hl) {
+  return (static_cast<long long>(hh) << 20) + hl;
+}
+
+__device__ __forceinline__ void hist_zero(const SelSmem& sh, int lane) {
+  int4* h = reinterpret_cast<int4*>(sh.hh);       // hh and hl: 2 * kHB ints
+#pragma unroll
+  for (int e = lane; e < 2 * kHB / 4; e += 32) h[e] = make_int4(0, 0, 0, 0);
+  __syncwarp();
+}
+
+// Warp scan over the buckets, lane l owning buckets 16 l .. 16 l + 15 (by_mass: mass
+// parts, else counts in hh).  Returns the total; excl / own: the sums before this lane's
+// buckets and of them.
+__device__ __forceinline__ long long hist_scan(const SelSmem& sh, bool by_mass, int lane, long long& excl,
+                                               long long& own) {
+  const int4* h = reinterpret_cast<const int4*>(sh.hh + 16 * lane);
+  const int4* l = reinterpret_cast<const int4*>(sh.hl + 16 * lane);
+  int sh_ = 0, sl_ = 0;
+#pragma unroll
+  for (int v = 0; v < 4; ++v) {
+    const int4 a = h[v];
+    sh_ += (a.x + a.y) + (a.z + a.w);
+    if (by_mass) {
+      const int4 b = l[v];
+      sl_ += (b.x + b.y) + (b.z + b.w);
+    }
+  }
+  own = by_mass ? parts64(sh_, sl_) : static_cast<long long>(sh_);
+  long long incl = own;
+#pragma unroll
+  for (int off = 1; off < 32; off <<= 1) {
+    const long long v = __shfl_up_sync(0xffffffffu, incl, off);
+    if (lane >= off) incl += v;
+  }
+  excl = incl - own;
+  return __shfl_sync(0xffffffffu, incl, 31);
+}
+
+// The first bucket at which the running sum reaches target (1 <= target <= total), and
+// the sum of the buckets before it.
+__device__ __forceinline__ int hist_cross(const SelSmem& sh, bool by_mass, int lane, long long excl, long long own,
+                                          long long target, long long& above) {
+  int found = -1;
+  long long f_above = 0;
+  if (excl < target && excl + own >= target) {
+    long long run = excl;
+#pragma unroll 1
+    for (int e = 0; e < 16; ++e) {
+      const int b = 16 * lane + e;
+      const long long v = by_mass ? parts64(sh.hh[b], sh.hl[b]) : static_cast<long long>(sh.hh[b]);
+      if (run + v >= target) {
+        found = b;
+        f_above = run;
+        break;
+      }
+      run += v;
+    }
+  }
+  const uint32_t hit = __ballot_sync(0xffffffffu, found >= 0);
+  const int src = hit ? __ffs(hit) - 1 : 31;
+  above = __shfl_sync(0xffffffffu, f_above, src);
+  return hit ? __shfl_sync(0xffffffffu, found, src) : kHB - 1;
+}
+
+// Among n <= 32 candidates (lane j < n holds logit xj, index ij, weight wj), the first in
+// the order (logit desc, index asc) at which base + (the sum of weights up to and
+// including it) >= target; its lane.  The last candidate in the order always qualifies
+// when the candidates hold all the weight up to the target.
+__device__ __forceinline__ int resolve32(int n, float xj, int ij, long long wj, long long base, long long target,
+                                         int lane) {
+  int rank = 0;
+  long long pre = 0;
+#pragma unroll 1
+  for (int t = 0; t < n; ++t) {
+    const float xt = __shfl_sync(0xffffffffu, xj, t);
+    const int it = __shfl_sync(0xffffffffu, ij, t);
+    const long long wt = __shfl_sync(0xffffffffu, wj, t);
+    const bool before = xt > xj || (xt == xj && it <= ij);
+    rank += (before && t != lane) ? 1 : 0;
+    pre += before ? wt : 0ll;
+  }
+  int code = 0x7fffffff;
+  if (lane < n) code = (base + pre >= target ? rank : 2 * n - 1 - rank) * 64 + lane;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) code = min(code, __shfl_xor_sync(0xffffffffu, code, off));
+  return code & 63;
+}
+
+template <bool TOKEN>
+__device__ __forceinline__ long long sel_weight(const Geo& g, bool by_mass, float x, float nmx, int i) {
+  if (!by_mass) return 1ll;
+  const MassParts m = sel_mass<TOKEN>(g, x, nmx, i);
+  return parts64(m.hh, m.hl);
+}
+
+// Exact fallback: u = the largest key whose prefix (all blocks of key >= u) reaches the
+// target, by a bitwise search over the row; then the blocks of key u in index order.
+// Returns false never; sets the cut (logit and index of the block where the sum reaches
+// the target).
+template <bool TOKEN>
+__device__ void sel_search(const Geo& g, const SelSmem& sh, int words, int nB, bool by_mass, float nmx,
+                           long long target, int lane, float& xcut, int& icut) {
+  uint32_t u = 0;
+#pragma unroll 1
+  for (int bit = 31; bit >= 0; --bit) {
+    const uint32_t cand = u | (1u << bit);
+    long long m = 0;
+#pragma unroll 1
+    for (int c = 0; c < words; ++c) {
+      const int i = c * 32 + lane;
+      const float x = sh.x[i];
+      if (i < nB && sel_key(x) >= cand) m += sel_weight<TOKEN>(g, by_mass, x, nmx, i);
+    }
+    if (warp_sum_ll(m) >= target) u = cand;
+  }
+  long long acc = 0;
+#pragma unroll 1
+  for (int c = 0; c < words; ++c) {
+    const int i = c * 32 + lane;
+    const float x = sh.x[i];
+    if (i < nB && sel_key(x) > u) acc += sel_weight<TOKEN>(g, by_mass, x, nmx, i);
+  }
+  acc = warp_sum_ll(acc);
+  int last = -1;
+#pragma unroll 1
+  for (int c = 0; c < words && acc < target; ++c) {
+    const int i = c * 32 + lane;
+    const bool tie = i < nB && sel_key(sh.x[i]) == u;
+    uint32_t tb = __ballot_sync(0xffffffffu, tie);
+    const long long w = tie ? sel_weight<TOKEN>(g, by_mass, sh.x[i], nmx, i) : 0ll;
+    while (tb != 0u && acc < target) {
+      const int l = __ffs(tb) - 1;
+      tb &= tb - 1u;
+      acc += __shfl_sync(0xffffffffu, w, l);
+      last = c * 32 + l;
+    }
+  }
+  xcut = key_value(u);
+  icut = last;
+}
+
+// The cut for one target: the block of the order at which the running sum (mass, or block
+// count) first reaches target.  The bucket histogram of that kind must be in sh.
+template <bool TOKEN>
+__device__ void sel_cut(const Geo& g, const SelSmem& sh, int words, int nB, bool by_mass, float nmx, float cb,
+                        long long excl, long long own, long long target, int lane, float& xcut, int& icut) {
+  long long base;
+  const int b0 = hist_cross(sh, by_mass, lane, excl, own, target, base);
+  // list the bucket's blocks, in index order (four words per step, loads first)
+  int n = 0;
+#pragma unroll 1
+  for (int c0 = 0; c0 < words; c0 += 4) {
+    float x[4];
+    bool in[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const int i = (c0 + u) * 32 + lane;
+      x[u] = c0 + u < words ? sh.x[i] : -INFINITY;
+      in[u] = c0 + u < words && i < nB && sel_bucket(x[u], cb) == b0;
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      const uint32_t bal = __ballot_sync(0xffffffffu, in[u]);
+      const int pos = n + __popc(bal & ((1u << lane) - 1u));
+      if (in[u] && pos < kSelList) {
+        sh.lx[pos] = x[u];
+        sh.li[pos] = (c0 + u) * 32 + lane;
+      }
+      n += __popc(bal);
+    }
+  }
+  __syncwarp();
+  if (n > kSelList) {
+    sel_search<TOKEN>(g, sh, words, nB, by_mass, nmx, target, lane, xcut, icut);
+    return;
+  }
+  // candidates: listed blocks with key in [klo, khi]; base = the order's sum before them
+  uint32_t klo = 0u, khi = 0xffffffffu;
+#pragma unroll 1
+  for (int level = 0;; ++level) {
+    int cnt = 0;
+    uint32_t kmin = 0xffffffffu, kmax = 0u;
+    for (int e = lane; e < n; e += 32) {
+      const uint32_t k = sel_key(sh.lx[e]);
+      if (k >= klo && k <= khi) {
+        ++cnt;
+        kmin = min(kmin, k);
+        kmax = max(kmax, k);
+      }
+    }
+    cnt = warp_sum_i(cnt);
+    kmin = __reduce_min_sync(0xffffffffu, kmin);
+    kmax = __reduce_max_sync(0xffffffffu, kmax);
+    if (cnt <= 32) {
+      // the candidates into lanes (list order = index order), then rank them exactly
+      float xj = 0.f;
+      int ij = 0;
+      long long wj = 0;
+      int m = 0;
+      for (int e0 = 0; e0 < n; e0 += 32) {
+        const int e = e0 + lane;
+        float x = 0.f;
+        bool in = false;
+        if (e < n) {
+          x = sh.lx[e];
+          const uint32_t k = sel_key(x);
+          in = k >= klo && k <= khi;
+        }
+        const uint32_t bal = __ballot_sync(0xffffffffu, in);
+        const int idx = e < n ? sh.li[e] : 0;
+        // lane m + r takes the r-th candidate of this chunk
+        uint32_t rest = bal;
+        for (int r = 0; rest != 0u; ++r) {
+          const int src = __ffs(rest) - 1;
+          rest &= rest - 1u;
+          const float xs = __shfl_sync(0xffffffffu, x, src);
+          const int is = __shfl_sync(0xffffffffu, idx, src);
+          if (lane == m + r) {
+            xj = xs;
+            ij = is;
+          }
+        }
+        m += __popc(bal);
+      }
+      if (lane < cnt) wj = sel_weight<TOKEN>(g, by_mass, xj, nmx, ij);
+      const int j = resolve32(cnt, xj, ij, wj, base, target, lane);
+      xcut = __shfl_sync(0xffffffffu, xj, j);
+      icut = __shfl_sync(0xffffffffu, ij, j);
+      return;
+    }
+    if (kmin == kmax || level > 4) {       // more than 32 blocks of one logit
+      sel_search<TOKEN>(g, sh, words, nB, by_mass, nmx, target, lane, xcut, icut);
+      return;
+    }
+    // sub-buckets: the 9 key bits below the highest bit where the candidates differ,
+    // counted down from kmax (sub-bucket 0 holds the highest keys)
+    const int s = max(31 - __clz(kmin ^ kmax) - 8, 0);
+    const uint32_t top = kmax >> s;
+    hist_zero(sh, lane);
+    for (int e = lane; e < n; e += 32) {
+      const float x = sh.lx[e];
+      const uint32_t k = sel_key(x);
+      if (k >= klo && k <= khi) {
+        const int sb = static_cast<int>(top - (k >> s));
+        if (by_mass) {
+          const MassParts mp = sel_mass<TOKEN>(g, x, nmx, sh.li[e]);
+          atomicAdd(&sh.hh[sb], mp.hh);
+          atomicAdd(&sh.hl[sb], mp.hl);
+        } else {
+          atomicAdd(&sh.hh[sb], 1);
+        }
+      }
+    }
+    __syncwarp();
+    long long ex, ow, add;
+    hist_scan(sh, by_mass, lane, ex, ow);
+    const int sb = hist_cross(sh, by_mass, lane, ex, ow, target - base, add);
+    base += add;
+    klo = (top - static_cast<uint32_t>(sb)) << s;
+    khi = s > 0 ? klo | ((1u << s) - 1u) : klo;
+  }
+}
+
+template <bool TOKEN>
+__device__ void select_row_hist(const Geo& g, const RouteOpts& o, const float* __restrict__ lrow, int nB,
+                                int words, int qb, float p, int k_floor, uint32_t* mrow, int32_t* cnt_out,
+                                int lane, const SelSmem& sh) {
+  // 1. the row, past-the-end blocks as -inf, and its maximum
+  float mx = -INFINITY;
+  {
+    const float4* src = reinterpret_cast<const float4*>(lrow);
+    float4* dst = reinterpret_cast<float4*>(sh.x);
+    const int n4 = words * 8;
+#pragma unroll 4
+    for (int q = lane; q < n4; q += 32) {
+      float4 v = __ldg(src + q);
+      const int i0 = 4 * q;
+      if (i0 + 4 > nB) {
+        if (i0 + 0 >= nB) v.x = -INFINITY;
+        if (i0 + 1 >= nB) v.y = -INFINITY;
+        if (i0 + 2 >= nB) v.z = -INFINITY;
+        if (i0 + 3 >= nB) v.w = -INFINITY;
+      }
+      dst[q] = v;
+      mx = fmaxf(mx, fmaxf(fmaxf(v.x, v.y), fmaxf(v.z, v.w)));
+    }
+    mx = warp_max(mx);
+    __syncwarp();
+  }
+  const float nmx = -mx;
+  const float cb = __fadd_rn(__fmul_rn(mx, 32.f), 12582912.f);
+  // 2. mass histogram, four blocks per step: the step's loads and exponentials overlap
+  // (a load cannot pass the previous step's atomics)
+  hist_zero(sh, lane);
+#pragma unroll 1
+  for (int c0 = 0; c0 < words; c0 += 4) {
+    float x[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) x[u] = c0 + u < words ? sh.x[(c0 + u) * 32 + lane] : -INFINITY;
+    MassParts m[4];
+    int b[4];
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      m[u] = sel_mass<TOKEN>(g, x[u], nmx, (c0 + u) * 32 + lane);
+      b[u] = sel_bucket(x[u], cb);
+    }
+#pragma unroll
+    for (int u = 0; u < 4; ++u) {
+      if (c0 + u < words) {
+        atomicAdd(&sh.hh[b[u]], m[u].hh);
+        atomicAdd(&sh.hl[b[u]], m[u].hl);
+      }
+    }
+  }
+  __syncwarp();
+  bool all = p >= 1.f;
+  float xcut = INFINITY;
+  int icut = -1;
+  if (!all) {
+    long long excl, own;
+    const long long z = hist_scan(sh, true, lane, excl, own);
+    // at least one unit, so that p = 0 still keeps the first block of the order
+    const long long target =
+        max(1ll, static_cast<long long>(ceil(static_cast<double>(p) * static_cast<double>(z))));
+    sel_cut<TOKEN>(g, sh, words, nB, true, nmx, cb, excl, own, target, lane, xcut, icut);
+  }
+  // 3. the mask; m_p = the blocks of the prefix rule
+  auto write_mask = [&]() -> int {
+    int mp = 0, cnt = 0;
+#pragma unroll 1
+    for (int c0 = 0; c0 < words; c0 += 4) {
+      float x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = c0 + u < words ? sh.x[(c0 + u) * 32 + lane] : -INFINITY;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) {
+        const int c = c0 + u;
+        if (c < words) {
+          const int i = c * 32 + lane;
+          const bool v = i < nB;
+          const bool kp = v && (all || x[u] > xcut || (x[u] == xcut && i <= icut));
+          mp += __popc(__ballot_sync(0xffffffffu, kp));
+          const bool kept = kp || (v && (i == qb || keyframe_block(g, o, i)));
+          const uint32_t word = __ballot_sync(0xffffffffu, kept);
+          cnt += __popc(word);
+          if (lane == 0) mrow[c] = word;
+        }
+      }
+    }
+    if (lane == 0) *cnt_out = cnt;
+    return mp;
+  };
+  const int m_p = write_mask();
+  if (all) return;
+  const int floor_k = min(max(k_floor, 0), nB);
+  const int M = max(max(m_p, floor_k), 1);
+  if (M <= m_p) return;
+  if (M >= nB) {
+    all = true;
+  } else {
+    // the Top-k floor: the cut of the first M blocks, on counts
+    hist_zero(sh, lane);
+#pragma unroll 4
+    for (int c = 0; c < words; ++c) {
+      const int i = c * 32 + lane;
+      if (i < nB) atomicAdd(&sh.hh[sel_bucket(sh.x[i], cb)], 1);
+    }
+    __syncwarp();
+    long long excl, own;
+    hist_scan(sh, false, lane, excl, own);
+    sel_cut<TOKEN>(g, sh, words, nB, false, nmx, cb, excl, own, static_cast<long long>(M), lane, xcut, icut);
+  }
+  write_mask();
+}
+
 __device__ __forceinline__ void cp_async16(uint32_t dst, const void* src, uint32_t src_bytes) {
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16, %2;" ::"r"(dst), "l"(src), "r"(src_bytes) : "memory");
 }
 __device__ __forceinline__ void cp_async_commit() { asm volatile("cp.async.commit_group;" ::: "memory"); }
 template <int N>
 __device__ __forceinline__ void cp_async_wait() { asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory"); }
-
-constexpr int kSelBuckets = 512;
-constexpr float kSelPerLogit = 32.f;
-constexpr int kSelCap = 32;             // gathered blocks: one per lane
-constexpr int kSelWarps = 4;            // rows (warps) per CTA
-
-// Shared memory of one warp (one row at a time): the mass histogram, the gathered list and
-// the row's order keys, lane l's keys in column l ([c][32], so a lane touches only its own
-// words and no synchronisation is needed for them).
-struct SelScratch {
-  uint32_t* hh;                          // mass per bucket (2^-32 units): high parts (w >> 20) ...
-  uint32_t* hl;                          //   ... and low parts (w & 0xfffff), both exact in 32 bits
-  uint32_t* hc;                          // blocks per bucket
-  unsigned long long* lw;                // gathered bucket: mass,
-  uint32_t* lkey;                        //   order key,
-  uint32_t* lidx;                        //   block index
-  uint32_t* key;                         // the row: key[c * 32 + lane] for block c * 32 + lane
-};
-
-__host__ __device__ constexpr size_t sel_warp_bytes(int words) {
-  return 3 * kSelBuckets * 4 + kSelCap * 8 + 2 * kSelCap * 4 + static_cast<size_t>(words) * 32 * 4;
-}
-
-__device__ __forceinline__ SelScratch sel_scratch(unsigned char* base) {
-  SelScratch sh;
-  sh.hh = reinterpret_cast<uint32_t*>(base);
-  sh.hl = sh.hh + kSelBuckets;
-  sh.hc = sh.hl + kSelBuckets;
-  sh.lw = reinterpret_cast<unsigned long long*>(sh.hc + kSelBuckets);
-  sh.lkey = reinterpret_cast<uint32_t*>(sh.lw + kSelCap);
-  sh.lidx = sh.lkey + kSelCap;
-  sh.key = sh.lidx + kSelCap;
-  return sh;
-}
-
-__device__ __forceinline__ float key_value(uint32_t k) {   // inverse of order_key
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7fffffffu) : ~k);
-}
-
-__device__ __forceinline__ unsigned long long warp_sum_u64(unsigned long long v) {
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
-  return v;
-}
-
-__device__ __forceinline__ unsigned long long sel_fixed(float w) {
-  return __float2ull_rn(w * 4294967296.0f);
-}
-
-// Bucket coordinate of a logit: t = (max - x) * 32; level-0 bucket floor(t) (capped), and
-// inside level-0 bucket b0 the level-1 bucket floor((t - b0) * 512) (exact in fp32: t < 512
-// carries at most 14 fraction bits, so t - b0 and the scaling round nothing).
-__device__ __forceinline__ float sel_t(float mx, float x) { return (mx - x) * kSelPerLogit; }
-__device__ __forceinline__ int sel_b0(float t) { return min(kSelBuckets - 1, __float2int_rz(t)); }
-__device__ __forceinline__ int sel_b1(float t, int b0) {
-  return min(kSelBuckets - 1, __float2int_rz((t - static_cast<float>(b0)) * static_cast<float>(kSelBuckets)));
-}
-
-__device__ __forceinline__ unsigned long long sel_bucket_mass(const SelScratch& sh, int b) {
-  return (static_cast<unsigned long long>(sh.hh[b]) << 20) + sh.hl[b];
-}
-
-// Finds the bucket where the running sum (mass when `by_mass`, else count) first reaches
-// `target`, scanning buckets from the top of the order.  Lane l owns buckets 16 l .. 16 l + 15.
-// Returns the bucket; `above` / `cnt_above` get the sum and block count before it.
-__device__ __forceinline__ int sel_find_bucket(const SelScratch& sh, bool by_mass, unsigned long long target,
-                                               unsigned long long& above, int& cnt_above, int lane) {
-  constexpr int PER = kSelBuckets / 32;
-  unsigned long long run = 0;
-  int crun = 0;
-#pragma unroll 4
-  for (int e = 0; e < PER; ++e) {
-    const int b = lane * PER + e;
-    const uint32_t n = sh.hc[b];
-    run += by_mass ? sel_bucket_mass(sh, b) : static_cast<unsigned long long>(n);
-    crun += static_cast<int>(n);
-  }
-  unsigned long long incl = run;
-  int cincl = crun;
-#pragma unroll
-  for (int off = 1; off < 32; off <<= 1) {
-    const unsigned long long v = __shfl_up_sync(0xffffffffu, incl, off);
-    const int cv = __shfl_up_sync(0xffffffffu, cincl, off);
-    if (lane >= off) { incl += v; cincl += cv; }
-  }
-  unsigned long long excl = incl - run;
-  int cexcl = cincl - crun;
-  int found = kSelBuckets;
-  unsigned long long f_above = 0;
-  int f_cnt = 0;
-  if (incl >= target && excl < target) {      // the crossing lies in this lane's buckets
-#pragma unroll 1
-    for (int e = 0; e < PER; ++e) {
-      const int b = lane * PER + e;
-      const uint32_t n = sh.hc[b];
-      const unsigned long long v = by_mass ? sel_bucket_mass(sh, b) : static_cast<unsigned long long>(n);
-      if (excl + v >= target) {
-        found = b;
-        f_above = excl;
-        f_cnt = cexcl;
-        break;
-      }
-      excl += v;
-      cexcl += static_cast<int>(n);
-    }
-  }
-  const uint32_t hit = __ballot_sync(0xffffffffu, found < kSelBuckets);
-  const int src = hit ? __ffs(hit) - 1 : 31;
-  above = __shfl_sync(0xffffffffu, f_above, src);
-  cnt_above = __shfl_sync(0xffffffffu, f_cnt, src);
-  return hit ? __shfl_sync(0xffffffffu, found, src) : kSelBuckets - 1;
-}
-
-__device__ void select_row_hist(const Geo& g, const RouteOpts& o, const float* lrow, int nB, int words, int qb,
-                                float p, int k_floor, uint32_t* mrow, int32_t* cnt_out, int lane,
-                                const SelScratch& sh) {
-  // the row's words * 32 logits into shared memory in one round trip (16-byte cp.async,
-  // all in flight), then each lane turns its column into order keys
-  {
-    const uint32_t dst = smem_u32(sh.key);
-    const int chunks = words * 8;            // 16-byte chunks of the row
-    for (int q = lane; q < chunks; q += 32) cp_async16(dst + q * 16, lrow + q * 4, 16u);
-    cp_async_commit();
-    cp_async_wait<0>();
-    __syncwarp();
-  }
-  uint32_t* key = sh.key + lane;   // this lane's column: key[c * 32]
-  float mx = -INFINITY;
-#pragma unroll 4
-  for (int c = 0; c < words; ++c) {
-    const int i = c * 32 + lane;
-    const float x = i < nB ? __uint_as_float(key[c * 32]) : -INFINITY;
-    key[c * 32] = i < nB ? order_key(x) : 0u;
-    mx = fmaxf(mx, x);
-  }
-  mx = warp_max(mx);
-  const float nmx = -mx;
-  // a block's mass in 2^-32 units: 2^((x - max) log2 e), times its real token count for
-  // the Top-p over tokens; the same rounded operations wherever it is evaluated
-  auto mass_of = [&](int c, float x) -> unsigned long long {
-    float w = ex2(__fmul_rn(__fadd_rn(x, nmx), 1.4426950408889634f));
-    if (o.token_mass) w *= static_cast<float>(block_info(g, c * 32 + lane).nvalid);
-    return sel_fixed(w);
-  };
-  // Histogram of the blocks of level-0 bucket in0 (all blocks when in0 < 0): 32-bit
-  // shared-memory atomics per block (a mass w < 2^40 goes in as w >> 20 and w & 0xfffff,
-  // so over at most 2^11 blocks the sums stay below 2^31), except for the last bucket
-  // (the tail, where the blocks of a sparse row pile up), which each lane sums in
-  // registers and one lane stores.  Returns the row's (or bucket's) mass.
-  auto histogram = [&](int in0) -> unsigned long long {
-#pragma unroll 4
-    for (int e = lane; e < kSelBuckets; e += 32) {
-      sh.hh[e] = 0u;
-      sh.hl[e] = 0u;
-      sh.hc[e] = 0u;
-    }
-    __syncwarp();
-    unsigned long long z = 0, tail_w = 0;
-    uint32_t tail_c = 0;
-#pragma unroll 2
-    for (int c = 0; c < words; ++c) {
-      const uint32_t k = key[c * 32];
-      if (k != 0u) {
-        const float x = key_value(k);
-        const float t = sel_t(mx, x);
-        const int b0 = sel_b0(t);
-        const int b = in0 < 0 ? b0 : (b0 == in0 ? sel_b1(t, b0) : -1);
-        if (b >= 0) {
-          const unsigned long long w = mass_of(c, x);
-          z += w;
-          if (b == kSelBuckets - 1) {
-            tail_w += w;
-            ++tail_c;
-          } else {
-            atomicAdd(&sh.hh[b], static_cast<uint32_t>(w >> 20));
-            atomicAdd(&sh.hl[b], static_cast<uint32_t>(w & 0xfffffu));
-            atomicAdd(&sh.hc[b], 1u);
-          }
-        }
-      }
-    }
-    tail_w = warp_sum_u64(tail_w);
-    tail_c = static_cast<uint32_t>(warp_sum_i(static_cast<int>(tail_c)));
-    __syncwarp();
-    if (lane == 0) {
-      sh.hh[kSelBuckets - 1] = static_cast<uint32_t>(tail_w >> 20);
-      sh.hl[kSelBuckets - 1] = static_cast<uint32_t>(tail_w & 0xfffffu);
-      sh.hc[kSelBuckets - 1] = tail_c;
-    }
-    __syncwarp();
-    return warp_sum_u64(z);
-  };
-  // Gathers the n <= 32 blocks of level-0 bucket b0 (and level-1 bucket b1 >= 0).
-  auto gather = [&](int b0, int b1) {
-    int base = 0;
-#pragma unroll 2
-    for (int c = 0; c < words; ++c) {
-      const uint32_t k = key[c * 32];
-      bool in = false;
-      float x = 0.f;
-      if (k != 0u) {
-        x = key_value(k);
-        const float t = sel_t(mx, x);
-        const int c0 = sel_b0(t);
-        in = c0 == b0 && (b1 < 0 || sel_b1(t, c0) == b1);
-      }
-      const uint32_t bal = __ballot_sync(0xffffffffu, in);
-      if (in) {
-        const int pos = base + __popc(bal & ((1u << lane) - 1u));
-        sh.lkey[pos] = k;
-        sh.lidx[pos] = static_cast<uint32_t>(c * 32 + lane);
-        sh.lw[pos] = mass_of(c, x);
-      }
-      base += __popc(bal);
-    }
-    __syncwarp();
-  };
-  // Among the n <= 32 gathered blocks (lane j holds block j), the one of smallest rank
-  // (key desc, index asc) at which above + (running sum of weights up to it) >= target;
-  // weight = mass or 1.
-  auto resolve = [&](int n, bool by_mass, unsigned long long above, unsigned long long target, int& rank_out,
-                     uint32_t& key_out, int& idx_out) {
-    int best = 0x7fffffff;
-    if (lane < n) {
-      const uint32_t kj = sh.lkey[lane], ij = sh.lidx[lane];
-      int rank = 0;
-      unsigned long long pre = 0;
-      for (int t = 0; t < n; ++t) {
-        const uint32_t kt = sh.lkey[t], it = sh.lidx[t];
-        const bool before = kt > kj || (kt == kj && it <= ij);
-        rank += (before && t != lane) ? 1 : 0;
-        pre += before ? (by_mass ? sh.lw[t] : 1ull) : 0ull;
-      }
-      // a block whose prefix reaches the target codes as its rank; the others code above
-      // every such rank, the last in the order lowest (the whole bucket)
-      best = above + pre >= target ? rank * 64 + lane : (2 * n - 1 - rank) * 64 + lane;
-    }
-#pragma unroll
-    for (int off = 16; off > 0; off >>= 1) best = min(best, __shfl_xor_sync(0xffffffffu, best, off));
-    const int j = best & 63;
-    rank_out = best >> 6;
-    key_out = sh.lkey[j];
-    idx_out = static_cast<int>(sh.lidx[j]);
-    __syncwarp();
-  };
-  // Exact fallback for a bucket of more than 32 near-tied blocks: a bitwise search for the
-  // cut's key over the whole row (u = the largest key whose prefix of keys >= u reaches the
-  // target), then tied keys in index order.
-  auto search = [&](bool by_mass, unsigned long long target, int& m_out, uint32_t& ucut, int& icut) {
-    uint32_t u = 0;
-#pragma unroll 1
-    for (int bit = 31; bit >= 0; --bit) {
-      const uint32_t cand = u | (1u << bit);
-      unsigned long long m = 0;
-#pragma unroll 1
-      for (int c = 0; c < words; ++c) {
-        const uint32_t k = key[c * 32];
-        if (k != 0u && k >= cand) m += by_mass ? mass_of(c, key_value(k)) : 1ull;
-      }
-      if (warp_sum_u64(m) >= target) u = cand;
-    }
-    unsigned long long acc = 0;
-    int gt = 0;
-#pragma unroll 1
-    for (int c = 0; c < words; ++c) {
-      const uint32_t k = key[c * 32];
-      if (k != 0u && k > u) {
-        acc += by_mass ? mass_of(c, key_value(k)) : 1ull;
-        ++gt;
-      }
-    }
-    acc = warp_sum_u64(acc);
-    gt = warp_sum_i(gt);
-    int r = 0, last = -1;
-#pragma unroll 1
-    for (int c = 0; c < words && acc < target; ++c) {
-      const uint32_t k = key[c * 32];
-      uint32_t tb = __ballot_sync(0xffffffffu, k != 0u && k == u);
-      while (tb != 0u && acc < target) {
-        const int l = __ffs(tb) - 1;
-        tb &= tb - 1u;
-        const unsigned long long w = by_mass ? mass_of(c, key_value(u)) : 1ull;
-        acc += __shfl_sync(0xffffffffu, w, l);
-        ++r;
-        last = c * 32 + l;
-      }
-    }
-    m_out = gt + r;
-    ucut = u;
-    icut = last;
-  };
-  // The cut: the block of the order at which the running sum reaches target (the level-0
-  // histogram is in place).
-  auto cut = [&](bool by_mass, unsigned long long target, int& m_out, uint32_t& ucut, int& icut) {
-    unsigned long long above;
-    int cnt_above;
-    const int b0 = sel_find_bucket(sh, by_mass, target, above, cnt_above, lane);
-    int b1 = -1;
-    int n = static_cast<int>(sh.hc[b0]);
-    if (n > kSelCap) {
-      histogram(b0);
-      unsigned long long above1;
-      int cnt1;
-      b1 = sel_find_bucket(sh, by_mass, target - above, above1, cnt1, lane);
-      above += above1;
-      cnt_above += cnt1;
-      n = static_cast<int>(sh.hc[b1]);
-      if (n > kSelCap) {
-        search(by_mass, target, m_out, ucut, icut);
-        return;
-      }
-    }
-    gather(b0, b1);
-    int rank;
-    resolve(n, by_mass, above, target, rank, ucut, icut);
-    m_out = cnt_above + rank + 1;
-  };
-
-  const unsigned long long z = histogram(-1);
-  const int floor_k = min(max(k_floor, 0), nB);
-  int m_p = nB;
-  uint32_t ucut = 0u;        // blocks with key > ucut, and key == ucut up to index icut, are kept
-  int icut = -1;
-  bool all = true;
-  if (p < 1.f) {
-    // at least one unit, so that p = 0 still keeps the first block of the order
-    const unsigned long long target =
-        max(1ull, static_cast<unsigned long long>(ceil(static_cast<double>(p) * static_cast<double>(z))));
-    cut(true, target, m_p, ucut, icut);
-    all = false;
-  }
-  const int M = max(max(m_p, floor_k), 1);
-  if (M >= nB) {
-    all = true;
-  } else if (M > m_p) {
-    histogram(-1);           // the cut may have left a finer histogram in place
-    int m;
-    cut(false, static_cast<unsigned long long>(M), m, ucut, icut);
-    all = false;
-  }
-  int cnt = 0;
-#pragma unroll 2
-  for (int c = 0; c < words; ++c) {
-    const int i = c * 32 + lane;
-    const uint32_t k = key[c * 32];
-    const bool kept = k != 0u && (all || k > ucut || (k == ucut && i <= icut) || i == qb ||
-                                  keyframe_block(g, o, i));
-    const uint32_t word = __ballot_sync(0xffffffffu, kept);
-    cnt += __popc(word);
-    if (lane == 0) mrow[c] = word;
-  }
-  if (lane == 0) *cnt_out = cnt;
-}
 
 constexpr int kRouteKT = 128;          // key blocks per staged tile
 constexpr int kRouteDC = 32;           // channels per staged tile
@@ -828,6 +917,7 @@ cudaError_t launch_route(const Geo& g, const float* qp, const float* kp, float p
 // the tensor cores (fv_route_tc.cu); then one warp per query block selects from its row
 // by mass histogram (select_row_hist).
 // ----------------------------------------------------------------------------
+template <bool TOKEN>
 __global__ void __launch_bounds__(32 * kSelWarps) select_hist_kernel(Geo g, RouteOpts o,
                                                                      const float* __restrict__ logits, float p,
                                                                      int k_floor, uint32_t* __restrict__ mask,
@@ -838,9 +928,9 @@ __global__ void __launch_bounds__(32 * kSelWarps) select_hist_kernel(Geo g, Rout
   const long long row = static_cast<long long>(blockIdx.x) * kSelWarps + warp;   // (b*h) * nB + qb
   if (row >= static_cast<long long>(g.B) * g.H * nB) return;
   const int qb = static_cast<int>(row % nB);
-  const SelScratch sh = sel_scratch(sel_smem + warp * sel_warp_bytes(g.words));
-  select_row_hist(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
-                  mask + static_cast<size_t>(row) * g.words, counts + row, lane, sh);
+  const SelSmem sh = sel_smem_at(sel_smem + warp * sel_warp_bytes(g.words));
+  select_row_hist<TOKEN>(g, o, logits + static_cast<size_t>(row) * nBpad, nB, g.words, qb, p, k_floor,
+                         mask + static_cast<size_t>(row) * g.words, counts + row, lane, sh);
 }
 
 // For rows of at most kHistMinWords mask words the route is the fp32 pair: logits_kernel
@@ -952,11 +1042,18 @@ static cudaError_t launch_select(const Geo& g, const RouteOpts& o, const float* 
     return cudaGetLastError();
   }
   const int smem = static_cast<int>(kSelWarps * sel_warp_bytes(g.words));
-  static SmemAttrCache sel_attr = {};
-  cudaError_t e = set_smem_once(reinterpret_cast<const void*>(select_hist_kernel), smem, sel_attr);
+  static SmemAttrCache sel_attr[2] = {};
+  const void* fn = o.token_mass ? reinterpret_cast<const void*>(select_hist_kernel<true>)
+                                : reinterpret_cast<const void*>(select_hist_kernel<false>);
+  // the largest carveout (all of the unified L1 / shared array as shared memory): four
+  // CTAs (16 rows) per SM fit at the longest rows (2 048 blocks) only with it
+  cudaError_t e = set_smem_once(fn, smem, sel_attr[o.token_mass ? 1 : 0], 100);
   if (e != cudaSuccess) return e;
-  select_hist_kernel<<<static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps), 32 * kSelWarps, smem, st>>>(
-      g, o, logits, p, k_floor, mask, counts);
+  const unsigned grid = static_cast<unsigned>((rows + kSelWarps - 1) / kSelWarps);
+  if (o.token_mass)
+    select_hist_kernel<true><<<grid, 32 * kSelWarps, smem, st>>>(g, o, logits, p, k_floor, mask, counts);
+  else
+    select_hist_kernel<false><<<grid, 32 * kSelWarps, smem, st>>>(g, o, logits, p, k_floor, mask, counts);
   return cudaGetLastError();
 }
 
@@ -972,18 +1069,19 @@ size_t route_logits_bytes(const Geo& g) {
 // B*H*nB*d floats) for the tensor-core logits.
 size_t route_ws_bytes(const Geo& g) { return kRouteHdr + route_logits_bytes(g) + logits_split_bytes(g); }
 
-cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
-                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st,
-                            const RouteOpts& o) {
-  uint32_t* hdr = static_cast<uint32_t*>(ws);
-  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kRouteHdr);
-  cudaError_t e = cudaMemsetAsync(hdr, 0, kRouteHdr, st);
+static cudaError_t num_sms(int& nsm) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
   if (e != cudaSuccess) return e;
-  int dev = 0, nsm = 0;
-  e = cudaGetDevice(&dev);
-  if (e != cudaSuccess) return e;
-  e = cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
-  if (e != cudaSuccess) return e;
+  return cudaDeviceGetAttribute(&nsm, cudaDevAttrMultiProcessorCount, dev);
+}
+
+// Logits of geometry g into `logits` (its rows padded to words * 32), then the selection.
+// split: the tensor-core path's scratch (logits_split_bytes(g)); err: its status word.
+static cudaError_t route_parts(const Geo& g, const float* qp, const float* kp, float p, int k_floor, float scale,
+                               uint32_t* mask, int32_t* counts, float* logits, float* split, uint32_t* err,
+                               int nsm, cudaStream_t st, const RouteOpts& o) {
+  cudaError_t e;
   if (g.words <= kHistMinWords) {
     const int tiles = (g.nB + kLogitTile - 1) / kLogitTile;
     const int smem = 2 * kLogitTile * (g.d + 4) * 4;
@@ -996,13 +1094,26 @@ cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, floa
     if (g.d == 128) logits_kernel<128><<<grid, 256, smem, st>>>(g, qp, kp, scale, logits);
     else logits_kernel<64><<<grid, 256, smem, st>>>(g, qp, kp, scale, logits);
   } else {
-    float* split = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(logits) + route_logits_bytes(g));
-    e = launch_logits_tc(g, qp, kp, scale, logits, split, hdr + 1, nsm, st);
+    e = launch_logits_tc(g, qp, kp, scale, logits, split, err, nsm, st);
   }
   if (e != cudaSuccess) return e;
   e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   return launch_select(g, o, logits, p, k_floor, mask, counts, st);
+}
+
+cudaError_t launch_route_ws(const Geo& g, const float* qp, const float* kp, float p, int k_floor,
+                            float scale, uint32_t* mask, int32_t* counts, void* ws, cudaStream_t st,
+                            const RouteOpts& o) {
+  uint32_t* hdr = static_cast<uint32_t*>(ws);
+  float* logits = reinterpret_cast<float*>(static_cast<unsigned char*>(ws) + kRouteHdr);
+  float* split = reinterpret_cast<float*>(reinterpret_cast<unsigned char*>(logits) + route_logits_bytes(g));
+  cudaError_t e = cudaMemsetAsync(hdr, 0, kRouteHdr, st);
+  if (e != cudaSuccess) return e;
+  int nsm = 0;
+  e = num_sms(nsm);
+  if (e != cudaSuccess) return e;
+  return route_parts(g, qp, kp, p, k_floor, scale, mask, counts, logits, split, hdr + 1, nsm, st, o);
 }
 
 // ----------------------------------------------------------------------------

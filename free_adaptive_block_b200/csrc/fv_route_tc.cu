@@ -322,8 +322,8 @@ static cudaError_t launch_logits_tc_d(const Geo& g, const float* qp, const float
   cudaError_t e = cudaGetLastError();
   if (e != cudaSuccess) return e;
   const size_t plane = static_cast<size_t>(S) * g.nB * D;
-  // the four maps depend only on the split buffer and the geometry: the last set a thread
-  // encoded is reused while they stay the same
+  // the four maps depend only on the split buffer and the geometry: the last eight sets a
+  // thread encoded are reused while they stay the same (a chunked call uses one per chunk)
   struct MapCache {
     unsigned long long ctx;
     const float* split;
@@ -331,21 +331,32 @@ static cudaError_t launch_logits_tc_d(const Geo& g, const float* qp, const float
     LgMaps maps;
     bool valid;
   };
-  thread_local MapCache mc = {};
+  constexpr int kCached = 8;
+  thread_local MapCache cache[kCached] = {};
+  thread_local int next = 0;
   const unsigned long long ctx = current_ctx_id();
-  if (!(mc.valid && ctx != 0 && mc.ctx == ctx && mc.split == split && mc.S == S && mc.nB == g.nB)) {
-    mc.valid = false;
-    if (!encode_rows_fp32(&mc.maps.qh, split, S, g.nB, D) ||
-        !encode_rows_fp32(&mc.maps.ql, split + plane, S, g.nB, D) ||
-        !encode_rows_fp32(&mc.maps.kh, split + 2 * plane, S, g.nB, D) ||
-        !encode_rows_fp32(&mc.maps.kl, split + 3 * plane, S, g.nB, D))
-      return cudaErrorInvalidValue;
-    mc.ctx = ctx;
-    mc.split = split;
-    mc.S = S;
-    mc.nB = g.nB;
-    mc.valid = true;
+  MapCache* mcp = nullptr;
+  for (int i = 0; i < kCached && mcp == nullptr; ++i) {
+    const MapCache& c = cache[i];
+    if (c.valid && ctx != 0 && c.ctx == ctx && c.split == split && c.S == S && c.nB == g.nB) mcp = &cache[i];
   }
+  if (mcp == nullptr) {
+    MapCache& c = cache[next];
+    next = (next + 1) % kCached;
+    c.valid = false;
+    if (!encode_rows_fp32(&c.maps.qh, split, S, g.nB, D) ||
+        !encode_rows_fp32(&c.maps.ql, split + plane, S, g.nB, D) ||
+        !encode_rows_fp32(&c.maps.kh, split + 2 * plane, S, g.nB, D) ||
+        !encode_rows_fp32(&c.maps.kl, split + 3 * plane, S, g.nB, D))
+      return cudaErrorInvalidValue;
+    c.ctx = ctx;
+    c.split = split;
+    c.S = S;
+    c.nB = g.nB;
+    c.valid = true;
+    mcp = &c;
+  }
+  const MapCache& mc = *mcp;
   LgParams prm;
   prm.g = g;
   prm.logits = logits;
