@@ -38,14 +38,17 @@ from free_adaptive_block_b200 import workloads as W  # noqa: E402
 
 METRIC = "sparse-attn ms/layer + effective TFLOPS (Wan2.1-480p shape), % of bf16 peak"
 
-# DRAM bytes (read + write) of one attention-kernel launch on this workload, from an
-# ncu capture of dram__bytes_read.sum + dram__bytes_write.sum; valid only for the
-# kernel source it was taken from.
-ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "c3520db57f7689b4", "bytes": 389974272}
+# DRAM bytes (read + write) of one attention-kernel launch on the Wan2.1-480p workload,
+# from an ncu capture of dram__bytes_read.sum + dram__bytes_write.sum; valid only for
+# that workload and the kernel source it was taken from.
+ATTN_NCU_TRAFFIC = {"fv_attn.cu sha256[:16]": "c3520db57f7689b4", "bytes": 389974272,
+                    "workload": "wan21_1.3b_480p_h12_21x30x52"}
 
 
-def attn_traffic():
+def attn_traffic(workload: str):
     import hashlib
+    if workload != ATTN_NCU_TRAFFIC["workload"]:
+        return None
     src = os.path.join(ROOT, "free_adaptive_block_b200", "csrc", "fv_attn.cu")
     try:
         h = hashlib.sha256(open(src, "rb").read()).hexdigest()[:16]
@@ -429,7 +432,7 @@ def run_ours(args, rank, world, local_rank, wl=None):
         "sm_busy_max_over_mean": round(float(busy.max() / busy.mean()), 4) if busy.size else None,
         "roofline": {"bound": "tensor", "kernel": "fvattn_block_sparse_attn (prep + attn_kernel)",
                      "achieved": round(attn_tflops_avg, 2), "peak": peaks["bf16"], "unit": "TFLOP/s",
-                     "frac": round(attn_tflops_avg / peaks["bf16"], 4), "traffic": attn_traffic(),
+                     "frac": round(attn_tflops_avg / peaks["bf16"], 4), "traffic": attn_traffic(wl.name),
                      "duration": f"mean of {len(attn_ts)} event-timed calls, {attn_ms_mean:.4f} ms",
                      "peak_source": f"{peaks['source']} bf16 (burst, cuBLAS)"},
         "e2e": {"value": round(whole_job_tflops(eff, world, e2e_ms), 3), "unit": UNIT,

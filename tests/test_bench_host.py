@@ -171,3 +171,14 @@ def test_reference_arm_json_line():
     assert d["e2e"] == {"value": d["value"], "unit": d["unit"], "h2d_bytes_per_step": 0,
                         "d2h_bytes_per_step": 0}
     assert d["config"]["workload"] == "wan21_1.3b_480p_h12_21x30x52"
+
+
+def test_attention_traffic_only_for_its_workload_and_source():
+    bench = load_bench()
+    w480 = bench.W.WAN21_480P.name
+    assert bench.ATTN_NCU_TRAFFIC["workload"] == w480
+    got = bench.attn_traffic(w480)
+    # the recorded bytes when the kernel source is the one they were taken from, else null
+    assert got in (bench.ATTN_NCU_TRAFFIC["bytes"], None)
+    for wl in (bench.W.TINY, bench.W.WAN22_720P, bench.W.WAN21_6X):
+        assert bench.attn_traffic(wl.name) is None
