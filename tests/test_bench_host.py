@@ -182,3 +182,14 @@ def test_attention_traffic_only_for_its_workload_and_source():
     assert got in (bench.ATTN_NCU_TRAFFIC["bytes"], None)
     for wl in (bench.W.TINY, bench.W.WAN22_720P, bench.W.WAN21_6X):
         assert bench.attn_traffic(wl.name) is None
+
+
+def test_e2e_chunks_default_divides_the_slices():
+    bench = load_bench()
+    assert bench.e2e_chunks(0, 12) == 6
+    assert bench.e2e_chunks(0, 40) == 5
+    assert bench.e2e_chunks(0, 2) == 2
+    assert bench.e2e_chunks(0, 7) == 4
+    assert bench.e2e_chunks(0, 1) == 1
+    assert bench.e2e_chunks(8, 12) == 8
+    assert bench.e2e_chunks(16, 12) == 12
