@@ -88,3 +88,17 @@ def test_sweep_lines_world_size_1():
                     "effective_tflops", "frac_of_bf16_peak", "timing"):
             assert key in d, key
         assert d["kept_block_frac"] == 1.0          # the stand-in route keeps every block
+
+
+def test_workload_flag_prints_one_line_for_that_workload():
+    """--workload runs one workload only (the profiler runs use it): one line, named for it,
+    not the headline, and the ncu traffic of the 480p kernel is not reported on it."""
+    r = subprocess.run([sys.executable, HARNESS, "--steps", "3", "--warmup", "3", "--no-cpu-baseline",
+                        "--workload", "tiny_h2_d64_4x8x8"], cwd=ROOT, capture_output=True, text=True, timeout=600)
+    assert r.returncode == 0, r.stderr[-3000:]
+    lines = json_lines(r.stdout)
+    assert len(lines) == 1
+    d = lines[0]
+    assert d["config"]["workload"] == "tiny_h2_d64_4x8x8"
+    assert "not the headline" in d["metric"]
+    assert d["roofline"]["traffic"] is None
