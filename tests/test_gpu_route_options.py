@@ -49,6 +49,19 @@ def test_token_topp(wl, pk):
           int((O.unpack_mask(res["mask"], og.nB) != plain.keep).any(-1).sum()))
 
 
+def test_token_topp_long_rows():
+    """Top-p over tokens on rows of more than 16 mask words (720p: 630 blocks, 20 words),
+    where the workspace route takes the tensor-core logits and the histogram selection
+    with token-weighted masses."""
+    wl = W.WAN22_720P
+    x = W.generate(wl)
+    og = O.block_geometry(wl.T, wl.Hs, wl.Ws, wl.bt, wl.bh, wl.bw)
+    _, res = _route_ex(wl, x, token_mass=1)
+    qp, kp = P.check_pool(wl, x, res, og)
+    st = P.check_route(wl, qp, kp, res, wl.p, wl.k_floor, real_count=og.real_count)
+    print(wl.name, st)
+
+
 @pytest.mark.parametrize("stride,phase", [(20, 0), (20, 7), (13, 5)])
 def test_keyframes_6x(stride, phase):
     import torch
